@@ -1,0 +1,688 @@
+// Attention partials (A, L = log Z) of block query rows over a key set, the
+// split-KV combine, and the FlashBlock log-space merge.
+//
+// One kernel family serves three key sets (FlashBlock technical summary, §2
+// "Core mechanism"; LoSA, §2 step 3):
+//   * the block-external prefix J_out (contiguous or paged cache),
+//   * the block's own tokens J_in (bidirectional, contiguous),
+//   * the union of LoSA-selected pages of a kv head (page list).
+// A CTA owns (sequence b, kv head hk, key split, row tile). Its rows are the
+// block rows taking part times the G q heads sharing hk (GQA stacking), so a
+// K/V tile read from HBM once serves every q head of the group.
+//
+// bf16 path: one producer warp streams K/V tiles of kTK keys with TMA
+// (128-byte swizzle, 3-stage mbarrier pipeline); four consumer warps run
+// QK^T and PV on bf16 tensor cores (mma.sync m16n8k16, fp32 accumulate) with
+// ldmatrix fragment loads and an online softmax in registers (exp2 domain).
+// Consumer warps split the tile's keys (RG row groups x KS key slices) and
+// merge their partial softmax states through shared memory at the end.
+// f32 path: CUDA-core FMA (the fp32 workloads are launch-bound).
+#pragma once
+
+#include "common.cuh"
+
+namespace fb {
+
+constexpr int kTK = 64;      // keys per pipeline stage / tile
+constexpr int kStages = 3;   // TMA pipeline depth
+constexpr int kNWC = 4;      // consumer warps per CTA (bf16)
+constexpr int kAttnThreads = (kNWC + 1) * 32;
+constexpr int kMaxChunks = kTK / 16;  // TMA boxes per tile and half (page >= 16)
+
+struct AttnArgs {
+  const void* q;  // [batch, B, Hq, D]
+  const void* k;  // [n_slots, Hkv, D] (f32 path; the bf16 path reads through TMA)
+  const void* v;
+  int batch, B, Hq, Hkv, G;
+  const int32_t* row_list;  // [batch, n_list] block rows taking part, or NULL (all B)
+  int n_list;
+  int R;  // rows per (b, hk): (row_list ? n_list : B) * G; row r = i_idx * G + g
+  int row_tile, n_row_tiles;
+  // key set
+  const int32_t* page_table;  // [batch, max_pages] or NULL (contiguous)
+  int max_pages, page_size;
+  const int32_t* seq_len;  // [batch] or NULL (all max_seq_len)
+  int max_seq_len;
+  const int32_t* page_list;   // [batch, Hkv, page_list_stride] or NULL (dense key set)
+  const int32_t* page_count;  // [batch, Hkv]
+  int page_list_stride;
+  int chunk;  // tokens per TMA box / metadata chunk: kTK (contiguous dense) or min(page, kTK)
+  long long n_slots;
+  // which heads compute
+  const uint8_t* head_mask;  // [batch, Hq] or NULL
+  unsigned long long seq_bits[4];
+  int use_seq_bits;
+  // split plan
+  int tiles_per_split, n_splits;
+  float scale_log2;  // softmax scale * log2(e)
+  // outputs: split partials (n_splits > 1) or final rows (n_splits == 1)
+  float* o_part;    // [n_splits, batch, Hkv, R, D] normalised partial outputs
+  float* lse_part;  // [n_splits, batch, Hkv, R] log2 normalisers (-inf: empty)
+  float* a_out;     // [batch, B, Hq, D]
+  float* l_out;     // [batch, B, Hq] natural log
+  float* a_prev;    // optional: old a_out rows are copied here before overwrite
+};
+
+__device__ __forceinline__ int seq_tokens(const AttnArgs& a, int b) {
+  return a.seq_len ? a.seq_len[b] : a.max_seq_len;
+}
+
+__device__ __forceinline__ bool cta_selected(const AttnArgs& a, int b, int hk) {
+  if (a.use_seq_bits && !((a.seq_bits[b >> 6] >> (b & 63)) & 1ull)) return false;
+  if (a.head_mask) {
+    for (int g = 0; g < a.G; ++g)
+      if (a.head_mask[b * a.Hq + hk * a.G + g]) return true;
+    return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ bool row_selected(const AttnArgs& a, int b, int h) {
+  if (a.use_seq_bits && !((a.seq_bits[b >> 6] >> (b & 63)) & 1ull)) return false;
+  return a.head_mask == nullptr || a.head_mask[b * a.Hq + h] != 0;
+}
+
+// Number of kTK-key tiles of (b, hk)'s key set.
+__device__ __forceinline__ int n_tiles_of(const AttnArgs& a, int b, int hk) {
+  if (a.page_list) {
+    const int per_tile = kTK / a.page_size;
+    const int cnt = a.page_count[b * a.Hkv + hk];
+    return (cnt + per_tile - 1) / per_tile;
+  }
+  return (seq_tokens(a, b) + kTK - 1) / kTK;
+}
+
+// Slot of the first token of chunk c of tile tl, and how many of the chunk's
+// tokens are valid (0 => the chunk is loaded out of bounds, i.e. zero-filled).
+__device__ __forceinline__ void chunk_slot(const AttnArgs& a, int b, int hk, int tl, int c,
+                                           long long& slot, int& valid) {
+  const int n_tok = seq_tokens(a, b);
+  int t0;
+  if (a.page_list) {
+    const int per_tile = kTK / a.page_size;
+    const int e = tl * per_tile + c;
+    if (e >= a.page_count[b * a.Hkv + hk]) {
+      slot = a.n_slots;
+      valid = 0;
+      return;
+    }
+    const int lp = a.page_list[((long long)b * a.Hkv + hk) * a.page_list_stride + e];
+    t0 = lp * a.page_size;
+  } else {
+    t0 = tl * kTK + c * a.chunk;
+  }
+  valid = min(max(n_tok - t0, 0), a.chunk);
+  if (valid == 0) {
+    slot = a.n_slots;
+    return;
+  }
+  if (a.page_table) {
+    const int lp = t0 / a.page_size;
+    const int off = t0 - lp * a.page_size;
+    slot = (long long)a.page_table[(long long)b * a.max_pages + lp] * a.page_size + off;
+  } else {
+    slot = (long long)b * a.max_seq_len + t0;
+  }
+}
+
+// Maps row r of (b, hk) to the block row i and q head h.
+__device__ __forceinline__ void row_of(const AttnArgs& a, int b, int hk, int r, int& i, int& h) {
+  const int i_idx = r / a.G;
+  h = hk * a.G + (r - i_idx * a.G);
+  i = a.row_list ? a.row_list[b * a.n_list + i_idx] : i_idx;
+}
+
+// Writes one finished row (acc already normalised, lse2 in log2 units).
+template <int NV>
+__device__ __forceinline__ void store_row(const AttnArgs& a, int b, int hk, int split, int r,
+                                          const float (&val)[NV], int col0, int col_stride,
+                                          float lse2, bool lane0) {
+  constexpr int D = NV * 32;  // NV values per lane, 32 lanes
+  (void)D;
+  if (a.n_splits > 1) {
+    const long long pidx = (((long long)split * a.batch + b) * a.Hkv + hk) * a.R + r;
+    float* dst = a.o_part + pidx * (NV * 32);
+#pragma unroll
+    for (int j = 0; j < NV; ++j) dst[col0 + j * col_stride] = val[j];
+    if (lane0) a.lse_part[pidx] = lse2;
+    return;
+  }
+  int i, h;
+  row_of(a, b, hk, r, i, h);
+  if (!row_selected(a, b, h)) return;
+  const long long row = ((long long)b * a.B + i) * a.Hq + h;
+  float* dst = a.a_out + row * (NV * 32);
+  if (a.a_prev) {
+    float* prv = a.a_prev + row * (NV * 32);
+#pragma unroll
+    for (int j = 0; j < NV; ++j) prv[col0 + j * col_stride] = dst[col0 + j * col_stride];
+  }
+#pragma unroll
+  for (int j = 0; j < NV; ++j) dst[col0 + j * col_stride] = val[j];
+  if (lane0) a.l_out[row] = lse2 * kLn2;
+}
+
+// ---------------------------------------------------------------------------
+// bf16 tensor-core kernel
+// ---------------------------------------------------------------------------
+template <int D>
+struct Bf16Smem {
+  static constexpr int kHalves = D / 64;  // 128-byte swizzle rows hold 64 bf16
+  static constexpr int kHalfBytes = kTK * 128;
+  static constexpr int kTileBytes = kHalves * kHalfBytes;  // K or V of one stage
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kRedStride = D + 4;  // padded fp32 row for the cross-warp merge
+  static constexpr int kRedBytes = kNWC * 16 * kRedStride * 4 + 2 * kNWC * 16 * 4;
+  static constexpr int kBytes =
+      (kStages * kStageBytes > kRedBytes ? kStages * kStageBytes : kRedBytes) + 1024;
+  static_assert(kRedBytes <= kStages * kStageBytes, "merge area must fit in the stages");
+};
+
+template <int D, int RG>
+__global__ void __launch_bounds__(kAttnThreads, 2)
+    attn_bf16_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV) {
+  using S = Bf16Smem<D>;
+  constexpr int KS = kNWC / RG;   // key slices
+  constexpr int KW = kTK / KS;    // keys per warp per tile
+  constexpr int SUB = KW < 32 ? KW : 32;
+  constexpr int NT = SUB / 8;     // n8 tiles per sub-chunk
+  constexpr int KD = D / 16;      // k16 steps over the head dim
+
+  __shared__ __align__(8) uint64_t full_bar[kStages];
+  __shared__ __align__(8) uint64_t empty_bar[kStages];
+  __shared__ int meta[kStages][kMaxChunks];
+  __shared__ int meta_full[kStages];
+  __shared__ int abort_flag;
+  extern __shared__ uint8_t dyn_smem[];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rt = blockIdx.x % a.n_row_tiles;
+  const int split = blockIdx.x / a.n_row_tiles;
+  const int hk = blockIdx.y, b = blockIdx.z;
+  if (!cta_selected(a, b, hk)) return;
+
+  const int n_tiles = n_tiles_of(a, b, hk);
+  const int tile0 = split * a.tiles_per_split;
+  const int n_it = max(0, min(a.tiles_per_split, n_tiles - tile0));
+  const int n_chunks = kTK / a.chunk;
+
+  const uint32_t base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+  uint8_t* base_ptr = dyn_smem + (base - smem_u32(dyn_smem));
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kNWC);
+    }
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == kNWC) {
+    // ----------------------------- producer -----------------------------
+    if (lane == 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      int issued = 0;
+      for (int it = 0; it < n_it; ++it) {
+        const int st = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        if (!mbar_wait(&empty_bar[st], ph ^ 1, &abort_flag)) break;
+        long long slots[kMaxChunks];
+        int all_full = 1;
+        for (int c = 0; c < n_chunks; ++c) {
+          int valid;
+          chunk_slot(a, b, hk, tile0 + it, c, slots[c], valid);
+          meta[st][c] = valid;
+          all_full &= (valid == a.chunk);
+        }
+        meta_full[st] = all_full;
+        mbar_arrive_expect_tx(&full_bar[st], S::kStageBytes);
+        uint8_t* sk = base_ptr + st * S::kStageBytes;
+        uint8_t* sv = sk + S::kTileBytes;
+        for (int c = 0; c < n_chunks; ++c) {
+          const int z = (int)slots[c];
+#pragma unroll
+          for (int hf = 0; hf < S::kHalves; ++hf) {
+            uint8_t* dk = sk + hf * S::kHalfBytes + c * a.chunk * 128;
+            uint8_t* dv = sv + hf * S::kHalfBytes + c * a.chunk * 128;
+            tma_load_3d(dk, &tmK, hf * 64, hk, z, &full_bar[st]);
+            tma_load_3d(dv, &tmV, hf * 64, hk, z, &full_bar[st]);
+          }
+        }
+        ++issued;
+      }
+      if (abort_flag) {
+        // let copies already in flight land before the CTA's memory goes away
+        const long long t0 = clock64();
+        for (int it = max(0, issued - kStages); it < issued; ++it) {
+          const int st = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          while (!mbar_try_wait(&full_bar[st], ph) && clock64() - t0 < kWaitBudgetCycles) {
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // ------------------------------ consumers ------------------------------
+  const int rg = warp % RG, ks = warp / RG;
+  const int g8 = lane >> 2, t4 = lane & 3;
+  const int row_base = rt * a.row_tile + rg * 16;
+
+  // Q fragments (A operand of QK^T), rows g8 and g8 + 8 of this row group.
+  uint32_t qa[KD][4];
+  {
+    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q);
+    const __nv_bfloat16* rowp[2] = {nullptr, nullptr};
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int r = row_base + g8 + hr * 8;
+      if (r < a.R) {
+        int i, h;
+        row_of(a, b, hk, r, i, h);
+        rowp[hr] = qb + (((long long)b * a.B + i) * a.Hq + h) * D;
+      }
+    }
+#pragma unroll
+    for (int kk = 0; kk < KD; ++kk) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int hr = j & 1;
+        const int col = kk * 16 + (j >> 1) * 8 + 2 * t4;
+        qa[kk][j] = rowp[hr] ? *reinterpret_cast<const uint32_t*>(rowp[hr] + col) : 0u;
+      }
+    }
+  }
+
+  float o[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float m_r[2] = {-INFINITY, -INFINITY};
+  float l_r[2] = {0.f, 0.f};
+
+  const int mi = lane >> 3, r8 = lane & 7;
+  for (int it = 0; it < n_it; ++it) {
+    const int st = it % kStages;
+    const uint32_t ph = (it / kStages) & 1;
+    if (!mbar_wait(&full_bar[st], ph, &abort_flag)) break;
+    const uint32_t sK = base + st * S::kStageBytes;
+    const uint32_t sV = sK + S::kTileBytes;
+    const bool tile_full = meta_full[st] != 0;
+    const int chunk = a.chunk;
+    bool wrote_smem = false;
+
+#pragma unroll
+    for (int sub = 0; sub < KW / SUB; ++sub) {
+      const int kb = ks * KW + sub * SUB;  // first key of this sub-chunk in the tile
+      float s[NT][4];
+#pragma unroll
+      for (int n = 0; n < NT; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < KD; ++kk) {
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+          const int key = kb + np * 16 + (mi >> 1) * 8 + r8;
+          const int ch = 2 * kk + (mi & 1);
+          const uint32_t addr =
+              sK + (ch >> 3) * S::kHalfBytes + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(addr, b0, b1, b2, b3);
+          mma_bf16(s[2 * np], qa[kk], b0, b1);
+          mma_bf16(s[2 * np + 1], qa[kk], b2, b3);
+        }
+      }
+      // scale into the exp2 domain and mask keys outside the key set
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[n][e] *= a.scale_log2;
+      if (!tile_full) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int key = kb + n * 8 + 2 * t4 + (e & 1);
+            const int c = key / chunk;
+            if (key - c * chunk >= meta[st][c]) s[n][e] = -INFINITY;
+          }
+        // V rows of masked keys may hold any bits: zero them so p = 0 stays 0
+        for (int idx = lane; idx < SUB * (D / 8); idx += 32) {
+          const int kr = idx / (D / 8), ch = idx % (D / 8);
+          const int key = kb + kr;
+          const int c = key / chunk;
+          if (key - c * chunk >= meta[st][c]) {
+            uint8_t* p = base_ptr + (sV - base) + (ch >> 3) * S::kHalfBytes + key * 128 +
+                         (((ch & 7) ^ (key & 7)) << 4);
+            *reinterpret_cast<uint4*>(p) = make_uint4(0u, 0u, 0u, 0u);
+            wrote_smem = true;
+          }
+        }
+        __syncwarp();
+      }
+      // online softmax (rows g8 and g8 + 8)
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        mx[0] = fmaxf(mx[0], fmaxf(s[n][0], s[n][1]));
+        mx[1] = fmaxf(mx[1], fmaxf(s[n][2], s[n][3]));
+      }
+      float alpha[2], bse[2];
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 1));
+        mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 2));
+        const float mn = fmaxf(m_r[hr], mx[hr]);
+        bse[hr] = (mn == -INFINITY) ? 0.f : mn;
+        alpha[hr] = fast_exp2(m_r[hr] - bse[hr]);
+        m_r[hr] = mn;
+      }
+      float rs[2] = {0.f, 0.f};
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          s[n][e] = fast_exp2(s[n][e] - bse[e >> 1]);
+          rs[e >> 1] += s[n][e];
+        }
+      }
+      l_r[0] = l_r[0] * alpha[0] + rs[0];
+      l_r[1] = l_r[1] * alpha[1] + rs[1];
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n) {
+        o[n][0] *= alpha[0];
+        o[n][1] *= alpha[0];
+        o[n][2] *= alpha[1];
+        o[n][3] *= alpha[1];
+      }
+      // O += P V
+#pragma unroll
+      for (int kst = 0; kst < SUB / 16; ++kst) {
+        const uint32_t pa[4] = {pack_bf16(s[2 * kst][0], s[2 * kst][1]),
+                                pack_bf16(s[2 * kst][2], s[2 * kst][3]),
+                                pack_bf16(s[2 * kst + 1][0], s[2 * kst + 1][1]),
+                                pack_bf16(s[2 * kst + 1][2], s[2 * kst + 1][3])};
+#pragma unroll
+        for (int dp = 0; dp < D / 16; ++dp) {
+          const int key = kb + kst * 16 + (mi & 1) * 8 + r8;
+          const int ch = 2 * dp + (mi >> 1);
+          const uint32_t addr =
+              sV + (ch >> 3) * S::kHalfBytes + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(addr, b0, b1, b2, b3);
+          mma_bf16(o[2 * dp], pa, b0, b1);
+          mma_bf16(o[2 * dp + 1], pa, b2, b3);
+        }
+      }
+    }
+    if (wrote_smem) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[st]);
+  }
+
+  // --------------------- cross-warp merge and output ----------------------
+#pragma unroll
+  for (int hr = 0; hr < 2; ++hr) {
+    l_r[hr] += __shfl_xor_sync(0xffffffffu, l_r[hr], 1);
+    l_r[hr] += __shfl_xor_sync(0xffffffffu, l_r[hr], 2);
+  }
+  named_bar_sync(1, kNWC * 32);  // every consumer is done with the stage buffers
+  float* redO = reinterpret_cast<float*>(base_ptr);
+  float* redM = redO + kNWC * 16 * S::kRedStride;
+  float* redL = redM + kNWC * 16;
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) {
+    const int col = n * 8 + 2 * t4;
+    *reinterpret_cast<float2*>(&redO[(warp * 16 + g8) * S::kRedStride + col]) =
+        make_float2(o[n][0], o[n][1]);
+    *reinterpret_cast<float2*>(&redO[(warp * 16 + g8 + 8) * S::kRedStride + col]) =
+        make_float2(o[n][2], o[n][3]);
+  }
+  if (t4 == 0) {
+    redM[warp * 16 + g8] = m_r[0];
+    redM[warp * 16 + g8 + 8] = m_r[1];
+    redL[warp * 16 + g8] = l_r[0];
+    redL[warp * 16 + g8 + 8] = l_r[1];
+  }
+  named_bar_sync(1, kNWC * 32);
+  constexpr int NV = D / 32;
+  for (int rl = warp; rl < RG * 16; rl += kNWC) {
+    const int r = rt * a.row_tile + rl;
+    if (r >= a.R) break;
+    const int rgi = rl >> 4, rr = rl & 15;
+    float M = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < KS; ++k) M = fmaxf(M, redM[(rgi + k * RG) * 16 + rr]);
+    const float bse = (M == -INFINITY) ? 0.f : M;
+    float lsum = 0.f;
+    float acc[NV];
+#pragma unroll
+    for (int j = 0; j < NV; ++j) acc[j] = 0.f;
+#pragma unroll
+    for (int k = 0; k < KS; ++k) {
+      const int wi = rgi + k * RG;
+      const float w = fast_exp2(redM[wi * 16 + rr] - bse);
+      lsum += w * redL[wi * 16 + rr];
+      const float* src = &redO[(wi * 16 + rr) * S::kRedStride + lane * NV];
+#pragma unroll
+      for (int j = 0; j < NV; ++j) acc[j] += w * src[j];
+    }
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) acc[j] *= inv;
+    const float lse2 = lsum > 0.f ? bse + log2f(lsum) : -INFINITY;
+    store_row<NV>(a, b, hk, split, r, acc, lane * NV, 1, lse2, lane == 0);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// fp32 CUDA-core kernel: row tile 16 (4 warps x 4 rows), tiles of kTK keys
+// loaded with plain coalesced loads; lane j of a warp owns key j of a half tile.
+// ---------------------------------------------------------------------------
+constexpr int kF32Rows = 16;
+
+template <int D>
+__global__ void __launch_bounds__(128) attn_f32_kernel(const __grid_constant__ AttnArgs a) {
+  constexpr int NV = D / 32;
+  __shared__ float Ks[32][D + 1];  // half a tile; +1: lanes reading different keys hit different banks
+  __shared__ float Vs[32][D];
+  __shared__ float Qs[kF32Rows][D];
+  __shared__ int meta[kMaxChunks];
+  __shared__ long long slots[kMaxChunks];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rt = blockIdx.x % a.n_row_tiles;
+  const int split = blockIdx.x / a.n_row_tiles;
+  const int hk = blockIdx.y, b = blockIdx.z;
+  if (!cta_selected(a, b, hk)) return;
+  const int n_tiles = n_tiles_of(a, b, hk);
+  const int tile0 = split * a.tiles_per_split;
+  const int n_it = max(0, min(a.tiles_per_split, n_tiles - tile0));
+  const int n_chunks = kTK / a.chunk;
+  const float* qf = static_cast<const float*>(a.q);
+  const float* kg = static_cast<const float*>(a.k);
+  const float* vg = static_cast<const float*>(a.v);
+
+  for (int idx = tid; idx < kF32Rows * D; idx += blockDim.x) {
+    const int rl = idx / D, c = idx % D;
+    const int r = rt * kF32Rows + rl;
+    float v = 0.f;
+    if (r < a.R) {
+      int i, h;
+      row_of(a, b, hk, r, i, h);
+      v = qf[(((long long)b * a.B + i) * a.Hq + h) * D + c];
+    }
+    Qs[rl][c] = v;
+  }
+
+  float m_r[4], l_r[4], o[4][NV];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    m_r[k] = -INFINITY;
+    l_r[k] = 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) o[k][j] = 0.f;
+  }
+
+  for (int it = 0; it < n_it; ++it) {
+    __syncthreads();
+    if (tid < n_chunks) {
+      long long sl;
+      int valid;
+      chunk_slot(a, b, hk, tile0 + it, tid, sl, valid);
+      slots[tid] = sl;
+      meta[tid] = valid;
+    }
+    __syncthreads();
+    for (int half = 0; half < kTK / 32; ++half) {
+      if (half) __syncthreads();
+      for (int idx = tid; idx < 32 * D; idx += blockDim.x) {
+        const int kr = idx / D, c = idx - (idx / D) * D;
+        const int key = half * 32 + kr;
+        const int ci = key / a.chunk, off = key - ci * a.chunk;
+        float kv = 0.f, vv = 0.f;
+        if (off < meta[ci]) {  // keys outside the key set stay 0 (and are masked below)
+          const long long e = ((slots[ci] + off) * a.Hkv + hk) * D + c;
+          kv = kg[e];
+          vv = vg[e];
+        }
+        Ks[kr][c] = kv;
+        Vs[kr][c] = vv;
+      }
+      __syncthreads();
+      const int key = half * 32 + lane;
+      const int ci = key / a.chunk;
+      const bool valid = (key - ci * a.chunk) < meta[ci];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int rl = warp * 4 + k;
+        float s = 0.f;
+#pragma unroll 16
+        for (int c = 0; c < D; ++c) s = fmaf(Qs[rl][c], Ks[lane][c], s);
+        s = valid ? s * a.scale_log2 : -INFINITY;
+        float mx = s;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float mn = fmaxf(m_r[k], mx);
+        const float bse = (mn == -INFINITY) ? 0.f : mn;
+        const float alpha = exp2f(m_r[k] - bse);
+        const float p = exp2f(s - bse);
+        float ps = p;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+        l_r[k] = l_r[k] * alpha + ps;
+        m_r[k] = mn;
+#pragma unroll
+        for (int j = 0; j < NV; ++j) o[k][j] *= alpha;
+        for (int jk = 0; jk < 32; ++jk) {
+          const float pj = __shfl_sync(0xffffffffu, p, jk);
+#pragma unroll
+          for (int j = 0; j < NV; ++j) o[k][j] = fmaf(pj, Vs[jk][lane + 32 * j], o[k][j]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = rt * kF32Rows + warp * 4 + k;
+    if (r >= a.R) break;
+    const float inv = l_r[k] > 0.f ? 1.f / l_r[k] : 0.f;
+    float val[NV];
+#pragma unroll
+    for (int j = 0; j < NV; ++j) val[j] = o[k][j] * inv;
+    const float lse2 = l_r[k] > 0.f ? m_r[k] + log2f(l_r[k]) : -INFINITY;
+    store_row<NV>(a, b, hk, split, r, val, lane, 32, lse2, lane == 0);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Split-KV combine: one warp per row of (b, hk); same log-space rule as the
+// FlashBlock merge, over n_splits partials. Empty partials (lse = -inf) are
+// skipped, so their (never written) outputs are never read.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ AttnArgs a) {
+  constexpr int NV = D / 32;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long rows = (long long)a.batch * a.Hkv * a.R;
+  if (warp >= rows) return;
+  const int r = warp % a.R;
+  const int hk = (warp / a.R) % a.Hkv;
+  const int b = warp / (a.R * a.Hkv);
+  int i, h;
+  row_of(a, b, hk, r, i, h);
+  if (!row_selected(a, b, h)) return;
+  float M = -INFINITY;
+  for (int s = 0; s < a.n_splits; ++s) {
+    const long long pidx = (((long long)s * a.batch + b) * a.Hkv + hk) * a.R + r;
+    M = fmaxf(M, a.lse_part[pidx]);
+  }
+  const float bse = (M == -INFINITY) ? 0.f : M;
+  float acc[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) acc[j] = 0.f;
+  float wsum = 0.f;
+  for (int s = 0; s < a.n_splits; ++s) {
+    const long long pidx = (((long long)s * a.batch + b) * a.Hkv + hk) * a.R + r;
+    const float l = a.lse_part[pidx];
+    if (l == -INFINITY) continue;
+    const float w = fast_exp2(l - bse);
+    wsum += w;
+    const float* src = a.o_part + pidx * D + lane * NV;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) acc[j] += w * src[j];
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  const long long row = ((long long)b * a.B + i) * a.Hq + h;
+  float* dst = a.a_out + row * D + lane * NV;
+  if (a.a_prev) {
+    float* prv = a.a_prev + row * D + lane * NV;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) prv[j] = dst[j];
+  }
+#pragma unroll
+  for (int j = 0; j < NV; ++j) dst[j] = acc[j] * inv;
+  if (lane == 0) a.l_out[row] = wsum > 0.f ? (bse + log2f(wsum)) * kLn2 : -INFINITY;
+}
+
+// ---------------------------------------------------------------------------
+// FlashBlock merge (technical summary §2, merge equation), one warp per row:
+//   m = max(L_out, L_in), w_x = e^{L_x - m},
+//   A_full = (w_out A_out + w_in A_in) / (w_out + w_in), L_full = m + log(w_out + w_in)
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256)
+    merge_kernel(const float* __restrict__ a_out, const float* __restrict__ l_out,
+                 const float* __restrict__ a_in, const float* __restrict__ l_in, long long rows,
+                 float* __restrict__ a_full, float* __restrict__ l_full) {
+  constexpr int NV = D / 32;
+  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  const float lo = l_out[warp], li = l_in[warp];
+  const float m = fmaxf(lo, li);
+  float wo = 0.f, wi = 0.f, den = 1.f, L = -INFINITY;
+  if (m != -INFINITY) {
+    wo = expf(lo - m);
+    wi = expf(li - m);
+    den = wo + wi;
+    L = m + logf(den);
+  }
+  const float inv = 1.f / den;
+  const float* so = a_out + warp * D + lane * NV;
+  const float* si = a_in + warp * D + lane * NV;
+  float* dst = a_full + warp * D + lane * NV;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    // a side whose weight is 0 is not read (it may hold stale bits)
+    const float x = (wo > 0.f ? wo * so[j] : 0.f) + (wi > 0.f ? wi * si[j] : 0.f);
+    dst[j] = x * inv;
+  }
+  if (l_full && lane == 0) l_full[warp] = L;
+}
+
+}  // namespace fb

@@ -1,0 +1,724 @@
+// C ABI of the block-diffusion attention library (declared in include/fb.h):
+// argument validation, split-KV planning, TMA descriptor creation and kernel
+// launches. Every step of the path runs in the kernels of attn.cuh, losa.cuh
+// and cosine.cuh; this file only decides what to launch.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/fb.h"
+#include "attn.cuh"
+#include "cosine.cuh"
+#include "losa.cuh"
+
+namespace {
+
+using namespace fb;
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FB_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return FB_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int next_pow2(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+size_t elem_size(fb_dtype t) { return t == FB_BF16 ? 2 : 4; }
+
+// --------------------------------------------------------------------------
+// Split-KV plan: row tiles per (b, hk), and how many kTK-key tiles each CTA
+// streams, chosen so that the grid covers the GPU for about four waves at two
+// resident CTAs per SM.
+// --------------------------------------------------------------------------
+struct Plan {
+  int row_tile, n_row_tiles, rg;
+  int tiles_per_split, n_splits;
+};
+
+Plan make_plan(fb_dtype dt, int batch, int Hkv, int R, int max_tiles, int num_sms) {
+  Plan p{};
+  if (dt == FB_F32) {
+    p.row_tile = kF32Rows;
+    p.rg = 1;
+  } else {
+    p.rg = R <= 16 ? 1 : (R <= 32 ? 2 : 4);
+    p.row_tile = 16 * p.rg;
+  }
+  p.n_row_tiles = ceil_div(R, p.row_tile);
+  const long long units = (long long)batch * Hkv * p.n_row_tiles;
+  const long long target = (long long)(num_sms > 0 ? num_sms : 148) * 2 * 4;
+  max_tiles = max_tiles < 1 ? 1 : max_tiles;
+  long long splits = (target + units - 1) / units;
+  if (splits < 1) splits = 1;
+  if (splits > max_tiles) splits = max_tiles;
+  p.tiles_per_split = ceil_div(max_tiles, splits);
+  p.n_splits = ceil_div(max_tiles, p.tiles_per_split);
+  return p;
+}
+
+size_t partial_bytes(const Plan& p, int batch, int Hkv, int R, int D) {
+  if (p.n_splits <= 1) return 0;
+  const size_t rows = (size_t)p.n_splits * batch * Hkv * R;
+  return round_up(rows * D * 4, 256) + round_up(rows * 4, 256);
+}
+
+// Workspace regions shared by every entry point (offsets in bytes).
+struct WsLayout {
+  size_t part, scores, cos, a_in, l_in, total;
+};
+
+int logical_pages(const fb_kv* kv) {
+  return kv->page_table ? kv->max_pages_per_seq : ceil_div(kv->max_seq_len, kv->page_size);
+}
+
+int max_union_entries(const fb_kv* kv, int G, int n_active, int topk) {
+  const long long u = (long long)n_active * G * topk;
+  const int np = logical_pages(kv);
+  return (int)(u < np ? u : np);
+}
+
+WsLayout ws_layout(const fb_kv* kv, int B, int Hq, int n_active, int topk, int num_sms) {
+  WsLayout w{};
+  const int G = Hq / kv->n_heads_kv, D = kv->head_dim;
+  const int R = B * G;
+  const Plan pd = make_plan(kv->dtype, kv->batch, kv->n_heads_kv, R, ceil_div(kv->max_seq_len, kTK),
+                            num_sms);
+  size_t part = partial_bytes(pd, kv->batch, kv->n_heads_kv, R, D);
+  size_t scores = 0;
+  if (n_active > 0 && topk > 0) {
+    const int na = n_active < B ? n_active : B;
+    const int per_tile = kTK / (kv->page_size < kTK ? kv->page_size : kTK);
+    const int ent = max_union_entries(kv, G, na, topk);
+    const Plan pg = make_plan(kv->dtype, kv->batch, kv->n_heads_kv, na * G, ceil_div(ent, per_tile),
+                              num_sms);
+    const size_t pgb = partial_bytes(pg, kv->batch, kv->n_heads_kv, na * G, D);
+    part = part > pgb ? part : pgb;
+    scores = round_up((size_t)kv->batch * na * Hq * logical_pages(kv) * 4, 256) +
+             round_up((size_t)kv->batch * B * 4, 256);
+  }
+  const int P = next_pow2(B * D);
+  const int T1 = P < kCosT1Max ? P : kCosT1Max;
+  const size_t cosb = round_up((size_t)kv->batch * Hq * 3 * T1 * 8, 256);
+  w.part = 0;
+  w.scores = w.part + part;
+  w.cos = w.scores + scores;
+  w.a_in = w.cos + cosb;
+  w.l_in = w.a_in + round_up((size_t)kv->batch * B * Hq * D * 4, 256);
+  w.total = w.l_in + round_up((size_t)kv->batch * B * Hq * 4, 256);
+  return w;
+}
+
+// --------------------------------------------------------------------------
+// TMA descriptors for the K / V pools: 3-D view [n_slots][Hkv][D] bf16, boxes
+// of 64 channels (128 bytes, swizzled) x 1 head x `chunk` tokens.
+// --------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+int make_tmap(CUtensorMap* m, const void* base, int D, int Hkv, long long n_slots, int chunk) {
+  auto fn = encode_fn();
+  if (!fn) return fail(FB_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)n_slots};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)chunk};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FB_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return FB_OK;
+}
+
+int validate_kv(const fb_kv* kv) {
+  if (!kv) return fail(FB_ERR_ARG, "kv is NULL");
+  if (!kv->k || !kv->v) return fail(FB_ERR_ARG, "kv->k / kv->v is NULL");
+  if (kv->batch <= 0 || kv->batch > 256) return fail(FB_ERR_ARG, "batch must be in [1, 256]");
+  if (kv->n_heads_kv <= 0 || kv->max_seq_len < 0 || kv->n_slots <= 0)
+    return fail(FB_ERR_ARG, "bad kv sizes");
+  if (kv->n_slots >= (1LL << 31)) return fail(FB_ERR_SHAPE, "n_slots must be < 2^31");
+  if (kv->head_dim != 64 && kv->head_dim != 128)
+    return fail(FB_ERR_SHAPE, "head_dim %d unsupported (64, 128)", kv->head_dim);
+  if (kv->dtype != FB_BF16 && kv->dtype != FB_F32) return fail(FB_ERR_ARG, "bad dtype");
+  if (!pow2(kv->page_size) || kv->page_size < 16)
+    return fail(FB_ERR_SHAPE, "page_size must be a power of two >= 16");
+  if (kv->page_table && kv->max_pages_per_seq * (long long)kv->page_size < kv->max_seq_len)
+    return fail(FB_ERR_ARG, "max_pages_per_seq * page_size < max_seq_len");
+  if (!kv->page_table && (long long)kv->batch * kv->max_seq_len > kv->n_slots)
+    return fail(FB_ERR_ARG, "contiguous cache needs batch * max_seq_len <= n_slots");
+  if (!aligned16(kv->k) || !aligned16(kv->v)) return fail(FB_ERR_ALIGN, "k / v not 16-byte aligned");
+  return FB_OK;
+}
+
+// Shared launcher of the attention partial (prefix, block, or LoSA gather).
+struct PartialCall {
+  const void* q;
+  int B, Hq;
+  float scale;
+  const fb_kv* kv;
+  const int32_t* row_list;
+  int n_list;
+  const int32_t* page_list;
+  const int32_t* page_count;
+  int page_list_stride, max_list_entries;
+  const uint8_t* head_mask;
+  const unsigned long long* seq_bits;  // 4 words or NULL
+  float* a_out;
+  float* l_out;
+  float* a_prev;
+  void* ws;
+  size_t ws_bytes;
+  size_t ws_offset;
+  int num_sms;
+  bool single_split;  // one CTA streams the whole key set (no workspace)
+};
+
+int launch_partial(const PartialCall& c, cudaStream_t stream) {
+  const fb_kv* kv = c.kv;
+  const int D = kv->head_dim, Hkv = kv->n_heads_kv, G = c.Hq / Hkv;
+  AttnArgs a{};
+  a.q = c.q;
+  a.k = kv->k;
+  a.v = kv->v;
+  a.batch = kv->batch;
+  a.B = c.B;
+  a.Hq = c.Hq;
+  a.Hkv = Hkv;
+  a.G = G;
+  a.row_list = c.row_list;
+  a.n_list = c.n_list;
+  a.R = (c.row_list ? c.n_list : c.B) * G;
+  a.page_table = kv->page_table;
+  a.max_pages = kv->max_pages_per_seq;
+  a.page_size = kv->page_size;
+  a.seq_len = kv->seq_len;
+  a.max_seq_len = kv->max_seq_len;
+  a.page_list = c.page_list;
+  a.page_count = c.page_count;
+  a.page_list_stride = c.page_list_stride;
+  a.n_slots = kv->n_slots;
+  a.head_mask = c.head_mask;
+  if (c.seq_bits) {
+    a.use_seq_bits = 1;
+    for (int i = 0; i < 4; ++i) a.seq_bits[i] = c.seq_bits[i];
+  }
+  a.scale_log2 = c.scale * kLog2e;
+  a.a_out = c.a_out;
+  a.l_out = c.l_out;
+  a.a_prev = c.a_prev;
+  if (a.R == 0) return FB_OK;
+  int max_tiles;
+  if (c.page_list) {
+    if (kv->page_size > kTK) return fail(FB_ERR_SHAPE, "page-list attention needs page_size <= 64");
+    a.chunk = kv->page_size;
+    max_tiles = ceil_div(c.max_list_entries, kTK / kv->page_size);
+  } else {
+    a.chunk = kv->page_table ? (kv->page_size < kTK ? kv->page_size : kTK) : kTK;
+    max_tiles = ceil_div(kv->max_seq_len, kTK);
+  }
+  Plan p = make_plan(kv->dtype, kv->batch, Hkv, a.R, max_tiles, c.num_sms);
+  if (c.single_split) {
+    p.tiles_per_split = max_tiles < 1 ? 1 : max_tiles;
+    p.n_splits = 1;
+  }
+  a.row_tile = p.row_tile;
+  a.n_row_tiles = p.n_row_tiles;
+  a.tiles_per_split = p.tiles_per_split;
+  a.n_splits = p.n_splits;
+  const size_t need = partial_bytes(p, kv->batch, Hkv, a.R, D);
+  if (need > 0) {
+    if (!c.ws || c.ws_offset + need > c.ws_bytes)
+      return fail(FB_ERR_WORKSPACE, "workspace too small: need %zu bytes at offset %zu, have %zu",
+                  need, c.ws_offset, c.ws_bytes);
+    if (!aligned16(c.ws)) return fail(FB_ERR_ALIGN, "workspace not 16-byte aligned");
+    const size_t rows = (size_t)p.n_splits * kv->batch * Hkv * a.R;
+    a.o_part = reinterpret_cast<float*>(static_cast<char*>(c.ws) + c.ws_offset);
+    a.lse_part = reinterpret_cast<float*>(static_cast<char*>(c.ws) + c.ws_offset +
+                                          round_up(rows * D * 4, 256));
+  }
+  const dim3 grid(p.n_row_tiles * p.n_splits, Hkv, kv->batch);
+  if (kv->dtype == FB_F32) {
+    if (D == 128)
+      attn_f32_kernel<128><<<grid, 128, 0, stream>>>(a);
+    else
+      attn_f32_kernel<64><<<grid, 128, 0, stream>>>(a);
+  } else {
+    CUtensorMap tk, tv;
+    int rc = make_tmap(&tk, kv->k, D, Hkv, kv->n_slots, a.chunk);
+    if (rc) return rc;
+    rc = make_tmap(&tv, kv->v, D, Hkv, kv->n_slots, a.chunk);
+    if (rc) return rc;
+#define FB_LAUNCH_BF16(DD, RGV)                                                              \
+  do {                                                                                       \
+    auto kfn = attn_bf16_kernel<DD, RGV>;                                                    \
+    const int smem = Bf16Smem<DD>::kBytes;                                                   \
+    static bool attr_set = false;                                                            \
+    if (!attr_set) {                                                                         \
+      cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);          \
+      attr_set = true;                                                                       \
+    }                                                                                        \
+    kfn<<<grid, kAttnThreads, smem, stream>>>(a, tk, tv);                                    \
+  } while (0)
+    if (D == 128) {
+      if (p.rg == 1)
+        FB_LAUNCH_BF16(128, 1);
+      else if (p.rg == 2)
+        FB_LAUNCH_BF16(128, 2);
+      else
+        FB_LAUNCH_BF16(128, 4);
+    } else {
+      if (p.rg == 1)
+        FB_LAUNCH_BF16(64, 1);
+      else if (p.rg == 2)
+        FB_LAUNCH_BF16(64, 2);
+      else
+        FB_LAUNCH_BF16(64, 4);
+    }
+#undef FB_LAUNCH_BF16
+  }
+  int rc = check_launch("attention partial kernel");
+  if (rc) return rc;
+  if (p.n_splits > 1) {
+    const long long rows = (long long)kv->batch * Hkv * a.R;
+    const int blocks = ceil_div(rows * 32, 256);
+    if (D == 128)
+      combine_kernel<128><<<blocks, 256, 0, stream>>>(a);
+    else
+      combine_kernel<64><<<blocks, 256, 0, stream>>>(a);
+    rc = check_launch("split combine kernel");
+  }
+  return rc;
+}
+
+int validate_q(const void* q, int B, int Hq, const fb_kv* kv) {
+  if (!q) return fail(FB_ERR_ARG, "q is NULL");
+  if (B <= 0 || Hq <= 0) return fail(FB_ERR_ARG, "B and n_heads_q must be positive");
+  if (Hq % kv->n_heads_kv) return fail(FB_ERR_SHAPE, "n_heads_q %% n_heads_kv != 0");
+  if (!aligned16(q)) return fail(FB_ERR_ALIGN, "q not 16-byte aligned");
+  return FB_OK;
+}
+
+int merge_launch(const float* ao, const float* lo, const float* ai, const float* li, long long rows,
+                 int D, float* af, float* lf, cudaStream_t stream) {
+  if (rows == 0) return FB_OK;
+  const int blocks = ceil_div(rows * 32, 256);
+  if (D == 128)
+    merge_kernel<128><<<blocks, 256, 0, stream>>>(ao, lo, ai, li, rows, af, lf);
+  else
+    merge_kernel<64><<<blocks, 256, 0, stream>>>(ao, lo, ai, li, rows, af, lf);
+  return check_launch("merge kernel");
+}
+
+KvView kv_view(const fb_kv* kv) {
+  KvView v{};
+  v.k = kv->k;
+  v.page_table = kv->page_table;
+  v.seq_len = kv->seq_len;
+  v.batch = kv->batch;
+  v.Hkv = kv->n_heads_kv;
+  v.D = kv->head_dim;
+  v.page_size = kv->page_size;
+  v.max_pages = kv->page_table ? kv->max_pages_per_seq : ceil_div(kv->max_seq_len, kv->page_size);
+  v.max_seq_len = kv->max_seq_len;
+  return v;
+}
+
+int block_attn_impl(const void* q, const void* k_in, const void* v_in, int batch, int B, int Hq,
+                    int Hkv, int D, float scale, fb_dtype dt, float* a_in, float* l_in,
+                    cudaStream_t stream) {
+  fb_kv kv{};
+  kv.k = k_in;
+  kv.v = v_in;
+  kv.n_slots = (long long)batch * B;
+  kv.batch = batch;
+  kv.n_heads_kv = Hkv;
+  kv.head_dim = D;
+  kv.page_size = 16;
+  kv.max_seq_len = B;
+  kv.dtype = dt;
+  int rc = validate_kv(&kv);
+  if (rc) return rc;
+  rc = validate_q(q, B, Hq, &kv);
+  if (rc) return rc;
+  if (!a_in || !l_in) return fail(FB_ERR_ARG, "a_in / l_in is NULL");
+  PartialCall c{};
+  c.q = q;
+  c.B = B;
+  c.Hq = Hq;
+  c.scale = scale;
+  c.kv = &kv;
+  c.a_out = a_in;
+  c.l_out = l_in;
+  // the block is short: one split per (b, hk, row tile), no workspace needed
+  c.single_split = true;
+  return launch_partial(c, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fb_last_error(void) { return g_last_error.c_str(); }
+
+int fb_device_status(void) {
+  int word = 0, zero = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return fail(FB_ERR_CUDA, "device synchronize failed");
+  if (cudaMemcpyFromSymbol(&word, g_fb_error_word, sizeof(int)) != cudaSuccess)
+    return fail(FB_ERR_CUDA, "reading the device error word failed");
+  cudaMemcpyToSymbol(g_fb_error_word, &zero, sizeof(int));
+  if (word) return fail(FB_ERR_TIMEOUT, "a device-side wait exceeded its budget");
+  return FB_OK;
+}
+
+size_t fb_workspace_size(const fb_kv* kv, int32_t block, int32_t n_heads_q, int32_t n_active,
+                         int32_t topk_pages, int32_t num_sms) {
+  if (!kv || block <= 0 || n_heads_q <= 0 || kv->n_heads_kv <= 0 || n_heads_q % kv->n_heads_kv ||
+      kv->batch <= 0 || kv->max_seq_len < 0 || kv->page_size <= 0)
+    return 0;
+  if (num_sms <= 0) num_sms = sm_count();
+  if (num_sms <= 0) return 0;
+  return ws_layout(kv, block, n_heads_q, n_active, topk_pages, num_sms).total;
+}
+
+int fb_prefix_attn(const void* q, int32_t B, int32_t n_heads_q, float scale, const fb_kv* kv,
+                   const uint8_t* head_mask, float* a_out, float* l_out, void* workspace,
+                   size_t workspace_bytes, cudaStream_t stream) {
+  int rc = validate_kv(kv);
+  if (rc) return rc;
+  rc = validate_q(q, B, n_heads_q, kv);
+  if (rc) return rc;
+  if (!a_out || !l_out) return fail(FB_ERR_ARG, "a_out / l_out is NULL");
+  PartialCall c{};
+  c.q = q;
+  c.B = B;
+  c.Hq = n_heads_q;
+  c.scale = scale;
+  c.kv = kv;
+  c.head_mask = head_mask;
+  c.a_out = a_out;
+  c.l_out = l_out;
+  c.ws = workspace;
+  c.ws_bytes = workspace_bytes;
+  c.num_sms = sm_count();
+  return launch_partial(c, stream);
+}
+
+int fb_block_attn(const void* q, const void* k_in, const void* v_in, int32_t batch, int32_t B,
+                  int32_t n_heads_q, int32_t n_heads_kv, int32_t head_dim, float scale,
+                  fb_dtype dtype, float* a_in, float* l_in, cudaStream_t stream) {
+  return block_attn_impl(q, k_in, v_in, batch, B, n_heads_q, n_heads_kv, head_dim, scale, dtype,
+                         a_in, l_in, stream);
+}
+
+int fb_merge(const float* a_out, const float* l_out, const float* a_in, const float* l_in,
+             int64_t rows, int32_t head_dim, float* a_full, float* l_full, cudaStream_t stream) {
+  if (!a_out || !l_out || !a_in || !l_in || !a_full) return fail(FB_ERR_ARG, "NULL argument");
+  if (rows < 0) return fail(FB_ERR_ARG, "rows < 0");
+  if (head_dim != 64 && head_dim != 128) return fail(FB_ERR_SHAPE, "head_dim must be 64 or 128");
+  return merge_launch(a_out, l_out, a_in, l_in, rows, head_dim, a_full, l_full, stream);
+}
+
+int fb_page_summary(const fb_kv* kv, void* page_min, void* page_max, cudaStream_t stream) {
+  int rc = validate_kv(kv);
+  if (rc) return rc;
+  if (!page_min || !page_max) return fail(FB_ERR_ARG, "page_min / page_max is NULL");
+  const KvView v = kv_view(kv);
+  const long long warps = (long long)v.batch * v.max_pages * v.Hkv;
+  if (warps == 0) return FB_OK;
+  const int blocks = ceil_div(warps * 32, 256);
+  if (kv->dtype == FB_BF16) {
+    auto* mn = static_cast<__nv_bfloat16*>(page_min);
+    auto* mx = static_cast<__nv_bfloat16*>(page_max);
+    if (v.D == 128)
+      page_summary_kernel<__nv_bfloat16, 128><<<blocks, 256, 0, stream>>>(v, mn, mx);
+    else
+      page_summary_kernel<__nv_bfloat16, 64><<<blocks, 256, 0, stream>>>(v, mn, mx);
+  } else {
+    auto* mn = static_cast<float*>(page_min);
+    auto* mx = static_cast<float*>(page_max);
+    if (v.D == 128)
+      page_summary_kernel<float, 128><<<blocks, 256, 0, stream>>>(v, mn, mx);
+    else
+      page_summary_kernel<float, 64><<<blocks, 256, 0, stream>>>(v, mn, mx);
+  }
+  return check_launch("page summary kernel");
+}
+
+int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_heads_q,
+                const void* page_min, const void* page_max, const fb_kv* kv, int32_t n_active,
+                int32_t topk_pages, int32_t* active_rows, float* row_scores,
+                uint32_t* union_bitmap, int32_t* union_list, int32_t* union_count,
+                void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  int rc = validate_kv(kv);
+  if (rc) return rc;
+  rc = validate_q(q_cur, B, n_heads_q, kv);
+  if (rc) return rc;
+  if (!q_prev || !page_min || !page_max || !active_rows || !union_bitmap || !union_list ||
+      !union_count)
+    return fail(FB_ERR_ARG, "NULL argument");
+  if (n_active < 0 || topk_pages < 0) return fail(FB_ERR_ARG, "n_active / topk_pages < 0");
+  const KvView v = kv_view(kv);
+  const int D = v.D, Hq = n_heads_q, G = Hq / v.Hkv;
+  const int na = n_active < B ? n_active : B;
+  const int words = ceil_div(v.max_pages, 32);
+  if (v.max_pages > 32768) return fail(FB_ERR_SHAPE, "LoSA selection supports <= 32768 pages");
+  if (Hq * D > 16384) return fail(FB_ERR_SHAPE, "LoSA selection supports n_heads_q * d <= 16384");
+  const int num_sms = sm_count();
+  const WsLayout w = ws_layout(kv, B, Hq, n_active, topk_pages, num_sms);
+  if (!workspace || workspace_bytes < w.total)
+    return fail(FB_ERR_WORKSPACE, "workspace too small: need %zu, have %zu", w.total,
+                workspace_bytes);
+  char* ws = static_cast<char*>(workspace);
+  float* page_scores = reinterpret_cast<float*>(ws + w.scores);
+  float* rs = row_scores
+                  ? row_scores
+                  : reinterpret_cast<float*>(ws + w.scores +
+                                             round_up((size_t)kv->batch * na * Hq * v.max_pages * 4,
+                                                      256));
+  const int N = Hq * D, N2 = next_pow2(N);
+  if (na == 0) {
+    // no active rows: an empty union (the bitmap and counts still get written)
+    cudaMemsetAsync(union_bitmap, 0, (size_t)kv->batch * v.Hkv * words * 4, stream);
+    cudaMemsetAsync(union_count, 0, (size_t)kv->batch * v.Hkv * 4, stream);
+    return check_launch("losa_select memset");
+  }
+  const dim3 g1(B, kv->batch);
+  if (N2 * 4 > 48 * 1024) {
+    cudaFuncSetAttribute(locality_score_kernel<__nv_bfloat16>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, N2 * 4);
+    cudaFuncSetAttribute(locality_score_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         N2 * 4);
+  }
+  if (kv->dtype == FB_BF16)
+    locality_score_kernel<__nv_bfloat16><<<g1, 256, N2 * 4, stream>>>(
+        static_cast<const __nv_bfloat16*>(q_cur), static_cast<const __nv_bfloat16*>(q_prev), B, N,
+        N2, rs);
+  else
+    locality_score_kernel<float><<<g1, 256, N2 * 4, stream>>>(
+        static_cast<const float*>(q_cur), static_cast<const float*>(q_prev), B, N, N2, rs);
+  rc = check_launch("locality score kernel");
+  if (rc) return rc;
+  active_rows_kernel<<<kv->batch, 256, B * 4, stream>>>(rs, B, na, active_rows);
+  rc = check_launch("active rows kernel");
+  if (rc) return rc;
+  const dim3 g2(ceil_div(v.max_pages, 8), v.Hkv, kv->batch);
+  const int qsm = na * G * D * 4;
+  if (kv->dtype == FB_BF16) {
+    auto kfn = D == 128 ? page_score_kernel<__nv_bfloat16, 128> : page_score_kernel<__nv_bfloat16, 64>;
+    if (qsm > 48 * 1024) cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, qsm);
+    kfn<<<g2, 256, qsm, stream>>>(static_cast<const __nv_bfloat16*>(q_cur), active_rows, B, Hq, G,
+                                  na, static_cast<const __nv_bfloat16*>(page_min),
+                                  static_cast<const __nv_bfloat16*>(page_max), v, page_scores,
+                                  union_bitmap, words);
+  } else {
+    auto kfn = D == 128 ? page_score_kernel<float, 128> : page_score_kernel<float, 64>;
+    if (qsm > 48 * 1024) cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, qsm);
+    kfn<<<g2, 256, qsm, stream>>>(static_cast<const float*>(q_cur), active_rows, B, Hq, G, na,
+                                  static_cast<const float*>(page_min),
+                                  static_cast<const float*>(page_max), v, page_scores,
+                                  union_bitmap, words);
+  }
+  rc = check_launch("page score kernel");
+  if (rc) return rc;
+  const int ksm = v.max_pages * 4;
+  if (ksm > 48 * 1024)
+    cudaFuncSetAttribute(topk_pages_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ksm);
+  topk_pages_kernel<<<dim3(na * Hq, kv->batch), kTopkThreads, ksm, stream>>>(
+      page_scores, v, Hq, G, na, topk_pages, union_bitmap, words);
+  rc = check_launch("top-k pages kernel");
+  if (rc) return rc;
+  union_compact_kernel<<<dim3(v.Hkv, kv->batch), 256, 0, stream>>>(union_bitmap, words, v.Hkv,
+                                                                   v.max_pages, union_list,
+                                                                   union_count);
+  return check_launch("union compaction kernel");
+}
+
+int losa_gather(const void* q, int32_t B, int32_t n_heads_q, const int32_t* active_rows,
+                int32_t n_active, const int32_t* union_list, const int32_t* union_count,
+                int32_t max_union, const fb_kv* kv, float scale, float* a_out, float* l_out,
+                void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  int rc = validate_kv(kv);
+  if (rc) return rc;
+  rc = validate_q(q, B, n_heads_q, kv);
+  if (rc) return rc;
+  if (!a_out || !l_out || !union_list || !union_count || (n_active > 0 && !active_rows))
+    return fail(FB_ERR_ARG, "NULL argument");
+  const int na = n_active < B ? n_active : B;
+  if (na <= 0) return FB_OK;
+  const KvView v = kv_view(kv);
+  PartialCall c{};
+  c.q = q;
+  c.B = B;
+  c.Hq = n_heads_q;
+  c.scale = scale;
+  c.kv = kv;
+  c.row_list = active_rows;
+  c.n_list = na;
+  c.page_list = union_list;
+  c.page_count = union_count;
+  c.page_list_stride = v.max_pages;
+  c.max_list_entries = (max_union > 0 && max_union < v.max_pages) ? max_union : v.max_pages;
+  c.a_out = a_out;
+  c.l_out = l_out;
+  c.ws = workspace;
+  c.ws_bytes = workspace_bytes;
+  c.num_sms = sm_count();
+  return launch_partial(c, stream);
+}
+
+int fb_step(const fb_policy* policy, fb_cache* cache, const void* q, const void* k_in,
+            const void* v_in, int32_t B, int32_t n_heads_q, const fb_kv* prefix,
+            const void* page_min, const void* page_max, const int32_t* m_updated, float* a_full,
+            float* l_full, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!policy || !cache) return fail(FB_ERR_ARG, "policy / cache is NULL");
+  int rc = validate_kv(prefix);
+  if (rc) return rc;
+  rc = validate_q(q, B, n_heads_q, prefix);
+  if (rc) return rc;
+  if (!k_in || !v_in || !a_full || !cache->a_out || !cache->l_out)
+    return fail(FB_ERR_ARG, "NULL argument");
+  const int batch = prefix->batch, Hq = n_heads_q, Hkv = prefix->n_heads_kv, D = prefix->head_dim;
+  const int s = cache->step;
+  const int num_sms = sm_count();
+  const int na = policy->mode == FB_LOSA ? policy->n_active : 0;
+  const int tk = policy->mode == FB_LOSA ? policy->topk_pages : 0;
+  const WsLayout w = ws_layout(prefix, B, Hq, na, tk, num_sms);
+  if (!workspace || workspace_bytes < w.total)
+    return fail(FB_ERR_WORKSPACE, "workspace too small: need %zu, have %zu", w.total,
+                workspace_bytes);
+  char* ws = static_cast<char*>(workspace);
+  PartialCall c{};
+  c.q = q;
+  c.B = B;
+  c.Hq = Hq;
+  c.scale = policy->scale;
+  c.kv = prefix;
+  c.a_out = cache->a_out;
+  c.l_out = cache->l_out;
+  c.ws = workspace;
+  c.ws_bytes = workspace_bytes;
+  c.ws_offset = w.part;
+  c.num_sms = num_sms;
+
+  if (policy->mode == FB_THRESHOLD) {
+    unsigned long long bits[4] = {0, 0, 0, 0};
+    int n_rec = 0;
+    for (int b = 0; b < batch; ++b) {
+      const bool rec = s == 0 || policy->tau <= 0 || (m_updated && m_updated[b] >= policy->tau);
+      if (rec) {
+        bits[b >> 6] |= 1ull << (b & 63);
+        ++n_rec;
+      }
+    }
+    cache->recomputed = n_rec;
+    if (n_rec > 0) {
+      c.seq_bits = n_rec < batch ? bits : nullptr;
+      rc = launch_partial(c, stream);
+      if (rc) return rc;
+    }
+  } else if (policy->mode == FB_PER_HEAD) {
+    if (!cache->head_mask || !cache->a_out_prev || !cache->head_cos)
+      return fail(FB_ERR_ARG, "PER_HEAD needs head_mask, a_out_prev and head_cos");
+    if (s == 0) {
+      cudaMemsetAsync(cache->head_mask, 1, (size_t)batch * Hq, stream);
+      rc = check_launch("head mask reset");
+      if (rc) return rc;
+    }
+    c.head_mask = cache->head_mask;
+    c.a_prev = cache->a_out_prev;
+    rc = launch_partial(c, stream);
+    if (rc) return rc;
+    if (s >= 1) {
+      const int N = B * D, P = next_pow2(N);
+      if (P > kCosT1Max * kCosEMax) return fail(FB_ERR_SHAPE, "B * d too large for the cosine");
+      const int T1 = P < kCosT1Max ? P : kCosT1Max, E = P / T1;
+      double* part = reinterpret_cast<double*>(ws + w.cos);
+      head_cos_stage1<<<dim3(ceil_div(T1, 256), batch * Hq), 256, 0, stream>>>(
+          cache->a_out, cache->a_out_prev, cache->head_mask, B, Hq, D, N, T1, E, part);
+      rc = check_launch("cosine stage 1");
+      if (rc) return rc;
+      head_cos_stage2<<<batch * Hq, 1024, 0, stream>>>(part, T1, policy->gamma, cache->head_mask,
+                                                      cache->head_cos);
+      rc = check_launch("cosine stage 2");
+      if (rc) return rc;
+    }
+  } else if (policy->mode == FB_LOSA) {
+    if (!cache->q_prev || !cache->active_rows || !cache->union_bitmap || !cache->union_list ||
+        !cache->union_count)
+      return fail(FB_ERR_ARG, "LOSA needs q_prev, active_rows and the union buffers");
+    if (s == 0) {
+      rc = launch_partial(c, stream);
+      if (rc) return rc;
+    } else {
+      rc = losa_select(q, cache->q_prev, B, Hq, page_min, page_max, prefix, policy->n_active,
+                       policy->topk_pages, cache->active_rows, cache->row_scores,
+                       cache->union_bitmap, cache->union_list, cache->union_count, workspace,
+                       workspace_bytes, stream);
+      if (rc) return rc;
+      const int na_c = policy->n_active < B ? policy->n_active : B;
+      rc = losa_gather(q, B, Hq, cache->active_rows, policy->n_active, cache->union_list,
+                       cache->union_count,
+                       max_union_entries(prefix, Hq / Hkv, na_c, policy->topk_pages), prefix,
+                       policy->scale, cache->a_out, cache->l_out, workspace, workspace_bytes,
+                       stream);
+      if (rc) return rc;
+    }
+    const size_t qbytes = (size_t)batch * B * Hq * D * elem_size(prefix->dtype);
+    if (cudaMemcpyAsync(cache->q_prev, q, qbytes, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+      return fail(FB_ERR_CUDA, "q_prev copy failed");
+  } else {
+    return fail(FB_ERR_ARG, "unknown mode");
+  }
+  float* a_in = reinterpret_cast<float*>(ws + w.a_in);
+  float* l_in = reinterpret_cast<float*>(ws + w.l_in);
+  rc = block_attn_impl(q, k_in, v_in, batch, B, Hq, Hkv, D, policy->scale, prefix->dtype, a_in,
+                       l_in, stream);
+  if (rc) return rc;
+  rc = merge_launch(cache->a_out, cache->l_out, a_in, l_in, (long long)batch * B * Hq, D, a_full,
+                    l_full, stream);
+  if (rc) return rc;
+  cache->step = s + 1;
+  return FB_OK;
+}
+
+}  // extern "C"

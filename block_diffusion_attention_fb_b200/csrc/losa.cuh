@@ -1,0 +1,341 @@
+// LoSA selection kernels ("LoSA: Locality Aware Sparse Attention for
+// Block-Wise Diffusion Language Models", §2 "El Algoritmo LoSA", steps 1 and 3)
+// and the per-page key summaries its QUEST-style selector scores.
+//
+// Decisions are integers chosen by float scores, so every score is computed
+// in one fixed float32 order: single-rounded products (__fmul_rn), and sums by
+// the stride-halving tree (pad to a power of two N; for stride = N/2 ... 1,
+// x[n] += x[n + stride] for n < stride). Ties go to the lower index.
+#pragma once
+
+#include "common.cuh"
+
+namespace fb {
+
+template <typename T>
+__device__ __forceinline__ float ld_f32(const T* p);
+template <>
+__device__ __forceinline__ float ld_f32<float>(const float* p) {
+  return *p;
+}
+template <>
+__device__ __forceinline__ float ld_f32<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(*p);
+}
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) {
+  return x;
+}
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);  // exact here: x is a bf16 value
+}
+
+struct KvView {
+  const void* k;
+  const int32_t* page_table;
+  const int32_t* seq_len;
+  int batch, Hkv, D, page_size, max_pages, max_seq_len;
+};
+
+__device__ __forceinline__ int kv_tokens(const KvView& kv, int b) {
+  return kv.seq_len ? kv.seq_len[b] : kv.max_seq_len;
+}
+
+__device__ __forceinline__ long long kv_slot(const KvView& kv, int b, int t) {
+  if (kv.page_table) {
+    const int lp = t / kv.page_size;
+    return (long long)kv.page_table[(long long)b * kv.max_pages + lp] * kv.page_size +
+           (t - lp * kv.page_size);
+  }
+  return (long long)b * kv.max_seq_len + t;
+}
+
+// ---------------------------------------------------------------------------
+// Per (sequence, logical page, kv head, channel): min and max of the page's
+// valid keys. One warp per (b, page, hk); lanes hold channels lane + 32 j.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+    page_summary_kernel(const KvView kv, T* __restrict__ pmin, T* __restrict__ pmax) {
+  constexpr int NV = D / 32;
+  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long total = (long long)kv.batch * kv.max_pages * kv.Hkv;
+  if (w >= total) return;
+  const int hk = (int)(w % kv.Hkv);
+  const int p = (int)((w / kv.Hkv) % kv.max_pages);
+  const int b = (int)(w / ((long long)kv.Hkv * kv.max_pages));
+  const int n = kv_tokens(kv, b);
+  const int t0 = p * kv.page_size;
+  if (t0 >= n) return;
+  const int t1 = min(n, t0 + kv.page_size);
+  const T* kg = static_cast<const T*>(kv.k);
+  float mn[NV], mx[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    mn[j] = INFINITY;
+    mx[j] = -INFINITY;
+  }
+  for (int t = t0; t < t1; ++t) {
+    const T* row = kg + (kv_slot(kv, b, t) * kv.Hkv + hk) * D;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const float x = ld_f32<T>(row + lane + 32 * j);
+      mn[j] = fminf(mn[j], x);
+      mx[j] = fmaxf(mx[j], x);
+    }
+  }
+  const long long o = (((long long)b * kv.max_pages + p) * kv.Hkv + hk) * D;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    pmin[o + lane + 32 * j] = from_f32<T>(mn[j]);
+    pmax[o + lane + 32 * j] = from_f32<T>(mx[j]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Step 1a: locality score of every block row, sum_{h,c} (q_cur - q_prev)^2
+// by the stride-halving tree over n = h * D + c. One CTA per (row, sequence);
+// the tree runs level by level in shared memory exactly as defined.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256)
+    locality_score_kernel(const T* __restrict__ qc, const T* __restrict__ qp, int B, int N,
+                          int N2, float* __restrict__ score) {
+  extern __shared__ float xs[];  // N2 floats
+  const int i = blockIdx.x, b = blockIdx.y;
+  const long long off = ((long long)b * B + i) * N;
+  for (int n = threadIdx.x; n < N2; n += blockDim.x) {
+    float v = 0.f;
+    if (n < N) {
+      const float d = __fsub_rn(ld_f32<T>(qc + off + n), ld_f32<T>(qp + off + n));
+      v = __fmul_rn(d, d);
+    }
+    xs[n] = v;
+  }
+  __syncthreads();
+  for (int s = N2 >> 1; s >= 1; s >>= 1) {
+    for (int n = threadIdx.x; n < s; n += blockDim.x) xs[n] = __fadd_rn(xs[n], xs[n + s]);
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) score[(long long)b * B + i] = xs[0];
+}
+
+// Step 1b: the n_act highest-scoring rows of each sequence, in rank order
+// (score descending, then row ascending). O(B^2) ranks; B is a block size.
+__global__ void __launch_bounds__(256)
+    active_rows_kernel(const float* __restrict__ score, int B, int n_act,
+                       int32_t* __restrict__ active) {
+  extern __shared__ float sc[];
+  const int b = blockIdx.x;
+  for (int i = threadIdx.x; i < B; i += blockDim.x) sc[i] = score[(long long)b * B + i];
+  __syncthreads();
+  for (int i = threadIdx.x; i < B; i += blockDim.x) {
+    const float si = sc[i];
+    int rank = 0;
+    for (int j = 0; j < B; ++j) {
+      const float sj = sc[j];
+      rank += (sj > si) || (sj == si && j < i);
+    }
+    if (rank < n_act) active[b * n_act + rank] = i;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Step 3a: QUEST-style page scores u_p = tree_sum_c max(q_c kmin_c, q_c kmax_c)
+// for every active row a and q head h of kv head hk. One warp per page; lane l
+// holds channels l + 32 j, so the first levels of the tree (strides >= 32) run
+// inside the lane and the last five through xor shuffles.
+// scores: [batch, n_act, Hq, max_pages]. Block (0, hk, b) also clears the
+// union bitmap of (b, hk) for the top-k kernel that follows.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+    page_score_kernel(const T* __restrict__ q, const int32_t* __restrict__ active, int B, int Hq,
+                      int G, int n_act, const T* __restrict__ pmin, const T* __restrict__ pmax,
+                      const KvView kv, float* __restrict__ scores, uint32_t* __restrict__ bitmap,
+                      int words) {
+  constexpr int NV = D / 32;
+  extern __shared__ float qs[];  // [n_act * G][D]
+  const int hk = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (blockIdx.x == 0)
+    for (int w = threadIdx.x; w < words; w += blockDim.x)
+      bitmap[((long long)b * kv.Hkv + hk) * words + w] = 0u;
+  const int RQ = n_act * G;
+  for (int idx = threadIdx.x; idx < RQ * D; idx += blockDim.x) {
+    const int rq = idx / D, c = idx - (idx / D) * D;
+    const int a_i = rq / G, g = rq - (rq / G) * G;
+    const int i = active[b * n_act + a_i];
+    qs[idx] = ld_f32<T>(q + (((long long)b * B + i) * Hq + hk * G + g) * D + c);
+  }
+  __syncthreads();
+  const int n_pages = (kv_tokens(kv, b) + kv.page_size - 1) / kv.page_size;
+  const int p = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (p >= n_pages) return;
+  const long long so = (((long long)b * kv.max_pages + p) * kv.Hkv + hk) * D;
+  float lo[NV], hi[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    lo[j] = ld_f32<T>(pmin + so + lane + 32 * j);
+    hi[j] = ld_f32<T>(pmax + so + lane + 32 * j);
+  }
+  for (int rq = 0; rq < RQ; ++rq) {
+    float x[NV];
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const float qv = qs[rq * D + lane + 32 * j];
+      x[j] = fmaxf(__fmul_rn(qv, lo[j]), __fmul_rn(qv, hi[j]));
+    }
+    // in-lane levels: strides D/2 ... 32 pair j with j + NV/2 ...
+#pragma unroll
+    for (int s = NV / 2; s >= 1; s >>= 1)
+#pragma unroll
+      for (int j = 0; j < s; ++j) x[j] = __fadd_rn(x[j], x[j + s]);
+    float v = x[0];
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, s));
+    if (lane == 0) {
+      const int a_i = rq / G, g = rq - (rq / G) * G;
+      scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = v;
+    }
+  }
+}
+
+// Order-preserving map float -> uint32 (larger float, larger key); -0 == +0.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  if (f == 0.f) f = 0.f;
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// ---------------------------------------------------------------------------
+// Step 3b: top-k pages of one (active row, q head): exact radix select of the
+// k-th largest key (4 passes of 8 bits), then every key above it plus the
+// lowest-index keys equal to it. The picks are OR-ed into the union bitmap of
+// the kv head. One CTA of kTopkThreads per (b, a, h).
+// ---------------------------------------------------------------------------
+constexpr int kTopkThreads = 512;
+
+__global__ void __launch_bounds__(kTopkThreads)
+    topk_pages_kernel(const float* __restrict__ scores, const KvView kv, int Hq, int G, int n_act,
+                      int topk, uint32_t* __restrict__ bitmap, int words) {
+  extern __shared__ uint32_t keys[];  // max_pages
+  __shared__ int hist[256];
+  __shared__ int seg_cnt[kTopkThreads];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_need;
+  const int ah = blockIdx.x, b = blockIdx.y;
+  const int h = ah % Hq;
+  const int hk = h / G;
+  const int tid = threadIdx.x;
+  const int n = (kv_tokens(kv, b) + kv.page_size - 1) / kv.page_size;
+  const int k = min(topk, n);
+  uint32_t* bm = bitmap + ((long long)b * kv.Hkv + hk) * words;
+  const float* sc = scores + ((long long)b * n_act * Hq + ah) * kv.max_pages;
+  if (k <= 0) return;
+  if (k == n) {
+    for (int p = tid; p < n; p += blockDim.x) atomicOr(&bm[p >> 5], 1u << (p & 31));
+    return;
+  }
+  for (int p = tid; p < n; p += blockDim.x) keys[p] = order_key(sc[p]);
+  if (tid == 0) {
+    s_prefix = 0u;
+    s_need = k;
+  }
+  uint32_t mask = 0u;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int d = tid; d < 256; d += blockDim.x) hist[d] = 0;
+    __syncthreads();
+    const uint32_t prefix = s_prefix;
+    for (int p = tid; p < n; p += blockDim.x) {
+      const uint32_t key = keys[p];
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int need = s_need, cum = 0, sel = 0;
+      for (int d = 255; d >= 0; --d) {
+        if (cum + hist[d] >= need) {
+          sel = d;
+          need -= cum;
+          break;
+        }
+        cum += hist[d];
+      }
+      s_prefix = prefix | ((uint32_t)sel << shift);
+      s_need = need;
+    }
+    mask |= 0xFFu << shift;
+    __syncthreads();
+  }
+  const uint32_t T = s_prefix;  // key of the k-th largest score
+  const int need = s_need;      // how many keys equal to T are taken
+  // keys equal to T: take the lowest indices, via a scan of per-thread segments
+  const int seg = (n + kTopkThreads - 1) / kTopkThreads;
+  const int p0 = tid * seg, p1 = min(n, p0 + seg);
+  int cnt = 0;
+  for (int p = p0; p < p1; ++p) cnt += (keys[p] == T);
+  seg_cnt[tid] = cnt;
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int t = 0; t < kTopkThreads; ++t) {
+      const int c = seg_cnt[t];
+      seg_cnt[t] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  int eq_before = seg_cnt[tid];
+  for (int p = p0; p < p1; ++p) {
+    const uint32_t key = keys[p];
+    bool take = key > T;
+    if (key == T) {
+      take = eq_before < need;
+      ++eq_before;
+    }
+    if (take) atomicOr(&bm[p >> 5], 1u << (p & 31));
+  }
+}
+
+// Step 3c: union bitmap -> ascending page list and count per (b, hk).
+__global__ void __launch_bounds__(256)
+    union_compact_kernel(const uint32_t* __restrict__ bitmap, int words, int Hkv, int stride,
+                         int32_t* __restrict__ list, int32_t* __restrict__ count) {
+  __shared__ int wsum[256];
+  const int hk = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const uint32_t* bm = bitmap + ((long long)b * Hkv + hk) * words;
+  int32_t* out = list + ((long long)b * Hkv + hk) * stride;
+  const int per = (words + 255) / 256;
+  const int w0 = tid * per, w1 = min(words, w0 + per);
+  int c = 0;
+  for (int w = w0; w < w1; ++w) c += __popc(bm[w]);
+  wsum[tid] = c;
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int t = 0; t < 256; ++t) {
+      const int x = wsum[t];
+      wsum[t] = run;
+      run += x;
+    }
+    count[b * Hkv + hk] = run;
+  }
+  __syncthreads();
+  int pos = wsum[tid];
+  for (int w = w0; w < w1; ++w) {
+    uint32_t bits = bm[w];
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      out[pos++] = w * 32 + bit;
+    }
+  }
+}
+
+}  // namespace fb

@@ -1,0 +1,253 @@
+/*
+ * fb.h - C ABI of the per-denoise-step block-diffusion attention library
+ * (FlashBlock cached block-external attention and the LoSA sparse variant),
+ * built for NVIDIA B200 (sm_100a).
+ *
+ * Method sources (cited by page title and section):
+ *  [FB]   "FlashBlock: Attention Caching for Efficient Long-Context Block
+ *         Diffusion", technical summary (gist.science, pt and ja), section 2
+ *         "Core mechanism" (block-internal / block-external split, cached
+ *         (A_out, L_out = log Z_out), merge equation) and "Adaptive reuse
+ *         strategies" (threshold tau, per-head gamma).
+ *  [LoSA] "LoSA: Locality Aware Sparse Attention for Block-Wise Diffusion
+ *         Language Models" (gist.science, es), section 2 "El Algoritmo LoSA",
+ *         steps 1-4.
+ *
+ * Conventions for every call:
+ *  - Pointers are DEVICE pointers owned by the caller unless a parameter says
+ *    "host". The library never allocates device memory; scratch comes from a
+ *    caller-provided workspace whose size fb_workspace_size() returns.
+ *  - Calls are asynchronous on `stream` and never synchronise, except where
+ *    stated (fb_device_status).
+ *  - Layouts are row-major. q: [batch, B, Hq, d]; block k/v: [batch, B, Hkv, d];
+ *    partials A: [batch, B, Hq, d] float32, L: [batch, B, Hq] float32.
+ *    L values are natural logarithms of the softmax normaliser (log Z).
+ *    q head h reads kv head h / (Hq / Hkv).
+ *  - Every call validates its arguments on the host before launching and
+ *    returns FB_OK (0) or a negative FB_ERR_* code; the text of the last error
+ *    of the calling thread is returned by fb_last_error().
+ *  - Supported: head_dim 128 (bf16 and f32) or 64; page_size a power of two in
+ *    [16, 128] for paged caches; 16-byte aligned tensors. Anything else is
+ *    FB_ERR_SHAPE / FB_ERR_ALIGN.
+ */
+#ifndef FB_H_
+#define FB_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FB_OK 0
+#define FB_ERR_ARG (-1)       /* null pointer, negative size, inconsistent shapes */
+#define FB_ERR_SHAPE (-2)     /* unsupported head_dim, page size, group size */
+#define FB_ERR_ALIGN (-3)     /* a tensor is not 16-byte aligned */
+#define FB_ERR_WORKSPACE (-4) /* workspace missing or smaller than required */
+#define FB_ERR_CUDA (-5)      /* launch or driver error; text in fb_last_error() */
+#define FB_ERR_TIMEOUT (-6)   /* a device-side wait exceeded its budget */
+
+typedef enum { FB_F32 = 0, FB_BF16 = 1 } fb_dtype;
+
+/*
+ * The frozen block-external KV cache (J_out in [FB] section 2).
+ *  k, v        [n_slots, n_heads_kv, head_dim] rows of `dtype`.
+ *  page_table  [batch, max_pages_per_seq] int32 physical page of each logical
+ *              page, or NULL for a contiguous cache where sequence b's token t
+ *              is row b * max_seq_len + t.
+ *              Paged: token t of sequence b is row
+ *                page_table[b][t / page_size] * page_size + t % page_size.
+ *  seq_len     [batch] int32 tokens per sequence (<= max_seq_len), or NULL when
+ *              every sequence has max_seq_len tokens.
+ *  page_size   tokens per logical page (also the LoSA page granularity).
+ * Rows past a sequence's end may hold any bits (NaN included): they never
+ * reach an output.
+ */
+typedef struct fb_kv {
+  const void* k;
+  const void* v;
+  const int32_t* page_table;
+  const int32_t* seq_len;
+  int64_t n_slots;
+  int32_t batch;
+  int32_t n_heads_kv;
+  int32_t head_dim;
+  int32_t page_size;
+  int32_t max_pages_per_seq;
+  int32_t max_seq_len;
+  fb_dtype dtype;
+} fb_kv;
+
+/*
+ * Bytes of workspace that fb_prefix_attn, losa_select, losa_gather and fb_step
+ * need for these shapes (n_active/topk_pages may be 0 when LoSA is unused).
+ * num_sms: SM count the split plan targets (0: query the current device).
+ * Returns 0 on invalid arguments.
+ */
+size_t fb_workspace_size(const fb_kv* kv, int32_t block, int32_t n_heads_q, int32_t n_active,
+                         int32_t topk_pages, int32_t num_sms);
+
+/*
+ * Block-external partial ([FB] section 2: A_out and L_out = log Z_out over J_out).
+ * For every block row i and q head h:
+ *   L_out = log sum_{t < seq_len[b]} exp(scale * <q_i,h , k_t>)
+ *   A_out = sum_t exp(scale * <q, k_t> - L_out) v_t
+ * computed by split-KV flash decoding (per-split partials merged with the same
+ * log-space rule as [FB]'s merge).
+ *  q          [batch, B, n_heads_q, head_dim] of kv->dtype.
+ *  head_mask  [batch, n_heads_q] uint8 or NULL; heads with 0 are skipped and
+ *             their a_out/l_out rows are left untouched (cache reuse).
+ *  a_out      [batch, B, n_heads_q, head_dim] float32 (output).
+ *  l_out      [batch, B, n_heads_q] float32 (output). An empty prefix gives
+ *             A_out = 0, L_out = -inf.
+ *  workspace  >= fb_workspace_size(kv, B, n_heads_q, 0, 0, 0) bytes.
+ */
+int fb_prefix_attn(const void* q, int32_t B, int32_t n_heads_q, float scale, const fb_kv* kv,
+                   const uint8_t* head_mask, float* a_out, float* l_out, void* workspace,
+                   size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Block-internal partial ([FB] section 2: A_in, L_in over J_in, recomputed
+ * every step). Bidirectional: every block row attends all B block tokens.
+ *  q [batch, B, n_heads_q, head_dim], k_in / v_in [batch, B, n_heads_kv, head_dim]
+ *  of `dtype`; a_in [batch, B, n_heads_q, head_dim], l_in [batch, B, n_heads_q]
+ *  float32 outputs.
+ */
+int fb_block_attn(const void* q, const void* k_in, const void* v_in, int32_t batch, int32_t B,
+                  int32_t n_heads_q, int32_t n_heads_kv, int32_t head_dim, float scale,
+                  fb_dtype dtype, float* a_in, float* l_in, cudaStream_t stream);
+
+/*
+ * Log-space merge ([FB] section 2, merge equation):
+ *   m = max(L_out, L_in)
+ *   A_full = (e^{L_out-m} A_out + e^{L_in-m} A_in) / (e^{L_out-m} + e^{L_in-m})
+ *   L_full = m + log(e^{L_out-m} + e^{L_in-m})
+ * rows = batch * B * Hq rows of head_dim floats. l_full may be NULL. A side
+ * with L = -inf contributes nothing; both -inf gives A = 0, L = -inf.
+ */
+int fb_merge(const float* a_out, const float* l_out, const float* a_in, const float* l_in,
+             int64_t rows, int32_t head_dim, float* a_full, float* l_full, cudaStream_t stream);
+
+/*
+ * Per-page key summary for the LoSA selector (QUEST-style upper bound).
+ * page_min / page_max: [batch, max_pages_per_seq, n_heads_kv, head_dim] of
+ * kv->dtype: per logical page, kv head and channel, the min / max of the
+ * page's keys over its valid tokens (t < seq_len). Pages past the end of a
+ * sequence are not written. Exact (no rounding).
+ */
+int fb_page_summary(const fb_kv* kv, void* page_min, void* page_max, cudaStream_t stream);
+
+/*
+ * LoSA selection ([LoSA] steps 1 and 3), one call per denoise step s >= 1.
+ *  1. locality score per block row: sum over heads and channels of
+ *     (q_cur - q_prev)^2, float32, squares rounded singly and summed by the
+ *     stride-halving tree over n = h * head_dim + c;
+ *  2. active_rows [batch, n_active]: the n_active highest scores per sequence,
+ *     in rank order (ties: lower row first); n_active is clamped to B;
+ *  3. for every active row and q head, page scores
+ *     u_p = tree_sum_c max(q_c * kmin_{p,c}, q_c * kmax_{p,c}) (float32) and the
+ *     topk_pages best pages (ties: lower page first);
+ *  4. union over active rows and the q heads of each kv head:
+ *     union_bitmap [batch, n_heads_kv, ceil(max_pages/32)] uint32 (bit p%32 of
+ *     word p/32), union_list [batch, n_heads_kv, max_pages_per_seq] int32 pages
+ *     in ascending order, union_count [batch, n_heads_kv] int32.
+ *  row_scores [batch, B] float32 receives the locality scores (may be NULL).
+ *  q_cur / q_prev: [batch, B, n_heads_q, head_dim] of kv->dtype.
+ */
+int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_heads_q,
+                const void* page_min, const void* page_max, const fb_kv* kv, int32_t n_active,
+                int32_t topk_pages, int32_t* active_rows, float* row_scores,
+                uint32_t* union_bitmap, int32_t* union_list, int32_t* union_count,
+                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * LoSA sparse prefix partial for the active rows ([LoSA] step 3, with step 2's
+ * reuse for the others): for every active row i (active_rows[b][0..n_active))
+ * and q head h, (A, L) over all tokens of the union pages of kv head h / G,
+ * written over a_out[b, i, h, :] and l_out[b, i, h]. Stable rows are untouched.
+ *  max_union: host upper bound of any union_count entry (the split plan and
+ *             the workspace are sized by it), e.g. min(n_active * G * topk_pages,
+ *             pages per sequence); <= 0 means pages per sequence. Counts above
+ *             it are clamped.
+ */
+int losa_gather(const void* q, int32_t B, int32_t n_heads_q, const int32_t* active_rows,
+                int32_t n_active, const int32_t* union_list, const int32_t* union_count,
+                int32_t max_union, const fb_kv* kv, float scale, float* a_out, float* l_out,
+                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Step controller ([FB] "Adaptive reuse strategies"; [LoSA] steps 1-4).
+ * ------------------------------------------------------------------------- */
+typedef enum { FB_THRESHOLD = 0, FB_PER_HEAD = 1, FB_LOSA = 2 } fb_mode;
+
+typedef struct fb_policy {
+  fb_mode mode;
+  int32_t tau;        /* THRESHOLD: recompute sequence b when m_updated[b] >= tau
+                         (tau <= 0: recompute every step, i.e. dense) */
+  double gamma;       /* PER_HEAD: a head that computed at steps s-1 and s stops
+                         computing for the rest of the block once
+                         cos(A_out^s, A_out^{s-1}) >= gamma (gamma > 1: dense) */
+  int32_t n_active;   /* LOSA: active rows per step */
+  int32_t topk_pages; /* LOSA: pages kept per active row and q head */
+  float scale;        /* softmax scale applied to <q, k> */
+} fb_policy;
+
+/*
+ * Caller-owned state of one (layer, block), reused across its denoise steps.
+ * All arrays are device memory sized for [batch, B, Hq, d] unless noted;
+ * fields a mode does not use may be NULL.
+ */
+typedef struct fb_cache {
+  float* a_out;           /* cached block-external partial A_out */
+  float* l_out;           /* its log normaliser L_out */
+  float* a_out_prev;      /* PER_HEAD: A_out of the previous computing step */
+  uint8_t* head_mask;     /* PER_HEAD: [batch, Hq], 1 = compute at this step */
+  double* head_cos;       /* PER_HEAD: [batch, Hq] last cosine (NaN if none) */
+  void* q_prev;           /* LOSA: previous step's q */
+  int32_t* active_rows;   /* LOSA: [batch, n_active] */
+  float* row_scores;      /* LOSA: [batch, B] (may be NULL) */
+  uint32_t* union_bitmap; /* LOSA: [batch, Hkv, ceil(max_pages/32)] */
+  int32_t* union_list;    /* LOSA: [batch, Hkv, max_pages] */
+  int32_t* union_count;   /* LOSA: [batch, Hkv] */
+  int32_t step;           /* host: index of the next step (0 = block start); fb_step advances it */
+  int32_t recomputed;     /* host: sequences (THRESHOLD) whose prefix partial the last step recomputed */
+} fb_cache;
+
+/*
+ * One denoise step of attention for the block:
+ *   THRESHOLD: sequence b recomputes A_out (fb_prefix_attn) when step == 0 or
+ *              m_updated[b] >= tau, otherwise reuses the cache;
+ *   PER_HEAD:  heads with head_mask = 1 recompute (all heads at steps 0, 1);
+ *              then the cosine per computing head updates head_mask on the
+ *              device (no host round trip);
+ *   LOSA:      step 0 computes the dense prefix partial; later steps run
+ *              losa_select + losa_gather; q is copied into q_prev.
+ * Then the block-internal partial is computed and merged:
+ *   a_full [batch, B, Hq, d] float32, l_full [batch, B, Hq] float32 (may be NULL).
+ *  q, k_in, v_in: this step's block tensors (dtype of prefix->dtype).
+ *  page_min / page_max: fb_page_summary output (LOSA only).
+ *  m_updated: HOST [batch] int32 rows updated since the previous step
+ *             (THRESHOLD only; may be NULL at step 0).
+ */
+int fb_step(const fb_policy* policy, fb_cache* cache, const void* q, const void* k_in,
+            const void* v_in, int32_t B, int32_t n_heads_q, const fb_kv* prefix,
+            const void* page_min, const void* page_max, const int32_t* m_updated, float* a_full,
+            float* l_full, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Reads and clears the device-side error word that bounded waits set when they
+ * give up (SYNCHRONISES the current device). Returns FB_OK or FB_ERR_TIMEOUT.
+ */
+int fb_device_status(void);
+
+/* Text of the calling thread's last error ("" if none). */
+const char* fb_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FB_H_ */

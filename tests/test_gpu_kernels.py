@@ -1,0 +1,260 @@
+"""GPU parity of each C-ABI call against the oracle at sizes that span several
+key tiles, several row tiles and ragged tails (seconds of oracle time).
+
+Sources: FlashBlock technical summary §2 (partials, merge, reuse rules); LoSA
+§2 steps 1-4 (locality score, active set, sparse selection, union).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import block_diffusion_attention_fb_b200 as fb
+import oracle
+from oracle import losa as olosa
+from tests.gpu_util import assert_close_A, assert_close_L, cpu, dev, make_kv, sync
+from workloads import make_workload
+
+pytestmark = pytest.mark.gpu
+
+
+def run_prefix(wl, q_np, head_mask=None):
+    sp = wl.spec
+    kv = make_kv(wl.prefix, sp.dtype)
+    q = dev(q_np, sp.dtype)
+    A = torch.full((sp.batch, sp.block, sp.n_heads_q, sp.head_dim), 7.0, device="cuda")
+    L = torch.full((sp.batch, sp.block, sp.n_heads_q), 7.0, device="cuda")
+    ws = torch.empty(fb.fb_workspace_size(kv, sp.block, sp.n_heads_q), dtype=torch.uint8,
+                     device="cuda")
+    hm = None if head_mask is None else torch.from_numpy(head_mask.astype(np.uint8)).cuda()
+    fb.fb_prefix_attn(q, kv, A, L, ws, head_mask=hm)
+    sync()
+    return cpu(A), cpu(L)
+
+
+PREFIX_CASES = {
+    # name: (workload, overrides)
+    "tiny_full_f32": ("tiny", {}),
+    "tiny_ragged_f32": ("tiny", dict(prefix_min=1001, prefix_max=1001, block=13)),
+    "dllm_small_ragged": ("dllm", dict(prefix_min=1000, prefix_max=1000, n_heads_q=4,
+                                       n_heads_kv=4)),
+    "dllm_block16": ("dllm", dict(prefix_min=777, prefix_max=777, block=16, n_heads_q=2,
+                                  n_heads_kv=2)),
+    "dllm_block1": ("dllm", dict(prefix_min=300, prefix_max=300, block=1, n_heads_q=2,
+                                 n_heads_kv=2)),
+    "gqa_paged_small": ("gqa", dict(prefix_min=100, prefix_max=700, batch=3, block=20,
+                                    n_heads_q=8, n_heads_kv=2)),
+    "gqa_paged_rows_gt_64": ("gqa", dict(prefix_min=50, prefix_max=400, batch=2, block=40,
+                                         n_heads_q=8, n_heads_kv=2)),
+    "video_rows_many_tiles": ("video", dict(prefix_min=500, prefix_max=500, block=150,
+                                            n_heads_q=2, n_heads_kv=2)),
+    "losa_contig_d128": ("losa", dict(prefix_min=2000, prefix_max=2000, n_heads_q=3,
+                                      n_heads_kv=3)),
+    "d64_bf16": ("dllm", dict(prefix_min=600, prefix_max=600, head_dim=64, n_heads_q=2,
+                              n_heads_kv=2)),
+}
+
+
+@pytest.mark.parametrize("case", sorted(PREFIX_CASES))
+def test_prefix_attn_matches_oracle(case):
+    name, ov = PREFIX_CASES[case]
+    wl = make_workload(name, **ov)
+    st = next(wl.steps(1))
+    A, L = run_prefix(wl, st.q)
+    A_ref, L_ref = oracle.prefix_partial(wl.prefix, st.q, wl.spec.dtype)
+    assert_close_A(A, A_ref, wl.spec.dtype, case)
+    assert_close_L(L, L_ref, case)
+
+
+def test_prefix_attn_head_mask_leaves_other_rows():
+    wl = make_workload("gqa", prefix_min=200, prefix_max=300, batch=2, block=8, n_heads_q=8,
+                       n_heads_kv=2)
+    st = next(wl.steps(1))
+    mask = np.zeros((2, 8), dtype=bool)
+    mask[0, 1] = mask[1, 4] = mask[1, 5] = True
+    A, L = run_prefix(wl, st.q, head_mask=mask)
+    A_ref, L_ref = oracle.prefix_partial(wl.prefix, st.q, "bf16")
+    sel = np.broadcast_to(mask[:, None, :], L.shape)
+    assert_close_A(A[sel], A_ref[sel], "bf16")
+    assert_close_L(L[sel], L_ref[sel])
+    assert np.all(A[~sel] == 7.0) and np.all(L[~sel] == 7.0)
+
+
+def test_prefix_attn_empty_and_short_sequences():
+    wl = make_workload("gqa", prefix_min=1, prefix_max=40, batch=4, block=6, n_heads_q=4,
+                       n_heads_kv=2)
+    wl.prefix.seq_len[2] = 0  # an empty prefix: A = 0, L = -inf
+    st = next(wl.steps(1))
+    A, L = run_prefix(wl, st.q)
+    A_ref, L_ref = oracle.prefix_partial(wl.prefix, st.q, "bf16")
+    assert np.all(A[2] == 0) and np.all(np.isneginf(L[2]))
+    assert_close_A(A, A_ref, "bf16")
+    assert_close_L(L, L_ref)
+
+
+@pytest.mark.parametrize("name,ov", [
+    ("tiny", {}),
+    ("dllm", dict(block=32, n_heads_q=4, n_heads_kv=4, prefix_min=64, prefix_max=64)),
+    ("gqa", dict(block=64, batch=2, n_heads_q=8, n_heads_kv=2, prefix_min=64, prefix_max=64)),
+    ("video", dict(block=130, n_heads_q=2, n_heads_kv=2, prefix_min=64, prefix_max=64)),
+    ("dllm", dict(block=5, n_heads_q=2, n_heads_kv=2, prefix_min=64, prefix_max=64)),
+])
+def test_block_attn_matches_oracle(name, ov):
+    wl = make_workload(name, **ov)
+    sp = wl.spec
+    st = next(wl.steps(1))
+    A = torch.zeros(sp.batch, sp.block, sp.n_heads_q, sp.head_dim, device="cuda")
+    L = torch.zeros(sp.batch, sp.block, sp.n_heads_q, device="cuda")
+    fb.fb_block_attn(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L)
+    sync()
+    A_ref, L_ref = oracle.block_partial(st.q, st.k_in, st.v_in, sp.dtype)
+    assert_close_A(cpu(A), A_ref, sp.dtype)
+    assert_close_L(cpu(L), L_ref)
+
+
+def test_merge_matches_oracle_including_empty_sides():
+    rng = np.random.default_rng(0)
+    rows, d = 1000, 128
+    Ao = rng.normal(size=(rows, d)).astype(np.float32)
+    Ai = rng.normal(size=(rows, d)).astype(np.float32)
+    Lo = rng.normal(size=rows).astype(np.float32) * 5
+    Li = rng.normal(size=rows).astype(np.float32) * 5
+    Lo[:10] = -np.inf
+    Li[5:15] = -np.inf
+    Ao[:10] = np.nan  # a side with L = -inf is never read
+    t = lambda x: torch.from_numpy(x).cuda()  # noqa: E731
+    Af = torch.zeros(rows, d, device="cuda")
+    Lf = torch.zeros(rows, device="cuda")
+    fb.fb_merge(t(Ao), t(Lo), t(Ai), t(Li), Af, Lf)
+    sync()
+    Ao64 = np.where(np.isnan(Ao), 0.0, Ao)
+    A_ref, L_ref = oracle.merge(Ao64, Lo, Ai, Li)
+    np.testing.assert_allclose(cpu(Af), A_ref, rtol=0, atol=2e-6)
+    assert_close_L(cpu(Lf), L_ref)
+    assert np.all(cpu(Af)[5:10] == 0)
+
+
+def _losa_small(**kw):
+    args = dict(prefix_min=3001, prefix_max=3001, block=16, n_heads_q=4, n_heads_kv=4)
+    args.update(kw)
+    return make_workload("losa", **args)
+
+
+def _bf16_bits(t):
+    return cpu(t.view(torch.int16)).view(np.uint16)
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_page_summary_is_exact(paged):
+    if paged:
+        wl = make_workload("gqa", prefix_min=100, prefix_max=600, batch=3, block=4, n_heads_q=4,
+                           n_heads_kv=2)
+    else:
+        wl = _losa_small()
+    kv = make_kv(wl.prefix, "bf16")
+    npg = kv.n_pages
+    pmin = torch.empty(kv.batch, npg, kv.c.n_heads_kv, 128, dtype=torch.bfloat16, device="cuda")
+    pmax = torch.empty_like(pmin)
+    fb.fb_page_summary(kv, pmin, pmax)
+    sync()
+    smin, smax = olosa.page_summary(wl.prefix, "bf16")
+    gmin = cpu(pmin.float())
+    gmax = cpu(pmax.float())
+    for b in range(kv.batch):
+        n = -(-int(wl.prefix.seq_len[b]) // 16)
+        np.testing.assert_array_equal(gmin[b, :n], smin[b, :n])
+        np.testing.assert_array_equal(gmax[b, :n], smax[b, :n])
+
+
+def run_select(wl, q_cur, q_prev, n_active, topk):
+    sp = wl.spec
+    kv = make_kv(wl.prefix, sp.dtype)
+    npg, hkv = kv.n_pages, sp.n_heads_kv
+    pmin = torch.empty(kv.batch, npg, hkv, sp.head_dim, dtype=torch.bfloat16, device="cuda")
+    pmax = torch.empty_like(pmin)
+    fb.fb_page_summary(kv, pmin, pmax)
+    na = min(n_active, sp.block)
+    act = torch.full((sp.batch, max(na, 1)), -1, dtype=torch.int32, device="cuda")
+    rs = torch.zeros(sp.batch, sp.block, device="cuda")
+    bm = torch.zeros(sp.batch, hkv, -(-npg // 32), dtype=torch.int32, device="cuda")
+    ul = torch.full((sp.batch, hkv, npg), -1, dtype=torch.int32, device="cuda")
+    uc = torch.zeros(sp.batch, hkv, dtype=torch.int32, device="cuda")
+    ws = torch.empty(fb.fb_workspace_size(kv, sp.block, sp.n_heads_q, n_active, topk),
+                     dtype=torch.uint8, device="cuda")
+    fb.losa_select(dev(q_cur, "bf16"), dev(q_prev, "bf16"), pmin, pmax, kv, n_active, topk, act,
+                   bm, ul, uc, ws, row_scores=rs)
+    sync()
+    return kv, act, rs, bm, ul, uc, ws
+
+
+@pytest.mark.parametrize("ov,n_active,topk", [
+    ({}, 4, 20),
+    (dict(prefix_min=999, prefix_max=999), 3, 7),
+    (dict(n_heads_q=4, n_heads_kv=2), 2, 9),
+    ({}, 4, 1000),       # top-k larger than the page count: every page
+    ({}, 40, 5),         # more active rows than block rows: all rows
+])
+def test_losa_select_is_bit_exact(ov, n_active, topk):
+    wl = _losa_small(**ov)
+    steps = list(wl.steps(2))
+    q_prev, q_cur = steps[0].q, steps[1].q
+    kv, act, rs, bm, ul, uc, _ = run_select(wl, q_cur, q_prev, n_active, topk)
+    score = olosa.locality_score(q_cur, q_prev, "bf16")
+    np.testing.assert_array_equal(cpu(rs), score)  # bit-exact float32 tree
+    act_ref = olosa.active_rows(score, n_active)
+    np.testing.assert_array_equal(cpu(act)[:, :act_ref.shape[1]], act_ref)
+    smin, smax = olosa.page_summary(wl.prefix, "bf16")
+    _, union = olosa.select_pages(wl.prefix, q_cur, "bf16", act_ref, topk, smin, smax)
+    npg = kv.n_pages
+    bm_ref = olosa.union_bitmap(union, kv.batch, kv.c.n_heads_kv, npg)
+    np.testing.assert_array_equal(cpu(bm).view(np.uint32), bm_ref)
+    for (b, hk), pages in union.items():
+        assert int(cpu(uc)[b, hk]) == len(pages)
+        np.testing.assert_array_equal(cpu(ul)[b, hk, :len(pages)], pages)
+
+
+def test_losa_gather_matches_oracle():
+    wl = _losa_small(n_heads_q=4, n_heads_kv=2)
+    steps = list(wl.steps(2))
+    q_prev, q_cur = steps[0].q, steps[1].q
+    n_active, topk = 3, 11
+    kv, act, rs, bm, ul, uc, ws = run_select(wl, q_cur, q_prev, n_active, topk)
+    A = torch.full((1, 16, 4, 128), 5.0, device="cuda")
+    L = torch.full((1, 16, 4), 5.0, device="cuda")
+    fb.losa_gather(dev(q_cur, "bf16"), act, n_active, ul, uc, kv, A, L, ws,
+                   max_union=n_active * 2 * topk)
+    sync()
+    act_ref = olosa.active_rows(olosa.locality_score(q_cur, q_prev, "bf16"), n_active)
+    smin, smax = olosa.page_summary(wl.prefix, "bf16")
+    _, union = olosa.select_pages(wl.prefix, q_cur, "bf16", act_ref, topk, smin, smax)
+    ref = olosa.sparse_partial(wl.prefix, q_cur, "bf16", act_ref, union)
+    A, L = cpu(A), cpu(L)
+    got_A = np.stack([A[b, i, h] for (b, i, h) in ref])
+    want_A = np.stack([v[0] for v in ref.values()])
+    assert_close_A(got_A, want_A, "bf16")
+    assert_close_L(np.array([L[k] for k in ref]), np.array([v[1] for v in ref.values()]))
+    stable = np.ones(16, dtype=bool)
+    stable[act_ref[0]] = False
+    assert np.all(A[0, stable] == 5.0) and np.all(L[0, stable] == 5.0)
+
+
+def test_invalid_arguments_are_rejected_on_the_host():
+    wl = make_workload("dllm", prefix_min=128, prefix_max=128, n_heads_q=2, n_heads_kv=2)
+    kv = make_kv(wl.prefix, "bf16")
+    q = dev(next(wl.steps(1)).q, "bf16")
+    A = torch.zeros(1, 32, 2, 128, device="cuda")
+    L = torch.zeros(1, 32, 2, device="cuda")
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(fb.FbError) as e:
+        fb.fb_prefix_attn(q, kv, A, L, ws)  # workspace far too small
+    assert e.value.code == fb.FB_ERR_WORKSPACE
+    bad = make_kv(wl.prefix, "bf16")
+    bad.c.head_dim = 96
+    with pytest.raises(fb.FbError) as e:
+        fb.fb_prefix_attn(q, bad, A, L, ws)
+    assert e.value.code == fb.FB_ERR_SHAPE
+    q3 = torch.zeros(1, 32, 3, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(fb.FbError) as e:
+        fb.fb_prefix_attn(q3, kv, A, L, ws)  # 3 q heads cannot share 2 kv heads
+    assert e.value.code == fb.FB_ERR_SHAPE
+    fb.fb_device_status()

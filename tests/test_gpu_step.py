@@ -1,0 +1,138 @@
+"""GPU parity of fb_step (the reuse controllers) against the oracle's step
+procedures, step by step over whole blocks at reduced sizes.
+
+FlashBlock technical summary §2 "Adaptive reuse strategies" (threshold tau,
+per-head gamma); LoSA §2 steps 1-4.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from block_diffusion_attention_fb_b200.runtime import BlockAttention
+from oracle.controllers import (LosaController, PerHeadController, ThresholdController,
+                                head_cosine)
+from tests.gpu_util import assert_close_A, assert_close_L, cpu, dev, make_kv, sync
+from workloads import make_workload
+
+pytestmark = pytest.mark.gpu
+
+
+def _out(sp):
+    A = torch.zeros(sp.batch, sp.block, sp.n_heads_q, sp.head_dim, device="cuda")
+    L = torch.zeros(sp.batch, sp.block, sp.n_heads_q, device="cuda")
+    return A, L
+
+
+@pytest.mark.parametrize("name,ov,tau", [
+    ("tiny", {}, 3),
+    ("tiny", {}, 0),
+    ("dllm", dict(prefix_min=900, prefix_max=900, n_heads_q=4, n_heads_kv=4, steps=12), 2),
+    ("gqa", dict(prefix_min=100, prefix_max=500, batch=3, block=16, n_heads_q=8, n_heads_kv=2,
+                 steps=10), 3),
+])
+def test_threshold_steps_match_oracle(name, ov, tau):
+    wl = make_workload(name, **ov)
+    sp = wl.spec
+    kv = make_kv(wl.prefix, sp.dtype)
+    blk = BlockAttention(kv, sp.block, sp.n_heads_q, "threshold", tau=tau)
+    ctl = ThresholdController(wl.prefix, sp.dtype, tau)
+    A, L = _out(sp)
+    n_rec = 0
+    for st in wl.steps():
+        blk.step(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L,
+                 m_updated=st.m_updated)
+        ref = ctl.step(st.step, st.q, st.k_in, st.v_in, st.m_updated)
+        sync()
+        assert blk.recomputed == int(ref["recompute"].sum()), f"step {st.step}"
+        n_rec += blk.recomputed
+        assert_close_A(cpu(A), ref["A_full"], sp.dtype, f"step {st.step}")
+        assert_close_L(cpu(L), ref["L_full"], f"step {st.step}")
+    assert blk.step_index == sp.steps
+    if tau == 0:
+        assert n_rec == sp.steps * sp.batch
+
+
+def test_per_head_steps_match_oracle_with_bit_exact_cosine_replay():
+    wl = make_workload("video", prefix_min=700, prefix_max=700, block=90, n_heads_q=6,
+                       n_heads_kv=6, steps=8)
+    sp = wl.spec
+    # cosines of this case lie in [0.959, 0.9994]: 0.997 stops two heads at
+    # step 1 and keeps the others computing, each with a margin above 1e-3
+    gamma = 0.997
+    kv = make_kv(wl.prefix, sp.dtype)
+    blk = BlockAttention(kv, sp.block, sp.n_heads_q, "per_head", gamma=gamma)
+    ctl = PerHeadController(wl.prefix, sp.dtype, gamma)
+    A, L = _out(sp)
+    prev_gpu_aout = None
+    stopped_any = False
+    for st in wl.steps():
+        mask_before = cpu(blk.t["head_mask"]).astype(bool)
+        blk.step(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L)
+        sync()
+        gpu_aout = cpu(blk.a_out).copy()
+        # teacher forcing: the oracle computes exactly the heads the GPU computed
+        ref = ctl.step(st.step, st.q, st.k_in, st.v_in, force_mask=mask_before,
+                       a_out_for_decision=(gpu_aout, prev_gpu_aout))
+        if st.step >= 1:
+            cos_gpu = cpu(blk.t["head_cos"])
+            for h in range(sp.n_heads_q):
+                if mask_before[0, h]:
+                    # replay: the oracle's cosine on the GPU's own float32 tiles
+                    want = head_cosine(gpu_aout[0, :, h], cpu(blk.t["a_out_prev"])[0, :, h])
+                    assert cos_gpu[0, h] == want, (st.step, h, cos_gpu[0, h], want)
+                    assert ref["cos"][0, h] == want
+            np.testing.assert_array_equal(cpu(blk.t["head_mask"]).astype(bool), ref["next_mask"])
+            stopped_any |= bool((~ref["next_mask"]).any())
+        assert_close_A(cpu(A), ref["A_full"], sp.dtype, f"step {st.step}")
+        assert_close_L(cpu(L), ref["L_full"], f"step {st.step}")
+        prev_gpu_aout = gpu_aout
+    assert stopped_any, "gamma chosen so that some heads start reusing"
+
+
+def test_per_head_oracle_mask_agrees_away_from_the_threshold():
+    """End to end: the oracle's own float64 A_out gives the same decisions as
+    the GPU wherever |c - gamma| > 1e-4."""
+    wl = make_workload("video", prefix_min=400, prefix_max=400, block=60, n_heads_q=4,
+                       n_heads_kv=4, steps=6)
+    sp = wl.spec
+    gamma = 0.999
+    kv = make_kv(wl.prefix, sp.dtype)
+    blk = BlockAttention(kv, sp.block, sp.n_heads_q, "per_head", gamma=gamma)
+    ctl = PerHeadController(wl.prefix, sp.dtype, gamma)
+    A, L = _out(sp)
+    for st in wl.steps():
+        mask_before = cpu(blk.t["head_mask"]).astype(bool)
+        blk.step(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L)
+        sync()
+        ref = ctl.step(st.step, st.q, st.k_in, st.v_in, force_mask=mask_before)
+        if st.step >= 1:
+            cos_gpu = cpu(blk.t["head_cos"])
+            for h in range(sp.n_heads_q):
+                if mask_before[0, h] and abs(ref["cos"][0, h] - gamma) > 1e-4:
+                    assert (cos_gpu[0, h] >= gamma) == (ref["cos"][0, h] >= gamma)
+
+
+@pytest.mark.parametrize("ov,n_active,topk", [
+    (dict(prefix_min=3000, prefix_max=3000, n_heads_q=4, n_heads_kv=4, steps=6), 4, 16),
+    (dict(prefix_min=2500, prefix_max=2500, n_heads_q=4, n_heads_kv=2, steps=5, block=20), 3, 9),
+])
+def test_losa_steps_match_oracle(ov, n_active, topk):
+    wl = make_workload("losa", **ov)
+    sp = wl.spec
+    kv = make_kv(wl.prefix, sp.dtype)
+    blk = BlockAttention(kv, sp.block, sp.n_heads_q, "losa", n_active=n_active, topk_pages=topk)
+    ctl = LosaController(wl.prefix, sp.dtype, n_active, topk)
+    A, L = _out(sp)
+    for st in wl.steps():
+        blk.step(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L)
+        ref = ctl.step(st.step, st.q, st.k_in, st.v_in)
+        sync()
+        if st.step >= 1:
+            np.testing.assert_array_equal(cpu(blk.t["active_rows"]), ref["active"])
+            for (b, hk), pages in ref["union"].items():
+                cnt = int(cpu(blk.t["union_count"])[b, hk])
+                assert cnt == len(pages)
+                np.testing.assert_array_equal(cpu(blk.t["union_list"])[b, hk, :cnt], pages)
+        assert_close_A(cpu(A), ref["A_full"], sp.dtype, f"step {st.step}")
+        assert_close_L(cpu(L), ref["L_full"], f"step {st.step}")
