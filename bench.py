@@ -1,0 +1,487 @@
+#!/usr/bin/env python
+"""Per-denoise-step block-diffusion attention benchmark (FlashBlock / LoSA).
+
+Workload: the dLLM configuration (bf16, batch 1, 32 heads MHA, d=128, frozen
+prefix of 32768 tokens, block of 32 tokens denoised over 32 steps, Poisson(2)
+row updates per step, tau=4), synthetic and seeded. One bench step is one
+whole block: 32 denoise steps of attention (prefix partial when needed,
+block partial, merge). Inputs are resident in HBM before timing; L2 is flushed
+(256 MiB write) between denoise steps, outside the timed events.
+
+Modes, each timed over the same K blocks:
+  reuse  FlashBlock threshold reuse (tau=4) through fb_step: the headline value
+  dense  prefix partial every step (fb_prefix_attn + fb_block_attn + fb_merge)
+  losa   LoSA (4 active rows, top-256 of 2048 pages) through fb_step
+
+value = microseconds per denoise step of the whole job (max over ranks of the
+device time / denoise steps of all ranks). With N GPUs every rank runs its own
+replica (weak scaling; the path has no exchange step).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "µs per denoise-step attention & prefix HBM GB/s (dense vs reuse vs LoSA)"
+UNIT = "µs"
+WORKLOAD = ("dllm: bf16, batch 1, 32 heads MHA, head_dim 128, prefix 32768 tokens, block 32, "
+            "32 denoise steps per block, Poisson(2) updates, tau 4; LoSA 4 active rows, top-256 pages")
+FLUSH_BYTES = 256 << 20
+LOSA_ACTIVE, LOSA_TOPK = 4, 256
+ORACLE_HEADS = 4  # oracle sample: this many of the 32 heads, scaled to all heads
+BASELINE_HEADS, BASELINE_BLOCKS = 8, 2  # CPU baseline sample of our arm (about 10 s)
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20, help="timed blocks of 32 denoise steps")
+    p.add_argument("--warmup", type=int, default=3, help="untimed blocks before timing")
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--mode", choices=["all", "reuse", "dense", "losa"], default="all",
+                   help="all: the contract line; one mode: time only that mode (for profiling)")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; only barriers and a MAX reduce)
+# ---------------------------------------------------------------------------
+def dist_init(n_gpus):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    import torch
+    import torch.distributed as dist
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [r for r in rows if r[2] > 250.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i in range(4) if r[3][i].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in load),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(load)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def kernel_source_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "block_diffusion_attention_fb_b200", "csrc")
+    for name in sorted(os.listdir(d)):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """dram bytes per launch of the prefix call from the committed ncu summary,
+    if it was taken on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "prefix_attn_dllm_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    for line in open(path):
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    if kv.get("kernel_sources_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return int(kv["dram_bytes_per_call"])
+    except (KeyError, ValueError):
+        return None
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        try:
+            return float(json.load(open(path))["hbm_gbs"]), "measured"
+        except (ValueError, KeyError):
+            pass
+    return 6650.0, "fallback"
+
+
+def run_ours(args, rank, world, local):
+    import numpy as np
+    import torch
+
+    import block_diffusion_attention_fb_b200 as fb
+    from block_diffusion_attention_fb_b200.runtime import BlockAttention
+    from workloads import make_workload
+    from workloads.torch_io import prefix_tensors, to_torch
+
+    fb.load_library()
+    wl = make_workload("dllm")
+    sp = wl.spec
+    S = sp.steps
+    t = prefix_tensors(wl.prefix, sp.dtype)
+    kv = fb.KV(t["k"], t["v"], seq_len=t["seq_len"], page_table=t["page_table"],
+               page_size=t["page_size"], max_seq_len=t["max_seq_len"])
+    steps = list(wl.steps())
+    dq = [to_torch(s.q, "bf16") for s in steps]
+    dk = [to_torch(s.k_in, "bf16") for s in steps]
+    dv = [to_torch(s.v_in, "bf16") for s in steps]
+    hq = [to_torch(s.q, "bf16", "cpu", pin=True) for s in steps]
+    hk = [to_torch(s.k_in, "bf16", "cpu", pin=True) for s in steps]
+    hv = [to_torch(s.v_in, "bf16", "cpu", pin=True) for s in steps]
+    ms = [s.m_updated.tolist() for s in steps]
+    B, Hq, d = sp.block, sp.n_heads_q, sp.head_dim
+    A = torch.zeros(1, B, Hq, d, device="cuda")
+    L = torch.zeros(1, B, Hq, device="cuda")
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    reuse = BlockAttention(kv, B, Hq, "threshold", tau=sp.tau)
+    losa = BlockAttention(kv, B, Hq, "losa", n_active=LOSA_ACTIVE, topk_pages=LOSA_TOPK)
+    a_out = torch.zeros(1, B, Hq, d, device="cuda")
+    l_out = torch.zeros(1, B, Hq, device="cuda")
+    a_in = torch.zeros_like(a_out)
+    l_in = torch.zeros_like(l_out)
+    ws = torch.empty(fb.fb_workspace_size(kv, B, Hq), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    def timed_blocks(n_blocks, one_step, timed, extra=None):
+        """Runs n_blocks blocks of S denoise steps; returns device ms of the steps."""
+        pairs, extra_pairs = [], []
+        for blk_i in range(n_blocks):
+            for s in range(S):
+                flush.zero_()
+                e0, e1 = ev(), ev()
+                if timed:
+                    e0.record(stream)
+                x = one_step(s, extra_pairs if timed else None)
+                if timed:
+                    e1.record(stream)
+                    pairs.append((e0, e1))
+        torch.cuda.synchronize()
+        total = sum(a.elapsed_time(b) for a, b in pairs)
+        ext = [a.elapsed_time(b) for a, b in extra_pairs]
+        return total, ext
+
+    def reuse_step(s, _):
+        if s == 0:
+            reuse.reset()
+        reuse.step(dq[s], dk[s], dv[s], A, L, m_updated=ms[s])
+        return reuse.recomputed
+
+    def dense_step(s, extra):
+        if extra is not None:
+            p0, p1 = ev(), ev()
+            p0.record(stream)
+        fb.fb_prefix_attn(dq[s], kv, a_out, l_out, ws)
+        if extra is not None:
+            p1.record(stream)
+            extra.append((p0, p1))
+        fb.fb_block_attn(dq[s], dk[s], dv[s], a_in, l_in)
+        fb.fb_merge(a_out, l_out, a_in, l_in, A, L)
+
+    def losa_step(s, _):
+        if s == 0:
+            losa.reset()
+        losa.step(dq[s], dk[s], dv[s], A, L)
+
+    hA = torch.empty(1, B, Hq, d, dtype=torch.float32).pin_memory()
+    hL = torch.empty(1, B, Hq, dtype=torch.float32).pin_memory()
+    qd, kd, vd = torch.empty_like(dq[0]), torch.empty_like(dk[0]), torch.empty_like(dv[0])
+
+    def e2e_step(s, _):
+        if s == 0:
+            reuse.reset()
+        qd.copy_(hq[s], non_blocking=True)
+        kd.copy_(hk[s], non_blocking=True)
+        vd.copy_(hv[s], non_blocking=True)
+        reuse.step(qd, kd, vd, A, L, m_updated=ms[s])
+        hA.copy_(A, non_blocking=True)
+        hL.copy_(L, non_blocking=True)
+
+    K, W = args.steps, args.warmup
+    if args.mode != "all":
+        fn = {"reuse": reuse_step, "dense": dense_step, "losa": losa_step}[args.mode]
+        timed_blocks(W, fn, False)
+        barrier(world)
+        t_mode, _ = timed_blocks(K, fn, True)
+        barrier(world)
+        fb.fb_device_status()
+        if rank == 0:
+            print(json.dumps({"mode": args.mode, "us_per_step": t_mode * 1000 / (K * S)}))
+        return
+    clocks = ClockSampler(local)
+    # warm-up of every path (untimed)
+    for fn in (reuse_step, dense_step, losa_step, e2e_step):
+        timed_blocks(W, fn, False)
+    barrier(world)
+    clocks.start()
+    barrier(world)
+    n0 = fb.fb_kernel_launches()
+    t_reuse, _ = timed_blocks(K, reuse_step, True)
+    launches = fb.fb_kernel_launches() - n0
+    barrier(world)
+    rec = 0
+    for s in range(S):  # recompute decisions of one block (identical every block)
+        rec += int(s == 0 or ms[s][0] >= sp.tau)
+    t_dense, prefix_ms = timed_blocks(K, dense_step, True)
+    barrier(world)
+    t_losa, _ = timed_blocks(K, losa_step, True)
+    barrier(world)
+    t_e2e, _ = timed_blocks(K, e2e_step, True)
+    barrier(world)
+    clk = clocks.stop()
+    fb.fb_device_status()
+
+    n_steps_all = K * S * world
+    t_reuse_max = max_over_ranks(t_reuse, world)
+    t_dense_max = max_over_ranks(t_dense, world)
+    t_losa_max = max_over_ranks(t_losa, world)
+    t_e2e_max = max_over_ranks(t_e2e, world)
+    us = lambda ms_total: ms_total * 1000.0 / n_steps_all  # noqa: E731
+
+    # roofline of the dominant kernel call: the dense prefix partial
+    kv_bytes = 2 * int(wl.prefix.seq_len.sum()) * sp.n_heads_kv * d * 2
+    io_bytes = B * Hq * d * 2 + B * Hq * (d + 1) * 4
+    alg_bytes = kv_bytes + io_bytes
+    prefix_avg_ms = statistics.mean(prefix_ms)
+    achieved = alg_bytes / (prefix_avg_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peak()
+    traffic = profiled_traffic()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC,
+        "value": round(us(t_reuse_max), 3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(t_reuse_max / K, 4),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded generator; no model weights or datasets)",
+        "config": {
+            "workload": WORKLOAD,
+            "global_batch": world,
+            "seq_len": int(wl.prefix.max_seq_len),
+            "block": B,
+            "denoise_steps_per_bench_step": S,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "flushed between denoise steps (256 MiB write, outside the timed events)",
+            "value_mode": "reuse (FlashBlock threshold, tau=4) through fb_step",
+        },
+        "modes": {
+            "reuse": {"us_per_step": round(us(t_reuse_max), 3),
+                      "prefix_recomputes_per_block": rec},
+            "dense": {"us_per_step": round(us(t_dense_max), 3),
+                      "prefix_call_us": round(prefix_avg_ms * 1000, 3),
+                      "prefix_gbs": round(achieved, 1)},
+            "losa": {"us_per_step": round(us(t_losa_max), 3), "n_active": LOSA_ACTIVE,
+                     "topk_pages": LOSA_TOPK},
+        },
+        "tokens_per_s": round(world * K * B / (t_reuse_max * 1e-3), 1),
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "fb_prefix_attn (split-KV attention + combine), dense dllm prefix",
+            "achieved": round(achieved, 1),
+            "peak": peak,
+            "peak_kind": f"{peak_kind} (copy bandwidth, burst)",
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "algorithmic_bytes_per_call": alg_bytes,
+            "traffic": traffic,
+        },
+        "e2e": {
+            "value": round(us(t_e2e_max), 3),
+            "unit": UNIT,
+            "h2d_bytes_per_step": 3 * B * Hq * d * 2 * S,
+            "d2h_bytes_per_step": (B * Hq * d * 4 + B * Hq * 4) * S,
+            "api": "fb_step (reuse) with q/k/v copied from pinned host memory and A_full/L_full "
+                   "copied back every denoise step",
+        },
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_baseline(wl)
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# oracle on the host cores (the reference arm and the CPU baseline)
+# ---------------------------------------------------------------------------
+class _HeadSlice:
+    """The first n heads of a prefix cache (a bounded sample of the workload)."""
+
+    def __init__(self, prefix, n):
+        self.k = prefix.k[:, :n]
+        self.v = prefix.v[:, :n]
+        self.seq_len = prefix.seq_len
+        self.page_table = prefix.page_table
+        self.page_size = prefix.page_size
+        self.max_seq_len = prefix.max_seq_len
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max(int(i.get("num_threads", 1)) for i in threadpool_info()) or 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_blocks(wl, blocks, steps_cache=None, n=ORACLE_HEADS):
+    """Wall-clock seconds of `blocks` oracle blocks (threshold reuse) on the
+    first n heads, scaled to all heads."""
+    from oracle.controllers import ThresholdController
+    sp = wl.spec
+    sub = _HeadSlice(wl.prefix, n)
+    steps = steps_cache if steps_cache is not None else list(wl.steps())
+    total = 0.0
+    for _ in range(blocks):
+        ctl = ThresholdController(sub, sp.dtype, sp.tau)
+        t0 = time.perf_counter()
+        for st in steps:
+            ctl.step(st.step, st.q[:, :, :n], st.k_in[:, :, :n], st.v_in[:, :, :n], st.m_updated)
+        total += time.perf_counter() - t0
+    return total * (sp.n_heads_q / n)
+
+
+def oracle_baseline(wl, blocks=BASELINE_BLOCKS, n=BASELINE_HEADS):
+    secs = oracle_blocks(wl, blocks, n=n)
+    per_step_us = secs * 1e6 / (blocks * wl.spec.steps)
+    return {"value": round(per_step_us, 1), "unit": UNIT, "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{blocks} block(s) of {wl.spec.steps} denoise steps, threshold reuse "
+                      f"(tau={wl.spec.tau}), {n} of {wl.spec.n_heads_q} heads, time "
+                      f"scaled by {wl.spec.n_heads_q // n} to all heads; float64 numpy"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from workloads import make_workload
+    wl = make_workload("dllm")
+    steps = list(wl.steps())
+    oracle_blocks(wl, args.warmup, steps)
+    secs = oracle_blocks(wl, args.steps, steps)
+    value = secs * 1e6 / (args.steps * wl.spec.steps)
+    cpu = {"value": round(value, 1), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+           "sample": f"each bench step: one block of {wl.spec.steps} denoise steps of the oracle "
+                     f"(threshold reuse, tau={wl.spec.tau}) on {ORACLE_HEADS} of "
+                     f"{wl.spec.n_heads_q} heads, scaled to all heads"}
+    line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(secs * 1000 / args.steps, 3), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": 1, "seq_len": 32768,
+                       "parallelism": "host cores"},
+            "impl": "reference", "cpu_baseline": cpu,
+            "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        run_reference(args, rank, world)
+        return
+    rank, world, local = dist_init(args.gpus)
+    try:
+        run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

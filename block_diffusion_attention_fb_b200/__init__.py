@@ -32,7 +32,8 @@ FB_LOSA = 2
 
 # Every entry point include/fb.h declares.
 EXPORTS = ("fb_workspace_size", "fb_prefix_attn", "fb_block_attn", "fb_merge", "fb_page_summary",
-           "losa_select", "losa_gather", "fb_step", "fb_device_status", "fb_last_error")
+           "losa_select", "losa_gather", "fb_step", "fb_device_status", "fb_last_error",
+           "fb_kernel_launches")
 
 
 class FbError(RuntimeError):
@@ -92,6 +93,7 @@ def load_library() -> ctypes.CDLL:
                                    I32, KV, P, P, P, P, P, P, SZ, P]),
         "fb_device_status": (ctypes.c_int, []),
         "fb_last_error": (ctypes.c_char_p, []),
+        "fb_kernel_launches": (ctypes.c_uint64, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -245,3 +247,7 @@ def fb_device_status() -> None:
 
 def fb_last_error() -> str:
     return load_library().fb_last_error().decode()
+
+
+def fb_kernel_launches() -> int:
+    return int(load_library().fb_kernel_launches())

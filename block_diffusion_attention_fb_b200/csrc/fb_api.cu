@@ -4,6 +4,7 @@
 // and cosine.cuh; this file only decides what to launch.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -20,6 +21,7 @@ namespace {
 using namespace fb;
 
 thread_local std::string g_last_error;
+std::atomic<unsigned long long> g_launches{0};  // kernels launched by this library
 
 int fail(int code, const char* fmt, ...) {
   char buf[512];
@@ -34,6 +36,7 @@ int fail(int code, const char* fmt, ...) {
 int check_launch(const char* what) {
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(FB_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   return FB_OK;
 }
 
@@ -400,6 +403,8 @@ extern "C" {
 
 const char* fb_last_error(void) { return g_last_error.c_str(); }
 
+uint64_t fb_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
 int fb_device_status(void) {
   int word = 0, zero = 0;
   if (cudaDeviceSynchronize() != cudaSuccess) return fail(FB_ERR_CUDA, "device synchronize failed");
@@ -520,7 +525,8 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
     // no active rows: an empty union (the bitmap and counts still get written)
     cudaMemsetAsync(union_bitmap, 0, (size_t)kv->batch * v.Hkv * words * 4, stream);
     cudaMemsetAsync(union_count, 0, (size_t)kv->batch * v.Hkv * 4, stream);
-    return check_launch("losa_select memset");
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? FB_OK : fail(FB_ERR_CUDA, "losa_select memset: %s", cudaGetErrorString(e));
   }
   const dim3 g1(B, kv->batch);
   if (N2 * 4 > 48 * 1024) {
@@ -660,9 +666,8 @@ int fb_step(const fb_policy* policy, fb_cache* cache, const void* q, const void*
     if (!cache->head_mask || !cache->a_out_prev || !cache->head_cos)
       return fail(FB_ERR_ARG, "PER_HEAD needs head_mask, a_out_prev and head_cos");
     if (s == 0) {
-      cudaMemsetAsync(cache->head_mask, 1, (size_t)batch * Hq, stream);
-      rc = check_launch("head mask reset");
-      if (rc) return rc;
+      if (cudaMemsetAsync(cache->head_mask, 1, (size_t)batch * Hq, stream) != cudaSuccess)
+        return fail(FB_ERR_CUDA, "head mask reset failed");
     }
     c.head_mask = cache->head_mask;
     c.a_prev = cache->a_out_prev;

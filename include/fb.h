@@ -246,6 +246,9 @@ int fb_device_status(void);
 /* Text of the calling thread's last error ("" if none). */
 const char* fb_last_error(void);
 
+/* Number of kernels this library has launched in this process (all threads). */
+uint64_t fb_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif
