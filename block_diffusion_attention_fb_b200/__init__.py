@@ -33,7 +33,7 @@ FB_LOSA = 2
 # Every entry point include/fb.h declares.
 EXPORTS = ("fb_workspace_size", "fb_prefix_attn", "fb_block_attn", "fb_merge", "fb_page_summary",
            "losa_select", "losa_gather", "fb_step", "fb_device_status", "fb_last_error",
-           "fb_kernel_launches")
+           "fb_kernel_launches", "fb_prefix_attn_noalloc")
 
 
 class FbError(RuntimeError):
@@ -94,6 +94,7 @@ def load_library() -> ctypes.CDLL:
         "fb_device_status": (ctypes.c_int, []),
         "fb_last_error": (ctypes.c_char_p, []),
         "fb_kernel_launches": (ctypes.c_uint64, []),
+        "fb_prefix_attn_noalloc": (ctypes.c_int, [P, I32, I32, F32, KV, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -247,6 +248,16 @@ def fb_device_status() -> None:
 
 def fb_last_error() -> str:
     return load_library().fb_last_error().decode()
+
+
+def fb_prefix_attn_noalloc(q, kv: KV, a_out, l_out, scale: float = 1.0, head_mask=None,
+                           stream=None) -> None:
+    """fb_prefix_attn with the library's static scratch instead of a workspace
+    (for callers that cannot allocate device memory; see include/fb.h)."""
+    batch, B, Hq, d = q.shape
+    _check(load_library().fb_prefix_attn_noalloc(_ptr(q), B, Hq, scale, ctypes.byref(kv.c),
+                                                 _ptr(head_mask), _ptr(a_out), _ptr(l_out),
+                                                 _stream(stream)))
 
 
 def fb_kernel_launches() -> int:

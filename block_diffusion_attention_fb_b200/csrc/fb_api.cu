@@ -6,6 +6,7 @@
 
 #include <atomic>
 #include <cmath>
+#include <mutex>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -15,6 +16,12 @@
 #include "attn.cuh"
 #include "cosine.cuh"
 #include "losa.cuh"
+
+// Scratch of fb_prefix_attn_noalloc: a fixed device array that every GPU which
+// loads this library keeps for the life of the process. Host code may not use
+// this name as a pointer (it is a host-side stand-in); the device address comes
+// from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char g_fb_noalloc_scratch[FB_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 
@@ -724,6 +731,65 @@ int fb_step(const fb_policy* policy, fb_cache* cache, const void* q, const void*
   if (rc) return rc;
   cache->step = s + 1;
   return FB_OK;
+}
+
+// Device address of g_fb_noalloc_scratch on the current device, looked up on
+// the first call made with that device current and remembered afterwards.
+static int noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[256] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256)
+    return fail(FB_ERR_CUDA, "fb_prefix_attn_noalloc: no current device");
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_fb_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(FB_ERR_CUDA, "fb_prefix_attn_noalloc: cudaGetSymbolAddress failed: %s",
+                  cudaGetErrorString(e));
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return FB_OK;
+}
+
+int fb_prefix_attn_noalloc(const void* q, int32_t B, int32_t n_heads_q, float scale,
+                           const fb_kv* kv, const uint8_t* head_mask, float* a_out, float* l_out,
+                           cudaStream_t stream) {
+  int rc = validate_kv(kv);
+  if (rc) return rc;
+  rc = validate_q(q, B, n_heads_q, kv);
+  if (rc) return rc;
+  if (!a_out || !l_out) return fail(FB_ERR_ARG, "a_out / l_out is NULL");
+  const int num_sms = sm_count();
+  const int R = B * (n_heads_q / kv->n_heads_kv);
+  const Plan p = make_plan(kv->dtype, kv->batch, kv->n_heads_kv, R, ceil_div(kv->max_seq_len, kTK),
+                           num_sms);
+  const size_t need = partial_bytes(p, kv->batch, kv->n_heads_kv, R, kv->head_dim);
+  if (need > (size_t)FB_NOALLOC_SCRATCH_BYTES)
+    return fail(FB_ERR_WORKSPACE,
+                "fb_prefix_attn_noalloc: these shapes need %zu bytes of scratch but the static "
+                "buffer holds %zu; use fb_prefix_attn with a workspace",
+                need, (size_t)FB_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc) return rc;
+  // Nothing in the scratch has to start at zero: every split writes its partial
+  // (or an empty-partial marker) before the combine reads it.
+  PartialCall c{};
+  c.q = q;
+  c.B = B;
+  c.Hq = n_heads_q;
+  c.scale = scale;
+  c.kv = kv;
+  c.head_mask = head_mask;
+  c.a_out = a_out;
+  c.l_out = l_out;
+  c.ws = scratch;
+  c.ws_bytes = FB_NOALLOC_SCRATCH_BYTES;
+  c.num_sms = num_sms;
+  return launch_partial(c, stream);
 }
 
 }  // extern "C"

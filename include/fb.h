@@ -110,6 +110,29 @@ int fb_prefix_attn(const void* q, int32_t B, int32_t n_heads_q, float scale, con
                    size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * fb_prefix_attn without a workspace argument, for callers that cannot allocate
+ * device memory on the call path: plugin interfaces that hand the plugin no
+ * scratch pointer, engines that reserve all device memory up front in their
+ * own pool (a stray cudaMalloc would fail or fragment it), and latency-bound
+ * loops where cudaMalloc / cudaFree may synchronise the device. The pages have
+ * no counterpart to this call; it is a deployment convenience.
+ * Same arguments, results and errors as fb_prefix_attn, except:
+ *  - the split-KV scratch lives in one static device array of
+ *    FB_NOALLOC_SCRATCH_BYTES (32 MiB), which every GPU that loads the library
+ *    holds until the process exits; shapes whose split plan needs more return
+ *    FB_ERR_WORKSPACE with the required size in fb_last_error();
+ *  - the array's device address is looked up on the first call made with a
+ *    given device current; make that first call before any stream capture;
+ *  - all calls share the one array, so calls that overlap on the GPU (other
+ *    streams, other host threads) race and must be serialised by the caller;
+ *  - nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ */
+#define FB_NOALLOC_SCRATCH_BYTES (32u << 20)
+int fb_prefix_attn_noalloc(const void* q, int32_t B, int32_t n_heads_q, float scale,
+                           const fb_kv* kv, const uint8_t* head_mask, float* a_out, float* l_out,
+                           cudaStream_t stream);
+
+/*
  * Block-internal partial ([FB] section 2: A_in, L_in over J_in, recomputed
  * every step). Bidirectional: every block row attends all B block tokens.
  *  q [batch, B, n_heads_q, head_dim], k_in / v_in [batch, B, n_heads_kv, head_dim]
