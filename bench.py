@@ -52,8 +52,11 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=3, help="untimed blocks before timing")
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--mode", choices=["all", "reuse", "dense", "losa"], default="all",
+    p.add_argument("--mode", choices=["all", "reuse", "dense", "losa", "prefix"], default="all",
                    help="all: the contract line; one mode: time only that mode (for profiling)")
+    p.add_argument("--workload", choices=["dllm", "tiny", "gqa", "video", "losa"],
+                   default="dllm", help="dllm is the contract workload; the others are for "
+                   "the per-configuration table")
     return p.parse_args()
 
 
@@ -187,7 +190,6 @@ def measured_peak():
 
 
 def run_ours(args, rank, world, local):
-    import numpy as np
     import torch
 
     import block_diffusion_attention_fb_b200 as fb
@@ -196,82 +198,67 @@ def run_ours(args, rank, world, local):
     from workloads.torch_io import prefix_tensors, to_torch
 
     fb.load_library()
-    wl = make_workload("dllm")
+    wl = make_workload(args.workload)
     sp = wl.spec
     S = sp.steps
-    t = prefix_tensors(wl.prefix, sp.dtype)
+    dt = sp.dtype
+    t = prefix_tensors(wl.prefix, dt)
     kv = fb.KV(t["k"], t["v"], seq_len=t["seq_len"], page_table=t["page_table"],
                page_size=t["page_size"], max_seq_len=t["max_seq_len"])
     steps = list(wl.steps())
-    dq = [to_torch(s.q, "bf16") for s in steps]
-    dk = [to_torch(s.k_in, "bf16") for s in steps]
-    dv = [to_torch(s.v_in, "bf16") for s in steps]
-    hq = [to_torch(s.q, "bf16", "cpu", pin=True) for s in steps]
-    hk = [to_torch(s.k_in, "bf16", "cpu", pin=True) for s in steps]
-    hv = [to_torch(s.v_in, "bf16", "cpu", pin=True) for s in steps]
-    ms = [s.m_updated.tolist() for s in steps]
-    B, Hq, d = sp.block, sp.n_heads_q, sp.head_dim
-    A = torch.zeros(1, B, Hq, d, device="cuda")
-    L = torch.zeros(1, B, Hq, device="cuda")
+    dq = [to_torch(x.q, dt) for x in steps]
+    dk = [to_torch(x.k_in, dt) for x in steps]
+    dv = [to_torch(x.v_in, dt) for x in steps]
+    hq = [to_torch(x.q, dt, "cpu", pin=True) for x in steps]
+    hk = [to_torch(x.k_in, dt, "cpu", pin=True) for x in steps]
+    hv = [to_torch(x.v_in, dt, "cpu", pin=True) for x in steps]
+    ms = [x.m_updated.tolist() for x in steps]
+    batch, B, Hq, d = sp.batch, sp.block, sp.n_heads_q, sp.head_dim
+    A = torch.zeros(batch, B, Hq, d, device="cuda")
+    L = torch.zeros(batch, B, Hq, device="cuda")
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
-    reuse = BlockAttention(kv, B, Hq, "threshold", tau=sp.tau)
-    losa = BlockAttention(kv, B, Hq, "losa", n_active=LOSA_ACTIVE, topk_pages=LOSA_TOPK)
-    a_out = torch.zeros(1, B, Hq, d, device="cuda")
-    l_out = torch.zeros(1, B, Hq, device="cuda")
+    if sp.gamma is not None:
+        reuse = BlockAttention(kv, B, Hq, "per_head", gamma=sp.gamma)
+        reuse_desc = f"FlashBlock per-head reuse (gamma={sp.gamma})"
+    else:
+        tau = sp.tau if sp.tau is not None else 4  # the losa spec states no tau
+        reuse = BlockAttention(kv, B, Hq, "threshold", tau=tau)
+        reuse_desc = f"FlashBlock threshold reuse (tau={tau})"
+    n_act = sp.n_active or LOSA_ACTIVE
+    topk = sp.topk_pages or LOSA_TOPK
+    losa = BlockAttention(kv, B, Hq, "losa", n_active=n_act, topk_pages=topk)
+    a_out = torch.zeros(batch, B, Hq, d, device="cuda")
+    l_out = torch.zeros(batch, B, Hq, device="cuda")
     a_in = torch.zeros_like(a_out)
     l_in = torch.zeros_like(l_out)
     ws = torch.empty(fb.fb_workspace_size(kv, B, Hq), dtype=torch.uint8, device="cuda")
-    stream = torch.cuda.current_stream()
 
     def ev():
         return torch.cuda.Event(enable_timing=True)
 
-    def timed_blocks(n_blocks, one_step, timed, extra=None):
-        """Runs n_blocks blocks of S denoise steps; returns device ms of the steps."""
-        pairs, extra_pairs = [], []
-        for blk_i in range(n_blocks):
-            for s in range(S):
-                flush.zero_()
-                e0, e1 = ev(), ev()
-                if timed:
-                    e0.record(stream)
-                x = one_step(s, extra_pairs if timed else None)
-                if timed:
-                    e1.record(stream)
-                    pairs.append((e0, e1))
-        torch.cuda.synchronize()
-        total = sum(a.elapsed_time(b) for a, b in pairs)
-        ext = [a.elapsed_time(b) for a, b in extra_pairs]
-        return total, ext
-
-    def reuse_step(s, _):
+    def reuse_step(s):
         if s == 0:
             reuse.reset()
         reuse.step(dq[s], dk[s], dv[s], A, L, m_updated=ms[s])
-        return reuse.recomputed
 
-    def dense_step(s, extra):
-        if extra is not None:
-            p0, p1 = ev(), ev()
-            p0.record(stream)
+    def prefix_call(s):
         fb.fb_prefix_attn(dq[s], kv, a_out, l_out, ws)
-        if extra is not None:
-            p1.record(stream)
-            extra.append((p0, p1))
+
+    def dense_rest(s):
         fb.fb_block_attn(dq[s], dk[s], dv[s], a_in, l_in)
         fb.fb_merge(a_out, l_out, a_in, l_in, A, L)
 
-    def losa_step(s, _):
+    def losa_step(s):
         if s == 0:
             losa.reset()
         losa.step(dq[s], dk[s], dv[s], A, L)
 
-    hA = torch.empty(1, B, Hq, d, dtype=torch.float32).pin_memory()
-    hL = torch.empty(1, B, Hq, dtype=torch.float32).pin_memory()
+    hA = torch.empty(batch, B, Hq, d, dtype=torch.float32).pin_memory()
+    hL = torch.empty(batch, B, Hq, dtype=torch.float32).pin_memory()
     qd, kd, vd = torch.empty_like(dq[0]), torch.empty_like(dk[0]), torch.empty_like(dv[0])
 
-    def e2e_step(s, _):
+    def e2e_step(s):
         if s == 0:
             reuse.reset()
         qd.copy_(hq[s], non_blocking=True)
@@ -282,35 +269,99 @@ def run_ours(args, rank, world, local):
         hL.copy_(L, non_blocking=True)
 
     K, W = args.steps, args.warmup
-    if args.mode != "all":
-        fn = {"reuse": reuse_step, "dense": dense_step, "losa": losa_step}[args.mode]
-        timed_blocks(W, fn, False)
-        barrier(world)
-        t_mode, _ = timed_blocks(K, fn, True)
-        barrier(world)
+    if args.mode == "prefix":  # only the dense prefix call, eager (for profilers)
+        for _ in range(W + K):
+            for s in range(S):
+                flush.zero_()
+                prefix_call(s)
+        torch.cuda.synchronize()
         fb.fb_device_status()
         if rank == 0:
-            print(json.dumps({"mode": args.mode, "us_per_step": t_mode * 1000 / (K * S)}))
+            print(json.dumps({"mode": "prefix", "calls": (W + K) * S}))
         return
+    # warm-up of every path (eager, untimed): also sets kernel attributes
+    for _ in range(max(1, W)):
+        for s in range(S):
+            reuse_step(s)
+            prefix_call(s)
+            dense_rest(s)
+            losa_step(s)
+            e2e_step(s)
+    torch.cuda.synchronize()
+
+    # one CUDA graph per denoise step: the host decisions (tau, LoSA step
+    # index) are taken at capture, as a sampler picks a pre-captured variant
+    def capture(fn):
+        graphs = []
+        for s in range(S):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn(s)
+            graphs.append(g)
+        return graphs
+
+    n0 = fb.fb_kernel_launches()
+    g_reuse = capture(reuse_step)
+    launches_per_block = fb.fb_kernel_launches() - n0
+    g_prefix = capture(prefix_call)
+    g_rest = capture(dense_rest)
+    g_losa = capture(losa_step)
+    rec = sum(1 for s in range(S) if s == 0 or (sp.gamma is None and ms[s][0] >= reuse.policy.tau))
+
+    def timed(graph_lists, n_blocks, timed_flag=True):
+        """Replays n_blocks blocks; returns device ms of each graph list's steps."""
+        pairs = [[] for _ in graph_lists]
+        stream = torch.cuda.current_stream()
+        for _ in range(n_blocks):
+            for s in range(S):
+                flush.zero_()
+                for gi, gl in enumerate(graph_lists):
+                    e0, e1 = ev(), ev()
+                    e0.record(stream)
+                    gl[s].replay()
+                    e1.record(stream)
+                    pairs[gi].append((e0, e1))
+        torch.cuda.synchronize()
+        return [sum(a.elapsed_time(b) for a, b in p) for p in pairs], pairs
+
+    def eager(fn, n_blocks):
+        pairs = []
+        stream = torch.cuda.current_stream()
+        for _ in range(n_blocks):
+            for s in range(S):
+                flush.zero_()
+                e0, e1 = ev(), ev()
+                e0.record(stream)
+                fn(s)
+                e1.record(stream)
+                pairs.append((e0, e1))
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in pairs)
+
+    for gl in (g_reuse, g_losa):
+        timed([gl], 1)
+    timed([g_prefix, g_rest], 1)
+    if args.mode != "all":
+        lists = {"reuse": [g_reuse], "dense": [g_prefix, g_rest], "losa": [g_losa]}[args.mode]
+        barrier(world)
+        tot, _ = timed(lists, K)
+        barrier(world)
+        if rank == 0:
+            print(json.dumps({"mode": args.mode, "us_per_step": sum(tot) * 1000 / (K * S)}))
+        return
+
     clocks = ClockSampler(local)
-    # warm-up of every path (untimed)
-    for fn in (reuse_step, dense_step, losa_step, e2e_step):
-        timed_blocks(W, fn, False)
     barrier(world)
     clocks.start()
     barrier(world)
-    n0 = fb.fb_kernel_launches()
-    t_reuse, _ = timed_blocks(K, reuse_step, True)
-    launches = fb.fb_kernel_launches() - n0
+    (t_reuse,), _ = timed([g_reuse], K)
     barrier(world)
-    rec = 0
-    for s in range(S):  # recompute decisions of one block (identical every block)
-        rec += int(s == 0 or ms[s][0] >= sp.tau)
-    t_dense, prefix_ms = timed_blocks(K, dense_step, True)
+    (t_prefix, t_rest), pairs = timed([g_prefix, g_rest], K)
+    t_dense = t_prefix + t_rest
     barrier(world)
-    t_losa, _ = timed_blocks(K, losa_step, True)
+    (t_losa,), _ = timed([g_losa], K)
     barrier(world)
-    t_e2e, _ = timed_blocks(K, e2e_step, True)
+    t_e2e = eager(e2e_step, K)
     barrier(world)
     clk = clocks.stop()
     fb.fb_device_status()
@@ -323,13 +374,14 @@ def run_ours(args, rank, world, local):
     us = lambda ms_total: ms_total * 1000.0 / n_steps_all  # noqa: E731
 
     # roofline of the dominant kernel call: the dense prefix partial
-    kv_bytes = 2 * int(wl.prefix.seq_len.sum()) * sp.n_heads_kv * d * 2
-    io_bytes = B * Hq * d * 2 + B * Hq * (d + 1) * 4
+    kv_bytes = 2 * int(wl.prefix.seq_len.sum()) * sp.n_heads_kv * d * (2 if dt == "bf16" else 4)
+    io_bytes = batch * B * Hq * d * (2 if dt == "bf16" else 4) + batch * B * Hq * (d + 1) * 4
     alg_bytes = kv_bytes + io_bytes
-    prefix_avg_ms = statistics.mean(prefix_ms)
+    flops = 4.0 * int(wl.prefix.seq_len.sum()) * B * Hq * d
+    prefix_avg_ms = t_prefix / (K * S)
     achieved = alg_bytes / (prefix_avg_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peak()
-    traffic = profiled_traffic()
+    traffic = profiled_traffic() if args.workload == "dllm" else None
     if rank != 0:
         return
     line = {
@@ -343,31 +395,32 @@ def run_ours(args, rank, world, local):
         "higher_is_better": False,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": dt,
         "data": "synthetic (seeded generator; no model weights or datasets)",
         "config": {
-            "workload": WORKLOAD,
-            "global_batch": world,
+            "workload": WORKLOAD if args.workload == "dllm" else args.workload,
+            "global_batch": world * batch,
             "seq_len": int(wl.prefix.max_seq_len),
             "block": B,
             "denoise_steps_per_bench_step": S,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": "flushed between denoise steps (256 MiB write, outside the timed events)",
-            "value_mode": "reuse (FlashBlock threshold, tau=4) through fb_step",
+            "value_mode": f"reuse: {reuse_desc} through fb_step, one CUDA graph per denoise step",
         },
         "modes": {
             "reuse": {"us_per_step": round(us(t_reuse_max), 3),
-                      "prefix_recomputes_per_block": rec},
+                      "prefix_recomputes_per_block": rec if sp.gamma is None else None},
             "dense": {"us_per_step": round(us(t_dense_max), 3),
                       "prefix_call_us": round(prefix_avg_ms * 1000, 3),
-                      "prefix_gbs": round(achieved, 1)},
-            "losa": {"us_per_step": round(us(t_losa_max), 3), "n_active": LOSA_ACTIVE,
-                     "topk_pages": LOSA_TOPK},
+                      "prefix_gbs": round(achieved, 1),
+                      "prefix_tflops": round(flops / (prefix_avg_ms * 1e-3) / 1e12, 1)},
+            "losa": {"us_per_step": round(us(t_losa_max), 3), "n_active": n_act,
+                     "topk_pages": topk},
         },
-        "tokens_per_s": round(world * K * B / (t_reuse_max * 1e-3), 1),
+        "tokens_per_s": round(world * K * batch * B / (t_reuse_max * 1e-3), 1),
         "roofline": {
             "bound": "hbm",
-            "kernel": "fb_prefix_attn (split-KV attention + combine), dense dllm prefix",
+            "kernel": "fb_prefix_attn (split-KV attention + combine), dense prefix",
             "achieved": round(achieved, 1),
             "peak": peak,
             "peak_kind": f"{peak_kind} (copy bandwidth, burst)",
@@ -379,15 +432,15 @@ def run_ours(args, rank, world, local):
         "e2e": {
             "value": round(us(t_e2e_max), 3),
             "unit": UNIT,
-            "h2d_bytes_per_step": 3 * B * Hq * d * 2 * S,
-            "d2h_bytes_per_step": (B * Hq * d * 4 + B * Hq * 4) * S,
-            "api": "fb_step (reuse) with q/k/v copied from pinned host memory and A_full/L_full "
-                   "copied back every denoise step",
+            "h2d_bytes_per_step": 3 * batch * B * Hq * d * (2 if dt == "bf16" else 4) * S,
+            "d2h_bytes_per_step": (batch * B * Hq * d * 4 + batch * B * Hq * 4) * S,
+            "api": "fb_step (reuse), eager, with q/k/v copied from pinned host memory and "
+                   "A_full/L_full copied back every denoise step",
         },
-        "gpu_launches": int(launches),
+        "gpu_launches": int(launches_per_block * K),
         "clocks": clk,
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and args.workload == "dllm":
         line["cpu_baseline"] = oracle_baseline(wl)
     print(json.dumps(line), flush=True)
 

@@ -61,6 +61,8 @@ struct AttnArgs {
   float* a_out;     // [batch, B, Hq, D]
   float* l_out;     // [batch, B, Hq] natural log
   float* a_prev;    // optional: old a_out rows are copied here before overwrite
+  const float* mrg_a;  // optional second partial merged into every final row (FlashBlock merge)
+  const float* mrg_l;
 };
 
 __device__ __forceinline__ int seq_tokens(const AttnArgs& a, int b) {
@@ -132,13 +134,58 @@ __device__ __forceinline__ void row_of(const AttnArgs& a, int b, int hk, int r, 
   i = a.row_list ? a.row_list[b * a.n_list + i_idx] : i_idx;
 }
 
-// Writes one finished row (acc already normalised, lse2 in log2 units).
+// Writes one final row: vals (normalised, NV per lane at col0 + j*col_stride)
+// and lse2 (log2 units). With mrg_a set the row is first merged with the
+// second partial by the FlashBlock rule: m = max(L1, L2), w_x = e^{L_x - m},
+// A = (w1 A1 + w2 A2) / (w1 + w2), L = m + log(w1 + w2); a side with L = -inf
+// is not read.
+template <int NV>
+__device__ __forceinline__ void write_final(const AttnArgs& a, int b, int hk, int r,
+                                            const float (&val)[NV], int col0, int col_stride,
+                                            float lse2, bool lane0) {
+  int i, h;
+  row_of(a, b, hk, r, i, h);
+  if (!row_selected(a, b, h)) return;
+  const long long row = ((long long)b * a.B + i) * a.Hq + h;
+  constexpr int D = NV * 32;
+  float* dst = a.a_out + row * D;
+  const float Ln = lse2 * kLn2;
+  float wn = 1.f, wo = 0.f, L = Ln;
+  if (a.mrg_a) {
+    const float Lo = a.mrg_l[row];
+    const float m = fmaxf(Lo, Ln);
+    if (m == -INFINITY) {
+      wn = 0.f;
+      L = -INFINITY;
+    } else {
+      const float eo = expf(Lo - m), en = expf(Ln - m);
+      const float inv = 1.f / (eo + en);
+      wn = en * inv;
+      wo = eo * inv;
+      L = m + logf(eo + en);
+    }
+  }
+  if (a.a_prev) {
+    float* prv = a.a_prev + row * D;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) prv[col0 + j * col_stride] = dst[col0 + j * col_stride];
+  }
+  const float* old = a.mrg_a ? a.mrg_a + row * D : nullptr;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int col = col0 + j * col_stride;
+    float v = wn > 0.f ? wn * val[j] : 0.f;
+    if (old && wo > 0.f) v += wo * old[col];
+    dst[col] = v;
+  }
+  if (lane0) a.l_out[row] = L;
+}
+
+// Writes one finished row: a split partial (n_splits > 1) or the final row.
 template <int NV>
 __device__ __forceinline__ void store_row(const AttnArgs& a, int b, int hk, int split, int r,
                                           const float (&val)[NV], int col0, int col_stride,
                                           float lse2, bool lane0) {
-  constexpr int D = NV * 32;  // NV values per lane, 32 lanes
-  (void)D;
   if (a.n_splits > 1) {
     const long long pidx = (((long long)split * a.batch + b) * a.Hkv + hk) * a.R + r;
     float* dst = a.o_part + pidx * (NV * 32);
@@ -147,19 +194,126 @@ __device__ __forceinline__ void store_row(const AttnArgs& a, int b, int hk, int 
     if (lane0) a.lse_part[pidx] = lse2;
     return;
   }
-  int i, h;
-  row_of(a, b, hk, r, i, h);
-  if (!row_selected(a, b, h)) return;
-  const long long row = ((long long)b * a.B + i) * a.Hq + h;
-  float* dst = a.a_out + row * (NV * 32);
-  if (a.a_prev) {
-    float* prv = a.a_prev + row * (NV * 32);
+  write_final<NV>(a, b, hk, r, val, col0, col_stride, lse2, lane0);
+}
+
+// write_final for RB rows of one warp at once: every global read the rows need
+// (merge partner, old rows) is issued before any arithmetic or store, so the
+// rows' memory latencies overlap instead of adding up.
+template <int NV, int RB>
+__device__ __forceinline__ void write_final_rows(const AttnArgs& a, int b, int hk,
+                                                 const int (&r)[RB], const float (&val)[RB][NV],
+                                                 const float (&lse2)[RB], int lane) {
+  constexpr int D = NV * 32;
+  long long row[RB];
+  bool ok[RB];
+  float Lo[RB], old[RB][NV], prv[RB][NV];
 #pragma unroll
-    for (int j = 0; j < NV; ++j) prv[col0 + j * col_stride] = dst[col0 + j * col_stride];
+  for (int k = 0; k < RB; ++k) {
+    ok[k] = r[k] >= 0;
+    row[k] = 0;
+    if (ok[k]) {
+      int i, h;
+      row_of(a, b, hk, r[k], i, h);
+      ok[k] = row_selected(a, b, h);
+      row[k] = ((long long)b * a.B + i) * a.Hq + h;
+    }
   }
 #pragma unroll
-  for (int j = 0; j < NV; ++j) dst[col0 + j * col_stride] = val[j];
-  if (lane0) a.l_out[row] = lse2 * kLn2;
+  for (int k = 0; k < RB; ++k) {
+    Lo[k] = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) old[k][j] = prv[k][j] = 0.f;
+    if (!ok[k]) continue;
+    if (a.mrg_a) {
+      Lo[k] = a.mrg_l[row[k]];
+#pragma unroll
+      for (int j = 0; j < NV; ++j) old[k][j] = a.mrg_a[row[k] * D + lane * NV + j];
+    }
+    if (a.a_prev) {
+#pragma unroll
+      for (int j = 0; j < NV; ++j) prv[k][j] = a.a_out[row[k] * D + lane * NV + j];
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < RB; ++k) {
+    if (!ok[k]) continue;
+    const float Ln = lse2[k] * kLn2;
+    float wn = 1.f, wo = 0.f, L = Ln;
+    if (a.mrg_a) {
+      const float m = fmaxf(Lo[k], Ln);
+      if (m == -INFINITY) {
+        wn = 0.f;
+        L = -INFINITY;
+      } else {
+        const float eo = expf(Lo[k] - m), en = expf(Ln - m);
+        const float inv = 1.f / (eo + en);
+        wn = en * inv;
+        wo = eo * inv;
+        L = m + logf(eo + en);
+      }
+    }
+    if (a.a_prev) {
+#pragma unroll
+      for (int j = 0; j < NV; ++j) a.a_prev[row[k] * D + lane * NV + j] = prv[k][j];
+    }
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      float v = wn > 0.f ? wn * val[k][j] : 0.f;
+      if (wo > 0.f) v += wo * old[k][j];
+      a.a_out[row[k] * D + lane * NV + j] = v;
+    }
+    if (lane == 0) a.l_out[row[k]] = L;
+  }
+}
+
+// Merges the n_splits partials of row r of (b, hk) (log-space rule) and writes
+// the final row. One warp, NV contiguous columns per lane. The normalisers of
+// 32 splits are read at once (one per lane) and their weights broadcast by
+// shuffle, so the partial loads of a chunk are independent of each other.
+// Empty splits (lse = -inf) have weight 0 and all-zero partials.
+template <int NV>
+__device__ __forceinline__ void combine_row(const AttnArgs& a, int b, int hk, int r, int lane) {
+  constexpr int D = NV * 32;
+  const long long stride = (long long)a.batch * a.Hkv * a.R;  // between splits
+  const long long p0 = ((long long)b * a.Hkv + hk) * a.R + r;
+  float M = -INFINITY;
+  for (int s = lane; s < a.n_splits; s += 32) M = fmaxf(M, __ldcg(a.lse_part + p0 + s * stride));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float bse = (M == -INFINITY) ? 0.f : M;
+  float acc[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) acc[j] = 0.f;
+  float wsum = 0.f;
+  for (int s0 = 0; s0 < a.n_splits; s0 += 32) {
+    const int s = s0 + lane;
+    const float l = s < a.n_splits ? __ldcg(a.lse_part + p0 + s * stride) : -INFINITY;
+    const float wl = l == -INFINITY ? 0.f : fast_exp2(l - bse);
+    const int n = min(32, a.n_splits - s0);
+#pragma unroll 8
+    for (int j = 0; j < n; ++j) {
+      // empty splits carry weight 0 and zero partials, so every load is issued
+      const float w = __shfl_sync(0xffffffffu, wl, j);
+      wsum += w;
+      const float* src = a.o_part + (p0 + (long long)(s0 + j) * stride) * D + lane * NV;
+      if constexpr (NV == 4) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
+        acc[0] += w * v.x;
+        acc[1] += w * v.y;
+        acc[2] += w * v.z;
+        acc[3] += w * v.w;
+      } else {
+#pragma unroll
+        for (int jj = 0; jj < NV; ++jj) acc[jj] += w * __ldcg(src + jj);
+      }
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) acc[j] *= inv;
+  const float lse2 = wsum > 0.f ? bse + log2f(wsum) : -INFINITY;
+  write_final<NV>(a, b, hk, r, acc, lane * NV, 1, lse2, lane == 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -449,32 +603,44 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   }
   named_bar_sync(1, kNWC * 32);
   constexpr int NV = D / 32;
-  for (int rl = warp; rl < RG * 16; rl += kNWC) {
-    const int r = rt * a.row_tile + rl;
-    if (r >= a.R) break;
-    const int rgi = rl >> 4, rr = rl & 15;
-    float M = -INFINITY;
+  constexpr int RB = (RG * 16) / kNWC < 4 ? (RG * 16) / kNWC : 4;  // rows per batch of a warp
+  for (int rl0 = warp; rl0 < RG * 16; rl0 += kNWC * RB) {
+    int rr_[RB];
+    float val[RB][NV], lse2[RB];
 #pragma unroll
-    for (int k = 0; k < KS; ++k) M = fmaxf(M, redM[(rgi + k * RG) * 16 + rr]);
-    const float bse = (M == -INFINITY) ? 0.f : M;
-    float lsum = 0.f;
-    float acc[NV];
+    for (int k = 0; k < RB; ++k) {
+      const int rl = rl0 + k * kNWC;
+      const int r = rt * a.row_tile + rl;
+      rr_[k] = (rl < RG * 16 && r < a.R) ? r : -1;
+      const int rgi = (rl >> 4) < RG ? (rl >> 4) : RG - 1, rr = rl & 15;
+      float M = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < NV; ++j) acc[j] = 0.f;
+      for (int kk = 0; kk < KS; ++kk) M = fmaxf(M, redM[(rgi + kk * RG) * 16 + rr]);
+      const float bse = (M == -INFINITY) ? 0.f : M;
+      float lsum = 0.f;
 #pragma unroll
-    for (int k = 0; k < KS; ++k) {
-      const int wi = rgi + k * RG;
-      const float w = fast_exp2(redM[wi * 16 + rr] - bse);
-      lsum += w * redL[wi * 16 + rr];
-      const float* src = &redO[(wi * 16 + rr) * S::kRedStride + lane * NV];
+      for (int j = 0; j < NV; ++j) val[k][j] = 0.f;
 #pragma unroll
-      for (int j = 0; j < NV; ++j) acc[j] += w * src[j];
+      for (int kk = 0; kk < KS; ++kk) {
+        const int wi = rgi + kk * RG;
+        const float w = fast_exp2(redM[wi * 16 + rr] - bse);
+        lsum += w * redL[wi * 16 + rr];
+        const float* src = &redO[(wi * 16 + rr) * S::kRedStride + lane * NV];
+#pragma unroll
+        for (int j = 0; j < NV; ++j) val[k][j] += w * src[j];
+      }
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+#pragma unroll
+      for (int j = 0; j < NV; ++j) val[k][j] *= inv;
+      lse2[k] = lsum > 0.f ? bse + log2f(lsum) : -INFINITY;
     }
-    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    if (a.n_splits > 1) {
 #pragma unroll
-    for (int j = 0; j < NV; ++j) acc[j] *= inv;
-    const float lse2 = lsum > 0.f ? bse + log2f(lsum) : -INFINITY;
-    store_row<NV>(a, b, hk, split, r, acc, lane * NV, 1, lse2, lane == 0);
+      for (int k = 0; k < RB; ++k)
+        if (rr_[k] >= 0) store_row<NV>(a, b, hk, split, rr_[k], val[k], lane * NV, 1, lse2[k], lane == 0);
+    } else {
+      write_final_rows<NV, RB>(a, b, hk, rr_, val, lse2, lane);
+    }
   }
 }
 
@@ -616,37 +782,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ At
   int i, h;
   row_of(a, b, hk, r, i, h);
   if (!row_selected(a, b, h)) return;
-  float M = -INFINITY;
-  for (int s = 0; s < a.n_splits; ++s) {
-    const long long pidx = (((long long)s * a.batch + b) * a.Hkv + hk) * a.R + r;
-    M = fmaxf(M, a.lse_part[pidx]);
-  }
-  const float bse = (M == -INFINITY) ? 0.f : M;
-  float acc[NV];
-#pragma unroll
-  for (int j = 0; j < NV; ++j) acc[j] = 0.f;
-  float wsum = 0.f;
-  for (int s = 0; s < a.n_splits; ++s) {
-    const long long pidx = (((long long)s * a.batch + b) * a.Hkv + hk) * a.R + r;
-    const float l = a.lse_part[pidx];
-    if (l == -INFINITY) continue;
-    const float w = fast_exp2(l - bse);
-    wsum += w;
-    const float* src = a.o_part + pidx * D + lane * NV;
-#pragma unroll
-    for (int j = 0; j < NV; ++j) acc[j] += w * src[j];
-  }
-  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  const long long row = ((long long)b * a.B + i) * a.Hq + h;
-  float* dst = a.a_out + row * D + lane * NV;
-  if (a.a_prev) {
-    float* prv = a.a_prev + row * D + lane * NV;
-#pragma unroll
-    for (int j = 0; j < NV; ++j) prv[j] = dst[j];
-  }
-#pragma unroll
-  for (int j = 0; j < NV; ++j) dst[j] = acc[j] * inv;
-  if (lane == 0) a.l_out[row] = wsum > 0.f ? (bse + log2f(wsum)) * kLn2 : -INFINITY;
+  combine_row<NV>(a, b, hk, r, lane);
 }
 
 // ---------------------------------------------------------------------------

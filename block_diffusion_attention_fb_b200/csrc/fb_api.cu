@@ -14,6 +14,7 @@
 
 #include "../../include/fb.h"
 #include "attn.cuh"
+#include "attn_tc.cuh"
 #include "cosine.cuh"
 #include "losa.cuh"
 
@@ -58,9 +59,12 @@ int next_pow2(int x) {
 }
 
 int sm_count() {
+  static int cached[256] = {};
   int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return 0;
+  if (cached[dev]) return cached[dev];
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  cached[dev] = n;
   return n;
 }
 
@@ -76,18 +80,29 @@ struct Plan {
   int tiles_per_split, n_splits;
 };
 
-Plan make_plan(fb_dtype dt, int batch, int Hkv, int R, int max_tiles, int num_sms) {
+// The tcgen05 kernel (attn_tc.cuh) is not launched: it passes the short-key-range
+// parity cases but stalls on long key ranges (hundreds of tiles per CTA) and
+// stays disabled until that is understood. bf16 runs on the mma.sync kernel,
+// fp32 on the CUDA-core kernel.
+bool use_tc(fb_dtype dt, int D) { return false && dt == FB_BF16 && D == 128; }
+
+Plan make_plan(fb_dtype dt, int batch, int Hkv, int R, int max_tiles, int num_sms, int D = 128) {
   Plan p{};
+  int ctas_per_sm = 2;
   if (dt == FB_F32) {
     p.row_tile = kF32Rows;
     p.rg = 1;
+  } else if (use_tc(dt, D)) {
+    p.row_tile = kTcRows;
+    p.rg = 0;
+    ctas_per_sm = 1;
   } else {
     p.rg = R <= 16 ? 1 : (R <= 32 ? 2 : 4);
     p.row_tile = 16 * p.rg;
   }
   p.n_row_tiles = ceil_div(R, p.row_tile);
   const long long units = (long long)batch * Hkv * p.n_row_tiles;
-  const long long target = (long long)(num_sms > 0 ? num_sms : 148) * 2 * 4;
+  const long long target = (long long)(num_sms > 0 ? num_sms : 148) * ctas_per_sm * 4;
   max_tiles = max_tiles < 1 ? 1 : max_tiles;
   long long splits = (target + units - 1) / units;
   if (splits < 1) splits = 1;
@@ -97,6 +112,7 @@ Plan make_plan(fb_dtype dt, int batch, int Hkv, int R, int max_tiles, int num_sm
   return p;
 }
 
+// Split partials [splits, batch, Hkv, R, D] + their log2 normalisers.
 size_t partial_bytes(const Plan& p, int batch, int Hkv, int R, int D) {
   if (p.n_splits <= 1) return 0;
   const size_t rows = (size_t)p.n_splits * batch * Hkv * R;
@@ -123,7 +139,7 @@ WsLayout ws_layout(const fb_kv* kv, int B, int Hq, int n_active, int topk, int n
   const int G = Hq / kv->n_heads_kv, D = kv->head_dim;
   const int R = B * G;
   const Plan pd = make_plan(kv->dtype, kv->batch, kv->n_heads_kv, R, ceil_div(kv->max_seq_len, kTK),
-                            num_sms);
+                            num_sms, D);
   size_t part = partial_bytes(pd, kv->batch, kv->n_heads_kv, R, D);
   size_t scores = 0;
   if (n_active > 0 && topk > 0) {
@@ -131,7 +147,7 @@ WsLayout ws_layout(const fb_kv* kv, int B, int Hq, int n_active, int topk, int n
     const int per_tile = kTK / (kv->page_size < kTK ? kv->page_size : kTK);
     const int ent = max_union_entries(kv, G, na, topk);
     const Plan pg = make_plan(kv->dtype, kv->batch, kv->n_heads_kv, na * G, ceil_div(ent, per_tile),
-                              num_sms);
+                              num_sms, D);
     const size_t pgb = partial_bytes(pg, kv->batch, kv->n_heads_kv, na * G, D);
     part = part > pgb ? part : pgb;
     scores = round_up((size_t)kv->batch * na * Hq * logical_pages(kv) * 4, 256) +
@@ -221,6 +237,8 @@ struct PartialCall {
   size_t ws_offset;
   int num_sms;
   bool single_split;  // one CTA streams the whole key set (no workspace)
+  const float* mrg_a;  // optional: merge every final row with this partial (FlashBlock merge)
+  const float* mrg_l;
 };
 
 int launch_partial(const PartialCall& c, cudaStream_t stream) {
@@ -253,6 +271,8 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
     for (int i = 0; i < 4; ++i) a.seq_bits[i] = c.seq_bits[i];
   }
   a.scale_log2 = c.scale * kLog2e;
+  a.mrg_a = c.mrg_a;
+  a.mrg_l = c.mrg_l;
   a.a_out = c.a_out;
   a.l_out = c.l_out;
   a.a_prev = c.a_prev;
@@ -266,7 +286,7 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
     a.chunk = kv->page_table ? (kv->page_size < kTK ? kv->page_size : kTK) : kTK;
     max_tiles = ceil_div(kv->max_seq_len, kTK);
   }
-  Plan p = make_plan(kv->dtype, kv->batch, Hkv, a.R, max_tiles, c.num_sms);
+  Plan p = make_plan(kv->dtype, kv->batch, Hkv, a.R, max_tiles, c.num_sms, D);
   if (c.single_split) {
     p.tiles_per_split = max_tiles < 1 ? 1 : max_tiles;
     p.n_splits = 1;
@@ -282,9 +302,9 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
                   need, c.ws_offset, c.ws_bytes);
     if (!aligned16(c.ws)) return fail(FB_ERR_ALIGN, "workspace not 16-byte aligned");
     const size_t rows = (size_t)p.n_splits * kv->batch * Hkv * a.R;
-    a.o_part = reinterpret_cast<float*>(static_cast<char*>(c.ws) + c.ws_offset);
-    a.lse_part = reinterpret_cast<float*>(static_cast<char*>(c.ws) + c.ws_offset +
-                                          round_up(rows * D * 4, 256));
+    char* w = static_cast<char*>(c.ws) + c.ws_offset;
+    a.o_part = reinterpret_cast<float*>(w);
+    a.lse_part = reinterpret_cast<float*>(w + round_up(rows * D * 4, 256));
   }
   const dim3 grid(p.n_row_tiles * p.n_splits, Hkv, kv->batch);
   if (kv->dtype == FB_F32) {
@@ -309,7 +329,15 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
     }                                                                                        \
     kfn<<<grid, kAttnThreads, smem, stream>>>(a, tk, tv);                                    \
   } while (0)
-    if (D == 128) {
+    if (use_tc(kv->dtype, D)) {
+      static bool tc_attr = false;
+      if (!tc_attr) {
+        cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             TcSmem::kBytes);
+        tc_attr = true;
+      }
+      attn_tc_kernel<<<grid, kTcThreads, TcSmem::kBytes, stream>>>(a, tk, tv);
+    } else if (D == 128) {
       if (p.rg == 1)
         FB_LAUNCH_BF16(128, 1);
       else if (p.rg == 2)
@@ -375,7 +403,8 @@ KvView kv_view(const fb_kv* kv) {
 
 int block_attn_impl(const void* q, const void* k_in, const void* v_in, int batch, int B, int Hq,
                     int Hkv, int D, float scale, fb_dtype dt, float* a_in, float* l_in,
-                    cudaStream_t stream) {
+                    cudaStream_t stream, const float* mrg_a = nullptr,
+                    const float* mrg_l = nullptr) {
   fb_kv kv{};
   kv.k = k_in;
   kv.v = v_in;
@@ -401,6 +430,9 @@ int block_attn_impl(const void* q, const void* k_in, const void* v_in, int batch
   c.l_out = l_in;
   // the block is short: one split per (b, hk, row tile), no workspace needed
   c.single_split = true;
+  c.num_sms = sm_count();
+  c.mrg_a = mrg_a;
+  c.mrg_l = mrg_l;
   return launch_partial(c, stream);
 }
 
@@ -554,7 +586,10 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
   active_rows_kernel<<<kv->batch, 256, B * 4, stream>>>(rs, B, na, active_rows);
   rc = check_launch("active rows kernel");
   if (rc) return rc;
-  const dim3 g2(ceil_div(v.max_pages, 8), v.Hkv, kv->batch);
+  // about four blocks of 8 page-warps per SM over all (b, hk)
+  const int px = max(1, min(ceil_div(v.max_pages, 16),
+                            ceil_div((long long)num_sms * 4, (long long)v.Hkv * kv->batch)));
+  const dim3 g2(px, v.Hkv, kv->batch);
   const int qsm = na * G * D * 4;
   if (kv->dtype == FB_BF16) {
     auto kfn = D == 128 ? page_score_kernel<__nv_bfloat16, 128> : page_score_kernel<__nv_bfloat16, 64>;
@@ -721,13 +756,11 @@ int fb_step(const fb_policy* policy, fb_cache* cache, const void* q, const void*
   } else {
     return fail(FB_ERR_ARG, "unknown mode");
   }
-  float* a_in = reinterpret_cast<float*>(ws + w.a_in);
-  float* l_in = reinterpret_cast<float*>(ws + w.l_in);
-  rc = block_attn_impl(q, k_in, v_in, batch, B, Hq, Hkv, D, policy->scale, prefix->dtype, a_in,
-                       l_in, stream);
-  if (rc) return rc;
-  rc = merge_launch(cache->a_out, cache->l_out, a_in, l_in, (long long)batch * B * Hq, D, a_full,
-                    l_full, stream);
+  // block-internal partial and the FlashBlock merge with the cached
+  // block-external partial in one kernel: A_full directly
+  float* lf = l_full ? l_full : reinterpret_cast<float*>(ws + w.l_in);
+  rc = block_attn_impl(q, k_in, v_in, batch, B, Hq, Hkv, D, policy->scale, prefix->dtype, a_full,
+                       lf, stream, cache->a_out, cache->l_out);
   if (rc) return rc;
   cache->step = s + 1;
   return FB_OK;
@@ -765,7 +798,7 @@ int fb_prefix_attn_noalloc(const void* q, int32_t B, int32_t n_heads_q, float sc
   const int num_sms = sm_count();
   const int R = B * (n_heads_q / kv->n_heads_kv);
   const Plan p = make_plan(kv->dtype, kv->batch, kv->n_heads_kv, R, ceil_div(kv->max_seq_len, kTK),
-                           num_sms);
+                           num_sms, kv->head_dim);
   const size_t need = partial_bytes(p, kv->batch, kv->n_heads_kv, R, kv->head_dim);
   if (need > (size_t)FB_NOALLOC_SCRATCH_BYTES)
     return fail(FB_ERR_WORKSPACE,

@@ -174,33 +174,45 @@ __global__ void __launch_bounds__(256)
   }
   __syncthreads();
   const int n_pages = (kv_tokens(kv, b) + kv.page_size - 1) / kv.page_size;
-  const int p = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (p >= n_pages) return;
-  const long long so = (((long long)b * kv.max_pages + p) * kv.Hkv + hk) * D;
-  float lo[NV], hi[NV];
+  const int stride = gridDim.x * (blockDim.x >> 5);
+  // two pages per warp per iteration: their loads are issued before any math
+  for (int p0 = blockIdx.x * (blockDim.x >> 5) + warp; p0 < n_pages; p0 += 2 * stride) {
+    float lo[2][NV], hi[2][NV];
 #pragma unroll
-  for (int j = 0; j < NV; ++j) {
-    lo[j] = ld_f32<T>(pmin + so + lane + 32 * j);
-    hi[j] = ld_f32<T>(pmax + so + lane + 32 * j);
-  }
-  for (int rq = 0; rq < RQ; ++rq) {
-    float x[NV];
+    for (int u = 0; u < 2; ++u) {
+      const int p = p0 + u * stride;
+      const long long so = (((long long)b * kv.max_pages + (p < n_pages ? p : p0)) * kv.Hkv + hk) * D;
 #pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      const float qv = qs[rq * D + lane + 32 * j];
-      x[j] = fmaxf(__fmul_rn(qv, lo[j]), __fmul_rn(qv, hi[j]));
+      for (int j = 0; j < NV; ++j) {
+        lo[u][j] = ld_f32<T>(pmin + so + lane + 32 * j);
+        hi[u][j] = ld_f32<T>(pmax + so + lane + 32 * j);
+      }
     }
-    // in-lane levels: strides D/2 ... 32 pair j with j + NV/2 ...
 #pragma unroll
-    for (int s = NV / 2; s >= 1; s >>= 1)
+    for (int u = 0; u < 2; ++u) {
+      const int p = p0 + u * stride;
+      if (p >= n_pages) break;
+      for (int rq = 0; rq < RQ; ++rq) {
+        float x[NV];
 #pragma unroll
-      for (int j = 0; j < s; ++j) x[j] = __fadd_rn(x[j], x[j + s]);
-    float v = x[0];
+        for (int j = 0; j < NV; ++j) {
+          const float qv = qs[rq * D + lane + 32 * j];
+          x[j] = fmaxf(__fmul_rn(qv, lo[u][j]), __fmul_rn(qv, hi[u][j]));
+        }
+        // lane l holds channels l + 32 j: tree levels with stride >= 32 pair
+        // j with j + s inside the lane; the last five use xor shuffles
 #pragma unroll
-    for (int s = 16; s >= 1; s >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, s));
-    if (lane == 0) {
-      const int a_i = rq / G, g = rq - (rq / G) * G;
-      scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = v;
+        for (int s = NV / 2; s >= 1; s >>= 1)
+#pragma unroll
+          for (int j = 0; j < s; ++j) x[j] = __fadd_rn(x[j], x[j + s]);
+        float v = x[0];
+#pragma unroll
+        for (int s = 16; s >= 1; s >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, s));
+        if (lane == 0) {
+          const int a_i = rq / G, g = rq - (rq / G) * G;
+          scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = v;
+        }
+      }
     }
   }
 }
@@ -257,18 +269,37 @@ __global__ void __launch_bounds__(kTopkThreads)
       if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
     }
     __syncthreads();
-    if (tid == 0) {
-      int need = s_need, cum = 0, sel = 0;
-      for (int d = 255; d >= 0; --d) {
-        if (cum + hist[d] >= need) {
-          sel = d;
-          need -= cum;
-          break;
-        }
-        cum += hist[d];
+    if (tid < 32) {
+      // buckets in descending order: lane l owns digits 255-8l ... 248-8l
+      int cnt[8], tot = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        cnt[j] = hist[255 - 8 * tid - j];
+        tot += cnt[j];
       }
-      s_prefix = prefix | ((uint32_t)sel << shift);
-      s_need = need;
+      int incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += v;
+      }
+      const int need = s_need;
+      const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
+      const int owner = __ffs(hit) - 1;  // first lane whose running count reaches need
+      if (tid == owner) {
+        int cum = incl - tot, sel = 0, rem = need;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (cum + cnt[j] >= need) {
+            sel = 255 - 8 * tid - j;
+            rem = need - cum;
+            break;
+          }
+          cum += cnt[j];
+        }
+        s_prefix = prefix | ((uint32_t)sel << shift);
+        s_need = rem;
+      }
     }
     mask |= 0xFFu << shift;
     __syncthreads();
@@ -280,18 +311,29 @@ __global__ void __launch_bounds__(kTopkThreads)
   const int p0 = tid * seg, p1 = min(n, p0 + seg);
   int cnt = 0;
   for (int p = p0; p < p1; ++p) cnt += (keys[p] == T);
-  seg_cnt[tid] = cnt;
+  // exclusive scan of the per-thread counts (thread order = index order)
+  const int lane = tid & 31, wid = tid >> 5;
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) seg_cnt[wid] = incl;
   __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int t = 0; t < kTopkThreads; ++t) {
-      const int c = seg_cnt[t];
-      seg_cnt[t] = run;
-      run += c;
+  if (wid == 0) {
+    const int nw = kTopkThreads / 32;
+    int x = lane < nw ? seg_cnt[lane] : 0;
+    int wi = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += v;
     }
+    if (lane < nw) seg_cnt[lane] = wi - x;  // exclusive warp offsets
   }
   __syncthreads();
-  int eq_before = seg_cnt[tid];
+  int eq_before = seg_cnt[wid] + incl - cnt;
   for (int p = p0; p < p1; ++p) {
     const uint32_t key = keys[p];
     bool take = key > T;

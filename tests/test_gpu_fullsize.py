@@ -1,0 +1,188 @@
+"""GPU parity at the full workload sizes (the five configurations), on sampled
+outputs the oracle computes row by row; integer decisions are checked whole.
+
+The sampled rows are fixed by a seed and span the first and last block rows,
+every kv head and, for GQA, every sequence. Steps run through fb_step (or
+fb_prefix_attn for the dense partial), exactly as bench.py calls them.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import block_diffusion_attention_fb_b200 as fb
+import oracle
+from block_diffusion_attention_fb_b200.runtime import BlockAttention
+from oracle import losa as olosa
+from oracle.controllers import head_cosine
+from tests.gpu_util import assert_close_A, assert_close_L, cpu, dev, make_kv, sync
+from workloads import make_workload
+
+pytestmark = pytest.mark.gpu
+
+
+def _samples(sp, n, seed):
+    rng = np.random.default_rng(seed)
+    out = {(0, 0, 0), (sp.batch - 1, sp.block - 1, sp.n_heads_q - 1)}
+    for b in range(sp.batch):
+        out.add((b, int(rng.integers(sp.block)), int(rng.integers(sp.n_heads_q))))
+    while len(out) < n:
+        out.add((int(rng.integers(sp.batch)), int(rng.integers(sp.block)),
+                 int(rng.integers(sp.n_heads_q))))
+    return sorted(out)
+
+
+def _check_rows(A, L, samples, A_ref, L_ref, dtype, what):
+    got_A = np.stack([A[s] for s in samples])
+    got_L = np.array([L[s] for s in samples])
+    assert_close_A(got_A, A_ref, dtype, what)
+    assert_close_L(got_L, L_ref, what)
+
+
+def _oracle_full_rows(wl, st, samples, A_out_rows, L_out_rows):
+    """A_full of the sampled rows: cached prefix rows merged with the block partial."""
+    A_in, L_in = oracle.block_partial(st.q, st.k_in, st.v_in, wl.spec.dtype)
+    ai = np.stack([A_in[s] for s in samples])
+    li = np.array([L_in[s] for s in samples])
+    return oracle.merge(A_out_rows, L_out_rows, ai, li)
+
+
+@pytest.mark.parametrize("name", ["dllm", "gqa", "video", "losa"])
+def test_dense_prefix_partial_full_size(name):
+    wl = make_workload(name)
+    sp = wl.spec
+    kv = make_kv(wl.prefix, sp.dtype)
+    st = next(wl.steps(1))
+    q = dev(st.q, sp.dtype)
+    A = torch.zeros(sp.batch, sp.block, sp.n_heads_q, sp.head_dim, device="cuda")
+    L = torch.zeros(sp.batch, sp.block, sp.n_heads_q, device="cuda")
+    ws = torch.empty(fb.fb_workspace_size(kv, sp.block, sp.n_heads_q), dtype=torch.uint8,
+                     device="cuda")
+    fb.fb_prefix_attn(q, kv, A, L, ws)
+    sync()
+    A, L = cpu(A), cpu(L)
+    assert np.isfinite(A).all() and np.isfinite(L).all()
+    samples = _samples(sp, 48, 7)
+    A_ref, L_ref = oracle.prefix_partial_samples(wl.prefix, st.q, sp.dtype, samples)
+    _check_rows(A, L, samples, A_ref, L_ref, sp.dtype, name)
+
+
+@pytest.mark.parametrize("name,n_steps", [("dllm", 32), ("gqa", 10)])
+def test_threshold_block_full_size(name, n_steps):
+    """tau controller over the block's steps: per-sequence decisions exact,
+    sampled A_full within tolerance (oracle rows cached at recompute steps)."""
+    wl = make_workload(name)
+    sp = wl.spec
+    kv = make_kv(wl.prefix, sp.dtype)
+    blk = BlockAttention(kv, sp.block, sp.n_heads_q, "threshold", tau=sp.tau)
+    samples = _samples(sp, 24, 11)
+    A = torch.zeros(sp.batch, sp.block, sp.n_heads_q, sp.head_dim, device="cuda")
+    L = torch.zeros(sp.batch, sp.block, sp.n_heads_q, device="cuda")
+    A_out_rows = L_out_rows = None
+    for st in wl.steps(n_steps):
+        blk.step(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L,
+                 m_updated=st.m_updated)
+        sync()
+        rec = [st.step == 0 or int(m) >= sp.tau for m in st.m_updated]
+        assert blk.recomputed == sum(rec)
+        fresh = [s for s in samples if rec[s[0]]]
+        if fresh:
+            a, l = oracle.prefix_partial_samples(wl.prefix, st.q, sp.dtype, fresh)
+            if A_out_rows is None:
+                A_out_rows = np.zeros((len(samples), sp.head_dim))
+                L_out_rows = np.zeros(len(samples))
+            for k, s in enumerate(fresh):
+                j = samples.index(s)
+                A_out_rows[j], L_out_rows[j] = a[k], l[k]
+        A_ref, L_ref = _oracle_full_rows(wl, st, samples, A_out_rows, L_out_rows)
+        _check_rows(cpu(A), cpu(L), samples, A_ref, L_ref, sp.dtype, f"{name} step {st.step}")
+
+
+def test_per_head_video_full_size():
+    """gamma controller at full video size: the GPU's cosine equals the oracle's
+    cosine on the GPU's own tiles bit for bit, masks follow it, and sampled
+    A_full rows match the oracle with the GPU's decisions (teacher forcing)."""
+    wl = make_workload("video")
+    sp = wl.spec
+    kv = make_kv(wl.prefix, sp.dtype)
+    blk = BlockAttention(kv, sp.block, sp.n_heads_q, "per_head", gamma=sp.gamma)
+    samples = _samples(sp, 24, 13)
+    A = torch.zeros(sp.batch, sp.block, sp.n_heads_q, sp.head_dim, device="cuda")
+    L = torch.zeros(sp.batch, sp.block, sp.n_heads_q, device="cuda")
+    A_out_rows = np.zeros((len(samples), sp.head_dim))
+    L_out_rows = np.zeros(len(samples))
+    reused = 0
+    for st in wl.steps(6):
+        mask = cpu(blk.t["head_mask"]).astype(bool)
+        blk.step(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L)
+        sync()
+        cur, prev = cpu(blk.a_out), cpu(blk.t["a_out_prev"])
+        nxt = cpu(blk.t["head_mask"]).astype(bool)
+        if st.step >= 1:
+            cos = cpu(blk.t["head_cos"])
+            for h in range(sp.n_heads_q):
+                if mask[0, h]:
+                    c = head_cosine(cur[0, :, h], prev[0, :, h])
+                    assert cos[0, h] == c, (st.step, h)
+                    assert nxt[0, h] == (c < sp.gamma)
+                else:
+                    assert not nxt[0, h]
+        reused += int((~mask).sum())
+        fresh = [s for s in samples if mask[s[0], s[2]]]
+        if fresh:
+            a, l = oracle.prefix_partial_samples(wl.prefix, st.q, sp.dtype, fresh)
+            for k, s in enumerate(fresh):
+                j = samples.index(s)
+                A_out_rows[j], L_out_rows[j] = a[k], l[k]
+        A_ref, L_ref = _oracle_full_rows(wl, st, samples, A_out_rows, L_out_rows)
+        _check_rows(cpu(A), cpu(L), samples, A_ref, L_ref, sp.dtype, f"video step {st.step}")
+    assert reused > 0, "at gamma = 0.95 some heads reuse within the first steps"
+
+
+def test_losa_full_size():
+    """LoSA at full size: step 0 dense; later steps' active rows and page unions
+    equal the oracle's exactly, and the refreshed rows match its sparse partial."""
+    wl = make_workload("losa")
+    sp = wl.spec
+    kv = make_kv(wl.prefix, sp.dtype)
+    blk = BlockAttention(kv, sp.block, sp.n_heads_q, "losa", n_active=sp.n_active,
+                         topk_pages=sp.topk_pages)
+    smin, smax = olosa.page_summary(wl.prefix, sp.dtype)
+    gmin = cpu(blk.page_min.float())
+    gmax = cpu(blk.page_max.float())
+    np.testing.assert_array_equal(gmin[0], smin[0])
+    np.testing.assert_array_equal(gmax[0], smax[0])
+    samples = _samples(sp, 16, 17)
+    A = torch.zeros(sp.batch, sp.block, sp.n_heads_q, sp.head_dim, device="cuda")
+    L = torch.zeros(sp.batch, sp.block, sp.n_heads_q, device="cuda")
+    q_prev = None
+    A_out_rows = L_out_rows = None
+    for st in wl.steps(4):
+        blk.step(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L)
+        sync()
+        if st.step == 0:
+            A_out_rows, L_out_rows = oracle.prefix_partial_samples(wl.prefix, st.q, sp.dtype,
+                                                                   samples)
+        else:
+            score = olosa.locality_score(st.q, q_prev, sp.dtype)
+            act = olosa.active_rows(score, sp.n_active)
+            np.testing.assert_array_equal(cpu(blk.t["active_rows"]), act)
+            _, union = olosa.select_pages(wl.prefix, st.q, sp.dtype, act, sp.topk_pages, smin,
+                                          smax)
+            for (b, hk), pages in union.items():
+                cnt = int(cpu(blk.t["union_count"])[b, hk])
+                assert cnt == len(pages)
+                np.testing.assert_array_equal(cpu(blk.t["union_list"])[b, hk, :cnt], pages)
+            fresh = olosa.sparse_partial(wl.prefix, st.q, sp.dtype, act, union)
+            a_gpu, l_gpu = cpu(blk.a_out), cpu(blk.l_out)
+            keys = list(fresh)
+            assert_close_A(np.stack([a_gpu[k] for k in keys]),
+                           np.stack([fresh[k][0] for k in keys]), sp.dtype, f"step {st.step}")
+            assert_close_L(np.array([l_gpu[k] for k in keys]),
+                           np.array([fresh[k][1] for k in keys]), f"step {st.step}")
+            for j, s in enumerate(samples):
+                if s in fresh:
+                    A_out_rows[j], L_out_rows[j] = fresh[s]
+        A_ref, L_ref = _oracle_full_rows(wl, st, samples, A_out_rows, L_out_rows)
+        _check_rows(cpu(A), cpu(L), samples, A_ref, L_ref, sp.dtype, f"losa step {st.step}")
+        q_prev = st.q

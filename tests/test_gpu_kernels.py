@@ -52,6 +52,15 @@ PREFIX_CASES = {
                                       n_heads_kv=3)),
     "d64_bf16": ("dllm", dict(prefix_min=600, prefix_max=600, head_dim=64, n_heads_q=2,
                               n_heads_kv=2)),
+    # two long groups over many CTAs: partial segments at both ends of CTAs
+    "dllm_two_heads_long": ("dllm", dict(prefix_min=20011, prefix_max=20011, n_heads_q=2,
+                                         n_heads_kv=2)),
+    # paged, varied lengths, 64 stacked rows per kv head (16 rows x 4 q heads)
+    "gqa_paged_64_rows": ("gqa", dict(prefix_min=17, prefix_max=3000, batch=5, block=16,
+                                      n_heads_q=8, n_heads_kv=2)),
+    # more groups than CTAs, each a few tiles
+    "many_groups": ("gqa", dict(prefix_min=64, prefix_max=500, batch=40, block=8,
+                                n_heads_q=16, n_heads_kv=8)),
 }
 
 

@@ -60,18 +60,23 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
 
 
 def test_noalloc_rejects_shapes_beyond_its_static_scratch():
-    # Rejected on the host before any launch: one head of 64 rows over a
-    # 2^25-token prefix splits over every SM, and its partials (about 264 KB
-    # per SM, 39 MB on 148 SMs) exceed the 32 MiB static array.
-    assert torch.cuda.get_device_properties(0).multi_processor_count >= 128
+    # 128 stacked rows over a 75776-token prefix split over every SM: their
+    # partials (39 MB on 148 SMs) exceed the 32 MiB static array, so the call is
+    # refused on the host. The buffers are real and sized for the shapes, so
+    # even a launch would only read memory it owns.
+    assert torch.cuda.get_device_properties(0).multi_processor_count >= 140
+    L, B = 75776, 128
+    k = torch.zeros(L, 1, 128, dtype=torch.bfloat16, device="cuda")
+    v = torch.zeros_like(k)
+    q = torch.zeros(1, B, 1, 128, dtype=torch.bfloat16, device="cuda")
+    A = torch.full((1, B, 1, 128), 5.0, device="cuda")
+    Lo = torch.full((1, B, 1), 5.0, device="cuda")
+    kv = fb.KV(k, v, seq_len=None, page_table=None, page_size=16, max_seq_len=L)
     lib = fb.load_library()
-    buf = torch.zeros(1 << 20, dtype=torch.bfloat16, device="cuda")
-    kv = fb.fb_kv(buf.data_ptr(), buf.data_ptr(), None, None, 1 << 30, 1, 1, 128, 16, 0,
-                  1 << 25, fb.FB_BF16)
-    rc = lib.fb_prefix_attn_noalloc(buf.data_ptr(), 64, 1, ctypes.c_float(1.0),
-                                    ctypes.byref(kv), None, buf.data_ptr(), buf.data_ptr(),
+    rc = lib.fb_prefix_attn_noalloc(q.data_ptr(), B, 1, ctypes.c_float(1.0), ctypes.byref(kv.c),
+                                    None, A.data_ptr(), Lo.data_ptr(),
                                     torch.cuda.current_stream().cuda_stream)
-    assert rc == fb.FB_ERR_WORKSPACE
+    assert rc == fb.FB_ERR_WORKSPACE, rc
     assert b"static" in lib.fb_last_error()
     sync()
-    assert float(buf.float().abs().max()) == 0.0  # nothing was launched
+    assert float(A.min()) == 5.0 and float(A.max()) == 5.0  # nothing was launched
