@@ -52,7 +52,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=3, help="untimed blocks before timing")
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--mode", choices=["all", "reuse", "dense", "losa", "prefix"], default="all",
+    p.add_argument("--mode", choices=["all", "reuse", "dense", "losa", "prefix", "block"],
+                   default="all",
                    help="all: the contract line; one mode: time only that mode (for profiling)")
     p.add_argument("--workload", choices=["dllm", "tiny", "gqa", "video", "losa"],
                    default="dllm", help="dllm is the contract workload; the others are for "
@@ -269,15 +270,18 @@ def run_ours(args, rank, world, local):
         hL.copy_(L, non_blocking=True)
 
     K, W = args.steps, args.warmup
-    if args.mode == "prefix":  # only the dense prefix call, eager (for profilers)
+    if args.mode in ("prefix", "block"):  # one call kind only, eager (for profilers)
         for _ in range(W + K):
             for s in range(S):
                 flush.zero_()
-                prefix_call(s)
+                if args.mode == "prefix":
+                    prefix_call(s)
+                else:
+                    fb.fb_block_attn(dq[s], dk[s], dv[s], a_in, l_in)
         torch.cuda.synchronize()
         fb.fb_device_status()
         if rank == 0:
-            print(json.dumps({"mode": "prefix", "calls": (W + K) * S}))
+            print(json.dumps({"mode": args.mode, "calls": (W + K) * S}))
         return
     # warm-up of every path (eager, untimed): also sets kernel attributes
     for _ in range(max(1, W)):

@@ -61,6 +61,7 @@ struct AttnArgs {
   float* a_out;     // [batch, B, Hq, D]
   float* l_out;     // [batch, B, Hq] natural log
   float* a_prev;    // optional: old a_out rows are copied here before overwrite
+  int* tickets;        // persistent kernel: [batch * Hkv], zero at launch
   const float* mrg_a;  // optional second partial merged into every final row (FlashBlock merge)
   const float* mrg_l;
 };
@@ -650,7 +651,19 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 // ---------------------------------------------------------------------------
 constexpr int kF32Rows = 16;
 
-template <int D>
+template <typename T>
+__device__ __forceinline__ float elem_f32(const T* p, long long i);
+template <>
+__device__ __forceinline__ float elem_f32<float>(const float* p, long long i) {
+  return p[i];
+}
+template <>
+__device__ __forceinline__ float elem_f32<__nv_bfloat16>(const __nv_bfloat16* p, long long i) {
+  return __bfloat162float(p[i]);
+}
+
+// fp32 attention partial (T = float); inputs are read through elem_f32.
+template <typename T, int D>
 __global__ void __launch_bounds__(128) attn_f32_kernel(const __grid_constant__ AttnArgs a) {
   constexpr int NV = D / 32;
   __shared__ float Ks[32][D + 1];  // half a tile; +1: lanes reading different keys hit different banks
@@ -668,9 +681,9 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const __grid_constant__ A
   const int tile0 = split * a.tiles_per_split;
   const int n_it = max(0, min(a.tiles_per_split, n_tiles - tile0));
   const int n_chunks = kTK / a.chunk;
-  const float* qf = static_cast<const float*>(a.q);
-  const float* kg = static_cast<const float*>(a.k);
-  const float* vg = static_cast<const float*>(a.v);
+  const T* qf = static_cast<const T*>(a.q);
+  const T* kg = static_cast<const T*>(a.k);
+  const T* vg = static_cast<const T*>(a.v);
 
   for (int idx = tid; idx < kF32Rows * D; idx += blockDim.x) {
     const int rl = idx / D, c = idx % D;
@@ -679,7 +692,7 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const __grid_constant__ A
     if (r < a.R) {
       int i, h;
       row_of(a, b, hk, r, i, h);
-      v = qf[(((long long)b * a.B + i) * a.Hq + h) * D + c];
+      v = elem_f32<T>(qf, (((long long)b * a.B + i) * a.Hq + h) * D + c);
     }
     Qs[rl][c] = v;
   }
@@ -712,8 +725,8 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const __grid_constant__ A
         float kv = 0.f, vv = 0.f;
         if (off < meta[ci]) {  // keys outside the key set stay 0 (and are masked below)
           const long long e = ((slots[ci] + off) * a.Hkv + hk) * D + c;
-          kv = kg[e];
-          vv = vg[e];
+          kv = elem_f32<T>(kg, e);
+          vv = elem_f32<T>(vg, e);
         }
         Ks[kr][c] = kv;
         Vs[kr][c] = vv;

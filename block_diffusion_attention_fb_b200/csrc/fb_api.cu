@@ -14,6 +14,7 @@
 
 #include "../../include/fb.h"
 #include "attn.cuh"
+#include "attn_persistent.cuh"
 #include "attn_tc.cuh"
 #include "cosine.cuh"
 #include "losa.cuh"
@@ -70,6 +71,11 @@ int sm_count() {
 
 size_t elem_size(fb_dtype t) { return t == FB_BF16 ? 2 : 4; }
 
+// Resident-CTA waves the split-KV plan aims for.
+#ifndef FB_SPLIT_WAVES
+#define FB_SPLIT_WAVES 4
+#endif
+
 // --------------------------------------------------------------------------
 // Split-KV plan: row tiles per (b, hk), and how many kTK-key tiles each CTA
 // streams, chosen so that the grid covers the GPU for about four waves at two
@@ -102,7 +108,7 @@ Plan make_plan(fb_dtype dt, int batch, int Hkv, int R, int max_tiles, int num_sm
   }
   p.n_row_tiles = ceil_div(R, p.row_tile);
   const long long units = (long long)batch * Hkv * p.n_row_tiles;
-  const long long target = (long long)(num_sms > 0 ? num_sms : 148) * ctas_per_sm * 4;
+  const long long target = (long long)(num_sms > 0 ? num_sms : 148) * ctas_per_sm * FB_SPLIT_WAVES;
   max_tiles = max_tiles < 1 ? 1 : max_tiles;
   long long splits = (target + units - 1) / units;
   if (splits < 1) splits = 1;
@@ -117,6 +123,44 @@ size_t partial_bytes(const Plan& p, int batch, int Hkv, int R, int D) {
   if (p.n_splits <= 1) return 0;
   const size_t rows = (size_t)p.n_splits * batch * Hkv * R;
   return round_up(rows * D * 4, 256) + round_up(rows * 4, 256);
+}
+
+// The persistent kernel serves the LoSA gather (bf16, page lists, at most one
+// 64-row tile per kv head): union sizes are known only on the device, and it
+// balances the tiles actually present over the SMs. Dense prefixes run on the
+// grid kernel, whose three-stage pipeline streams faster (measured: dllm prefix
+// 135 us against 156 us).
+bool use_persistent(fb_dtype dt, int batch, int Hkv, int R, bool page_list) {
+  return dt == FB_BF16 && page_list && R <= 64 && (long long)batch * Hkv <= kMaxGroupsP;
+}
+
+// Persistent launch: CTAs (two per SM, at most one per tile) and workspace
+// (two partial slots per CTA + one ticket per group).
+struct PersistPlan {
+  int n_cta;
+  size_t o_off, l_off, t_off, bytes;
+};
+
+PersistPlan persist_plan(int batch, int Hkv, int R, int D, int max_tiles, int num_sms) {
+  PersistPlan p{};
+  const long long upper = (long long)batch * Hkv * (max_tiles < 1 ? 1 : max_tiles);
+  const long long slots = (long long)(num_sms > 0 ? num_sms : 148) * kPersistCtasPerSm;
+  p.n_cta = (int)(upper < slots ? upper : slots);
+  if (p.n_cta < 1) p.n_cta = 1;
+  const size_t rows = (size_t)p.n_cta * 2 * R;
+  p.o_off = 0;
+  p.l_off = round_up(rows * D * 4, 256);
+  p.t_off = p.l_off + round_up(rows * 4, 256);
+  p.bytes = p.t_off + round_up((size_t)batch * Hkv * 4, 256);
+  return p;
+}
+
+// Workspace bytes of one attention-partial launch, whichever kernel serves it.
+size_t partial_ws_bytes(fb_dtype dt, int batch, int Hkv, int R, int D, int max_tiles,
+                        int num_sms, bool page_list = false) {
+  if (use_persistent(dt, batch, Hkv, R, page_list))
+    return persist_plan(batch, Hkv, R, D, max_tiles, num_sms).bytes;
+  return partial_bytes(make_plan(dt, batch, Hkv, R, max_tiles, num_sms, D), batch, Hkv, R, D);
 }
 
 // Workspace regions shared by every entry point (offsets in bytes).
@@ -138,17 +182,15 @@ WsLayout ws_layout(const fb_kv* kv, int B, int Hq, int n_active, int topk, int n
   WsLayout w{};
   const int G = Hq / kv->n_heads_kv, D = kv->head_dim;
   const int R = B * G;
-  const Plan pd = make_plan(kv->dtype, kv->batch, kv->n_heads_kv, R, ceil_div(kv->max_seq_len, kTK),
-                            num_sms, D);
-  size_t part = partial_bytes(pd, kv->batch, kv->n_heads_kv, R, D);
+  size_t part = partial_ws_bytes(kv->dtype, kv->batch, kv->n_heads_kv, R, D,
+                                 ceil_div(kv->max_seq_len, kTK), num_sms);
   size_t scores = 0;
   if (n_active > 0 && topk > 0) {
     const int na = n_active < B ? n_active : B;
     const int per_tile = kTK / (kv->page_size < kTK ? kv->page_size : kTK);
     const int ent = max_union_entries(kv, G, na, topk);
-    const Plan pg = make_plan(kv->dtype, kv->batch, kv->n_heads_kv, na * G, ceil_div(ent, per_tile),
-                              num_sms, D);
-    const size_t pgb = partial_bytes(pg, kv->batch, kv->n_heads_kv, na * G, D);
+    const size_t pgb = partial_ws_bytes(kv->dtype, kv->batch, kv->n_heads_kv, na * G, D,
+                                        ceil_div(ent, per_tile), num_sms, true);
     part = part > pgb ? part : pgb;
     scores = round_up((size_t)kv->batch * na * Hq * logical_pages(kv) * 4, 256) +
              round_up((size_t)kv->batch * B * 4, 256);
@@ -286,6 +328,58 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
     a.chunk = kv->page_table ? (kv->page_size < kTK ? kv->page_size : kTK) : kTK;
     max_tiles = ceil_div(kv->max_seq_len, kTK);
   }
+  if (use_persistent(kv->dtype, kv->batch, Hkv, a.R, c.page_list != nullptr)) {
+    const PersistPlan pp = persist_plan(kv->batch, Hkv, a.R, D, max_tiles, c.num_sms);
+    if (!c.ws || c.ws_offset + pp.bytes > c.ws_bytes)
+      return fail(FB_ERR_WORKSPACE, "workspace too small: need %zu bytes at offset %zu, have %zu",
+                  pp.bytes, c.ws_offset, c.ws_bytes);
+    if (!aligned16(c.ws)) return fail(FB_ERR_ALIGN, "workspace not 16-byte aligned");
+    char* w = static_cast<char*>(c.ws) + c.ws_offset;
+    a.o_part = reinterpret_cast<float*>(w + pp.o_off);
+    a.lse_part = reinterpret_cast<float*>(w + pp.l_off);
+    a.tickets = reinterpret_cast<int*>(w + pp.t_off);
+    // tickets count a group's partials in; they start at zero on every call
+    if (cudaMemsetAsync(a.tickets, 0, (size_t)kv->batch * Hkv * 4, stream) != cudaSuccess)
+      return fail(FB_ERR_CUDA, "ticket reset failed");
+    a.row_tile = 64;
+    a.n_row_tiles = 1;
+    a.n_splits = 1;
+    a.tiles_per_split = max_tiles;
+    CUtensorMap tk, tv;
+    int rc = make_tmap(&tk, kv->k, D, Hkv, kv->n_slots, a.chunk);
+    if (rc) return rc;
+    rc = make_tmap(&tv, kv->v, D, Hkv, kv->n_slots, a.chunk);
+    if (rc) return rc;
+    const int rg = a.R <= 16 ? 1 : (a.R <= 32 ? 2 : 4);
+#define FB_LAUNCH_PERSIST(DD, RGV)                                                       \
+  do {                                                                                   \
+    auto kfn = attn_bf16_persistent<DD, RGV>;                                            \
+    static bool attr_set = false;                                                        \
+    if (!attr_set) {                                                                     \
+      cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,             \
+                           PersistSmem<DD>::kBytes);                                     \
+      attr_set = true;                                                                   \
+    }                                                                                    \
+    kfn<<<pp.n_cta, kAttnThreads, PersistSmem<DD>::kBytes, stream>>>(a, tk, tv);         \
+  } while (0)
+    if (D == 128) {
+      if (rg == 1)
+        FB_LAUNCH_PERSIST(128, 1);
+      else if (rg == 2)
+        FB_LAUNCH_PERSIST(128, 2);
+      else
+        FB_LAUNCH_PERSIST(128, 4);
+    } else {
+      if (rg == 1)
+        FB_LAUNCH_PERSIST(64, 1);
+      else if (rg == 2)
+        FB_LAUNCH_PERSIST(64, 2);
+      else
+        FB_LAUNCH_PERSIST(64, 4);
+    }
+#undef FB_LAUNCH_PERSIST
+    return check_launch("persistent attention kernel");
+  }
   Plan p = make_plan(kv->dtype, kv->batch, Hkv, a.R, max_tiles, c.num_sms, D);
   if (c.single_split) {
     p.tiles_per_split = max_tiles < 1 ? 1 : max_tiles;
@@ -309,9 +403,9 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
   const dim3 grid(p.n_row_tiles * p.n_splits, Hkv, kv->batch);
   if (kv->dtype == FB_F32) {
     if (D == 128)
-      attn_f32_kernel<128><<<grid, 128, 0, stream>>>(a);
+      attn_f32_kernel<float, 128><<<grid, 128, 0, stream>>>(a);
     else
-      attn_f32_kernel<64><<<grid, 128, 0, stream>>>(a);
+      attn_f32_kernel<float, 64><<<grid, 128, 0, stream>>>(a);
   } else {
     CUtensorMap tk, tv;
     int rc = make_tmap(&tk, kv->k, D, Hkv, kv->n_slots, a.chunk);
@@ -430,6 +524,7 @@ int block_attn_impl(const void* q, const void* k_in, const void* v_in, int batch
   c.l_out = l_in;
   // the block is short: one split per (b, hk, row tile), no workspace needed
   c.single_split = true;
+
   c.num_sms = sm_count();
   c.mrg_a = mrg_a;
   c.mrg_l = mrg_l;
@@ -541,6 +636,8 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
       !union_count)
     return fail(FB_ERR_ARG, "NULL argument");
   if (n_active < 0 || topk_pages < 0) return fail(FB_ERR_ARG, "n_active / topk_pages < 0");
+  if (!aligned16(page_min) || !aligned16(page_max) || !aligned16(q_prev))
+    return fail(FB_ERR_ALIGN, "page summaries / q_prev not 16-byte aligned");
   const KvView v = kv_view(kv);
   const int D = v.D, Hq = n_heads_q, G = Hq / v.Hkv;
   const int na = n_active < B ? n_active : B;
@@ -568,40 +665,62 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
     return e == cudaSuccess ? FB_OK : fail(FB_ERR_CUDA, "losa_select memset: %s", cudaGetErrorString(e));
   }
   const dim3 g1(B, kv->batch);
-  if (N2 * 4 > 48 * 1024) {
-    cudaFuncSetAttribute(locality_score_kernel<__nv_bfloat16>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, N2 * 4);
-    cudaFuncSetAttribute(locality_score_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         N2 * 4);
+  if (N2 >= 256 && N2 <= 256 * 32) {
+    // register tree (E elements per thread)
+#define FB_LOC(TT, EE)                                                                         \
+  locality_score_reg_kernel<TT, EE><<<g1, 256, 0, stream>>>(static_cast<const TT*>(q_cur),     \
+                                                             static_cast<const TT*>(q_prev), B, \
+                                                             N, rs)
+#define FB_LOC_E(TT)          \
+  switch (N2 / 256) {         \
+    case 1: FB_LOC(TT, 1); break;   \
+    case 2: FB_LOC(TT, 2); break;   \
+    case 4: FB_LOC(TT, 4); break;   \
+    case 8: FB_LOC(TT, 8); break;   \
+    case 16: FB_LOC(TT, 16); break; \
+    default: FB_LOC(TT, 32); break; \
   }
-  if (kv->dtype == FB_BF16)
-    locality_score_kernel<__nv_bfloat16><<<g1, 256, N2 * 4, stream>>>(
-        static_cast<const __nv_bfloat16*>(q_cur), static_cast<const __nv_bfloat16*>(q_prev), B, N,
-        N2, rs);
-  else
-    locality_score_kernel<float><<<g1, 256, N2 * 4, stream>>>(
-        static_cast<const float*>(q_cur), static_cast<const float*>(q_prev), B, N, N2, rs);
+    if (kv->dtype == FB_BF16) {
+      FB_LOC_E(__nv_bfloat16)
+    } else {
+      FB_LOC_E(float)
+    }
+#undef FB_LOC_E
+#undef FB_LOC
+  } else {
+    if (N2 * 4 > 48 * 1024) {
+      cudaFuncSetAttribute(locality_score_kernel<__nv_bfloat16>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, N2 * 4);
+      cudaFuncSetAttribute(locality_score_kernel<float>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, N2 * 4);
+    }
+    if (kv->dtype == FB_BF16)
+      locality_score_kernel<__nv_bfloat16><<<g1, 256, N2 * 4, stream>>>(
+          static_cast<const __nv_bfloat16*>(q_cur), static_cast<const __nv_bfloat16*>(q_prev), B,
+          N, N2, rs);
+    else
+      locality_score_kernel<float><<<g1, 256, N2 * 4, stream>>>(
+          static_cast<const float*>(q_cur), static_cast<const float*>(q_prev), B, N, N2, rs);
+  }
   rc = check_launch("locality score kernel");
   if (rc) return rc;
   active_rows_kernel<<<kv->batch, 256, B * 4, stream>>>(rs, B, na, active_rows);
   rc = check_launch("active rows kernel");
   if (rc) return rc;
-  // about four blocks of 8 page-warps per SM over all (b, hk)
-  const int px = max(1, min(ceil_div(v.max_pages, 16),
-                            ceil_div((long long)num_sms * 4, (long long)v.Hkv * kv->batch)));
-  const dim3 g2(px, v.Hkv, kv->batch);
-  const int qsm = na * G * D * 4;
+  const dim3 g2(ceil_div(v.max_pages, kPsPages), v.Hkv, kv->batch);
+  const int psm = na * G * D * 4 + 2 * kPsPages * (D + 4 / (int)elem_size(kv->dtype)) *
+                                       (int)elem_size(kv->dtype);
   if (kv->dtype == FB_BF16) {
     auto kfn = D == 128 ? page_score_kernel<__nv_bfloat16, 128> : page_score_kernel<__nv_bfloat16, 64>;
-    if (qsm > 48 * 1024) cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, qsm);
-    kfn<<<g2, 256, qsm, stream>>>(static_cast<const __nv_bfloat16*>(q_cur), active_rows, B, Hq, G,
+    if (psm > 48 * 1024) cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, psm);
+    kfn<<<g2, 256, psm, stream>>>(static_cast<const __nv_bfloat16*>(q_cur), active_rows, B, Hq, G,
                                   na, static_cast<const __nv_bfloat16*>(page_min),
                                   static_cast<const __nv_bfloat16*>(page_max), v, page_scores,
                                   union_bitmap, words);
   } else {
     auto kfn = D == 128 ? page_score_kernel<float, 128> : page_score_kernel<float, 64>;
-    if (qsm > 48 * 1024) cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, qsm);
-    kfn<<<g2, 256, qsm, stream>>>(static_cast<const float*>(q_cur), active_rows, B, Hq, G, na,
+    if (psm > 48 * 1024) cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, psm);
+    kfn<<<g2, 256, psm, stream>>>(static_cast<const float*>(q_cur), active_rows, B, Hq, G, na,
                                   static_cast<const float*>(page_min),
                                   static_cast<const float*>(page_max), v, page_scores,
                                   union_bitmap, words);
@@ -797,9 +916,8 @@ int fb_prefix_attn_noalloc(const void* q, int32_t B, int32_t n_heads_q, float sc
   if (!a_out || !l_out) return fail(FB_ERR_ARG, "a_out / l_out is NULL");
   const int num_sms = sm_count();
   const int R = B * (n_heads_q / kv->n_heads_kv);
-  const Plan p = make_plan(kv->dtype, kv->batch, kv->n_heads_kv, R, ceil_div(kv->max_seq_len, kTK),
-                           num_sms, kv->head_dim);
-  const size_t need = partial_bytes(p, kv->batch, kv->n_heads_kv, R, kv->head_dim);
+  const size_t need = partial_ws_bytes(kv->dtype, kv->batch, kv->n_heads_kv, R, kv->head_dim,
+                                       ceil_div(kv->max_seq_len, kTK), num_sms);
   if (need > (size_t)FB_NOALLOC_SCRATCH_BYTES)
     return fail(FB_ERR_WORKSPACE,
                 "fb_prefix_attn_noalloc: these shapes need %zu bytes of scratch but the static "

@@ -124,6 +124,47 @@ __global__ void __launch_bounds__(256)
   if (threadIdx.x == 0) score[(long long)b * B + i] = xs[0];
 }
 
+// Same score with the tree in registers: 256 threads, thread t owns elements
+// n = t + 256 j (j < E, E = N2 / 256), so the tree levels with stride >= 256
+// pair j with j + E/2, ... inside the thread; strides 128..32 go through
+// shared memory and 16..1 through xor shuffles (lane t + s for t < s).
+template <typename T, int E>
+__global__ void __launch_bounds__(256)
+    locality_score_reg_kernel(const T* __restrict__ qc, const T* __restrict__ qp, int B, int N,
+                              float* __restrict__ score) {
+  __shared__ float red[256];
+  const int i = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+  const long long off = ((long long)b * B + i) * N;
+  float x[E];
+#pragma unroll
+  for (int j = 0; j < E; ++j) {
+    const int n = t + 256 * j;
+    float v = 0.f;
+    if (n < N) {
+      const float d = __fsub_rn(ld_f32<T>(qc + off + n), ld_f32<T>(qp + off + n));
+      v = __fmul_rn(d, d);
+    }
+    x[j] = v;
+  }
+#pragma unroll
+  for (int s = E / 2; s >= 1; s >>= 1)
+#pragma unroll
+    for (int j = 0; j < s; ++j) x[j] = __fadd_rn(x[j], x[j + s]);
+  red[t] = x[0];
+  __syncthreads();
+#pragma unroll
+  for (int s = 128; s >= 32; s >>= 1) {
+    if (t < s) red[t] = __fadd_rn(red[t], red[t + s]);
+    __syncthreads();
+  }
+  if (t < 32) {
+    float v = red[t];
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, s));
+    if (t == 0) score[(long long)b * B + i] = v;
+  }
+}
+
 // Step 1b: the n_act highest-scoring rows of each sequence, in rank order
 // (score descending, then row ascending). O(B^2) ranks; B is a block size.
 __global__ void __launch_bounds__(256)
@@ -146,74 +187,81 @@ __global__ void __launch_bounds__(256)
 
 // ---------------------------------------------------------------------------
 // Step 3a: QUEST-style page scores u_p = tree_sum_c max(q_c kmin_c, q_c kmax_c)
-// for every active row a and q head h of kv head hk. One warp per page; lane l
-// holds channels l + 32 j, so the first levels of the tree (strides >= 32) run
-// inside the lane and the last five through xor shuffles.
+// for every active row a and q head h of kv head hk. A block stages the
+// summaries of kPsPages pages (coalesced) and the active q rows in shared
+// memory; then one thread per (page, row) forms the products and runs the
+// stride-halving tree in registers (level 1 pairs c with c + D/2, ...).
 // scores: [batch, n_act, Hq, max_pages]. Block (0, hk, b) also clears the
 // union bitmap of (b, hk) for the top-k kernel that follows.
 // ---------------------------------------------------------------------------
+constexpr int kPsPages = 64;
+
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
     page_score_kernel(const T* __restrict__ q, const int32_t* __restrict__ active, int B, int Hq,
                       int G, int n_act, const T* __restrict__ pmin, const T* __restrict__ pmax,
                       const KvView kv, float* __restrict__ scores, uint32_t* __restrict__ bitmap,
                       int words) {
-  constexpr int NV = D / 32;
-  extern __shared__ float qs[];  // [n_act * G][D]
+  // rows padded by one 32-bit word: threads reading the same channel of
+  // consecutive pages hit different banks
+  constexpr int PS = D + 4 / (int)sizeof(T);
+  constexpr int VE = 16 / (int)sizeof(T);  // elements per 16-byte global load
+  extern __shared__ float sm[];
+  const int RQ = n_act * G;
+  float* qs = sm;                                   // [RQ][D]
+  T* smn = reinterpret_cast<T*>(qs + RQ * D);       // [kPsPages][PS]
+  T* smx = smn + kPsPages * PS;
   const int hk = blockIdx.y, b = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p0 = blockIdx.x * kPsPages;
   if (blockIdx.x == 0)
     for (int w = threadIdx.x; w < words; w += blockDim.x)
       bitmap[((long long)b * kv.Hkv + hk) * words + w] = 0u;
-  const int RQ = n_act * G;
+  const int n_pages = (kv_tokens(kv, b) + kv.page_size - 1) / kv.page_size;
+  if (p0 >= n_pages) return;
   for (int idx = threadIdx.x; idx < RQ * D; idx += blockDim.x) {
     const int rq = idx / D, c = idx - (idx / D) * D;
     const int a_i = rq / G, g = rq - (rq / G) * G;
     const int i = active[b * n_act + a_i];
     qs[idx] = ld_f32<T>(q + (((long long)b * B + i) * Hq + hk * G + g) * D + c);
   }
+  // stage the summaries with 16-byte loads (rows of one head are contiguous)
+  for (int idx = threadIdx.x; idx < kPsPages * (D / VE); idx += blockDim.x) {
+    const int pg = idx / (D / VE), cv = idx - (idx / (D / VE)) * (D / VE);
+    const int p = p0 + pg;
+    uint4 mn = make_uint4(0u, 0u, 0u, 0u), mx = make_uint4(0u, 0u, 0u, 0u);
+    if (p < n_pages) {
+      const long long so = (((long long)b * kv.max_pages + p) * kv.Hkv + hk) * D + cv * VE;
+      mn = *reinterpret_cast<const uint4*>(pmin + so);
+      mx = *reinterpret_cast<const uint4*>(pmax + so);
+    }
+    uint32_t* dn = reinterpret_cast<uint32_t*>(smn + pg * PS + cv * VE);  // 4-byte aligned
+    uint32_t* dx = reinterpret_cast<uint32_t*>(smx + pg * PS + cv * VE);
+    dn[0] = mn.x; dn[1] = mn.y; dn[2] = mn.z; dn[3] = mn.w;
+    dx[0] = mx.x; dx[1] = mx.y; dx[2] = mx.z; dx[3] = mx.w;
+  }
   __syncthreads();
-  const int n_pages = (kv_tokens(kv, b) + kv.page_size - 1) / kv.page_size;
-  const int stride = gridDim.x * (blockDim.x >> 5);
-  // two pages per warp per iteration: their loads are issued before any math
-  for (int p0 = blockIdx.x * (blockDim.x >> 5) + warp; p0 < n_pages; p0 += 2 * stride) {
-    float lo[2][NV], hi[2][NV];
+  for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
+    const int pg = task % kPsPages, rq = task / kPsPages;
+    const int p = p0 + pg;
+    if (p >= n_pages) continue;
+    const float* qr = qs + rq * D;
+    const T* mnr = smn + pg * PS;
+    const T* mxr = smx + pg * PS;
+    float y[D / 2];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int p = p0 + u * stride;
-      const long long so = (((long long)b * kv.max_pages + (p < n_pages ? p : p0)) * kv.Hkv + hk) * D;
-#pragma unroll
-      for (int j = 0; j < NV; ++j) {
-        lo[u][j] = ld_f32<T>(pmin + so + lane + 32 * j);
-        hi[u][j] = ld_f32<T>(pmax + so + lane + 32 * j);
-      }
+    for (int c = 0; c < D / 2; ++c) {
+      const float q0 = qr[c], q1 = qr[c + D / 2];
+      const float x0 = fmaxf(__fmul_rn(q0, ld_f32<T>(mnr + c)), __fmul_rn(q0, ld_f32<T>(mxr + c)));
+      const float x1 = fmaxf(__fmul_rn(q1, ld_f32<T>(mnr + c + D / 2)),
+                             __fmul_rn(q1, ld_f32<T>(mxr + c + D / 2)));
+      y[c] = __fadd_rn(x0, x1);
     }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int p = p0 + u * stride;
-      if (p >= n_pages) break;
-      for (int rq = 0; rq < RQ; ++rq) {
-        float x[NV];
+    for (int st = D / 4; st >= 1; st >>= 1)
 #pragma unroll
-        for (int j = 0; j < NV; ++j) {
-          const float qv = qs[rq * D + lane + 32 * j];
-          x[j] = fmaxf(__fmul_rn(qv, lo[u][j]), __fmul_rn(qv, hi[u][j]));
-        }
-        // lane l holds channels l + 32 j: tree levels with stride >= 32 pair
-        // j with j + s inside the lane; the last five use xor shuffles
-#pragma unroll
-        for (int s = NV / 2; s >= 1; s >>= 1)
-#pragma unroll
-          for (int j = 0; j < s; ++j) x[j] = __fadd_rn(x[j], x[j + s]);
-        float v = x[0];
-#pragma unroll
-        for (int s = 16; s >= 1; s >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, s));
-        if (lane == 0) {
-          const int a_i = rq / G, g = rq - (rq / G) * G;
-          scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = v;
-        }
-      }
-    }
+      for (int c = 0; c < st; ++c) y[c] = __fadd_rn(y[c], y[c + st]);
+    const int a_i = rq / G, g = rq - (rq / G) * G;
+    scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = y[0];
   }
 }
 
