@@ -230,6 +230,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[j & 1]);
       const int st = j % kTcStages;
+      // acquire the producer's tile metadata through the TMA barrier itself
+      // (its phase for tile j is complete: S_j was computed from that stage)
+      mbar_wait(&full_bar[st], (j / kTcStages) & 1, &abort_flag);
       const bool tile_full = meta_full[st] != 0;
       const int chunk = a.chunk;
       float mx = -INFINITY;
@@ -387,6 +390,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   }
   // ------------------------------- teardown ---------------------------------
+  // Warps 0 and 1 ran their loops on lane 0 alone: reconverge every warp before
+  // the block-wide barrier (an aligned barrier reached by a divergent warp is
+  // undefined and can complete without the busy lane, letting TMEM be freed
+  // under in-flight MMAs and leaving that lane waiting forever).
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

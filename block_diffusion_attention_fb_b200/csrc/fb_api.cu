@@ -86,11 +86,13 @@ struct Plan {
   int tiles_per_split, n_splits;
 };
 
-// The tcgen05 kernel (attn_tc.cuh) is not launched: it passes the short-key-range
-// parity cases but stalls on long key ranges (hundreds of tiles per CTA) and
-// stays disabled until that is understood. bf16 runs on the mma.sync kernel,
-// fp32 on the CUDA-core kernel.
-bool use_tc(fb_dtype dt, int D) { return false && dt == FB_BF16 && D == 128; }
+// Kernel choice for bf16, head_dim 128: the tcgen05 kernel when a kv head has
+// more than 64 stacked query rows (GQA groups, video blocks: its 128-row MMA
+// tiles are full), the mma.sync kernel for up to 64 rows (dLLM blocks: a
+// 128-row tile would be mostly padding and one softmax warpgroup per SM leaves
+// the stream latency-bound; measured dllm prefix 135 us against 191 us).
+// fp32 runs on the CUDA-core kernel.
+bool use_tc(fb_dtype dt, int D, int R) { return dt == FB_BF16 && D == 128 && R > 64; }
 
 Plan make_plan(fb_dtype dt, int batch, int Hkv, int R, int max_tiles, int num_sms, int D = 128) {
   Plan p{};
@@ -98,7 +100,7 @@ Plan make_plan(fb_dtype dt, int batch, int Hkv, int R, int max_tiles, int num_sm
   if (dt == FB_F32) {
     p.row_tile = kF32Rows;
     p.rg = 1;
-  } else if (use_tc(dt, D)) {
+  } else if (use_tc(dt, D, R)) {
     p.row_tile = kTcRows;
     p.rg = 0;
     ctas_per_sm = 1;
@@ -423,7 +425,7 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
     }                                                                                        \
     kfn<<<grid, kAttnThreads, smem, stream>>>(a, tk, tv);                                    \
   } while (0)
-    if (use_tc(kv->dtype, D)) {
+    if (use_tc(kv->dtype, D, a.R)) {
       static bool tc_attr = false;
       if (!tc_attr) {
         cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
