@@ -11,9 +11,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libfb_b200.so")
 SOURCES = [os.path.join(HERE, "csrc", "fb_api.cu")]
-DEPS = SOURCES + [os.path.join(HERE, "csrc", f) for f in
-                  ("common.cuh", "attn.cuh", "losa.cuh", "cosine.cuh")] + \
-       [os.path.join(ROOT, "include", "fb.h")]
+DEPS = SOURCES + sorted(os.path.join(HERE, "csrc", f) for f in os.listdir(os.path.join(HERE, "csrc"))
+                        if f.endswith(".cuh")) + [os.path.join(ROOT, "include", "fb.h")]
 
 
 def nvcc_path() -> str:

@@ -374,6 +374,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  // Every CTA of this grid is resident from here on: let the split combine
+  // (launched as a programmatic dependent) be scheduled into the spare slots.
+  allow_dependent_launch();
 
   if (warp == kNWC) {
     // ----------------------------- producer -----------------------------
@@ -784,6 +787,9 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const __grid_constant__ A
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ AttnArgs a) {
+  // Launched as a programmatic dependent of the partial kernel: wait until that
+  // grid has completed and its partials are visible (no-op on a plain launch).
+  grid_dependency_wait();
   constexpr int NV = D / 32;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;

@@ -9,8 +9,11 @@
 #include <mutex>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <string>
+#include <utility>
+#include <vector>
 
 #include "../../include/fb.h"
 #include "attn.cuh"
@@ -69,17 +72,62 @@ int sm_count() {
   return n;
 }
 
+// The dynamic shared-memory limit is a per-device function attribute: raise it
+// for each (device, kernel) pair when a launch needs more than was set so far.
+int set_smem_once(const void* fn, int bytes) {
+  if (bytes <= 48 * 1024) return FB_OK;
+  struct Entry {
+    int dev;
+    const void* fn;
+    int bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(FB_ERR_CUDA, "cudaGetDevice failed");
+  std::lock_guard<std::mutex> lock(mu);
+  Entry* hit = nullptr;
+  for (auto& d : done)
+    if (d.dev == dev && d.fn == fn) hit = &d;
+  if (hit && hit->bytes >= bytes) return FB_OK;
+  const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess)
+    return fail(FB_ERR_CUDA, "cudaFuncSetAttribute(%d bytes): %s", bytes, cudaGetErrorString(e));
+  if (hit)
+    hit->bytes = bytes;
+  else
+    done.push_back(Entry{dev, fn, bytes});
+  return FB_OK;
+}
+
 size_t elem_size(fb_dtype t) { return t == FB_BF16 ? 2 : 4; }
 
-// Resident-CTA waves the split-KV plan aims for.
-#ifndef FB_SPLIT_WAVES
-#define FB_SPLIT_WAVES 4
-#endif
+// Tuning overrides read from the environment (0 or unset: automatic):
+//   FB_SPLIT_WAVES  resident-CTA waves of the streaming (mma.sync / fp32) plan
+//   FB_TC_SPLITS    splits per row tile of the tcgen05 plan
+int env_int(const char* name, int lo, int hi) {
+  const char* e = getenv(name);
+  if (e && *e) {
+    const int v = atoi(e);
+    if (v >= lo && v <= hi) return v;
+  }
+  return 0;
+}
 
 // --------------------------------------------------------------------------
 // Split-KV plan: row tiles per (b, hk), and how many kTK-key tiles each CTA
-// streams, chosen so that the grid covers the GPU for about four waves at two
-// resident CTAs per SM.
+// streams.
+//  - Streaming kernels (HBM-bound, two CTAs per SM): one wave of CTAs. The
+//    split count is the largest whose grid fits the resident slots, so every
+//    CTA starts at once, streams a long key range and pays its start-up and
+//    epilogue once (measured on the dllm prefix: 96 us at one wave, 110 us at
+//    two, 137 us at four).
+//  - tcgen05 kernel (compute-bound, one CTA per SM, long per-CTA work): the
+//    split count minimises the wave-quantised makespan ceil(u*s/slots)/s plus
+//    a small per-split cost (partials written and combined, per-CTA start-up);
+//    caches of several sequences (lengths vary, the plan sees only the
+//    longest) keep at most 128 tiles per CTA so short sequences free their
+//    SMs early.
 // --------------------------------------------------------------------------
 struct Plan {
   int row_tile, n_row_tiles, rg;
@@ -94,25 +142,48 @@ struct Plan {
 // fp32 runs on the CUDA-core kernel.
 bool use_tc(fb_dtype dt, int D, int R) { return dt == FB_BF16 && D == 128 && R > 64; }
 
+int tc_splits(long long units, int slots, int max_tiles, int batch) {
+  if (const int forced = env_int("FB_TC_SPLITS", 1, 4096)) return forced;
+  // cost in key-tile times: waves x (tiles per CTA + start-up) + combine reads
+  int best = 1;
+  double best_cost = 1e300;
+  const int s_max = max_tiles < 4 * slots ? max_tiles : 4 * slots;
+  for (int s = 1; s <= s_max; ++s) {
+    const long long waves = (units * s + slots - 1) / slots;
+    const double cost = (double)waves * (ceil_div(max_tiles, s) + 3) + 0.04 * (double)(units * s);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  const int s_len = ceil_div(max_tiles, 128);
+  if (batch > 1 && best < s_len) best = s_len;
+  return best;
+}
+
 Plan make_plan(fb_dtype dt, int batch, int Hkv, int R, int max_tiles, int num_sms, int D = 128) {
   Plan p{};
-  int ctas_per_sm = 2;
-  if (dt == FB_F32) {
-    p.row_tile = kF32Rows;
-    p.rg = 1;
-  } else if (use_tc(dt, D, R)) {
+  const int sms = num_sms > 0 ? num_sms : 148;
+  max_tiles = max_tiles < 1 ? 1 : max_tiles;
+  long long splits;
+  if (use_tc(dt, D, R)) {
     p.row_tile = kTcRows;
     p.rg = 0;
-    ctas_per_sm = 1;
+    p.n_row_tiles = ceil_div(R, p.row_tile);
+    splits = tc_splits((long long)batch * Hkv * p.n_row_tiles, sms, max_tiles, batch);
   } else {
-    p.rg = R <= 16 ? 1 : (R <= 32 ? 2 : 4);
-    p.row_tile = 16 * p.rg;
+    if (dt == FB_F32) {
+      p.row_tile = kF32Rows;
+      p.rg = 1;
+    } else {
+      p.rg = R <= 16 ? 1 : (R <= 32 ? 2 : 4);
+      p.row_tile = 16 * p.rg;
+    }
+    p.n_row_tiles = ceil_div(R, p.row_tile);
+    const long long units = (long long)batch * Hkv * p.n_row_tiles;
+    const int waves = env_int("FB_SPLIT_WAVES", 1, 64);
+    splits = (long long)sms * 2 * (waves ? waves : 1) / units;
   }
-  p.n_row_tiles = ceil_div(R, p.row_tile);
-  const long long units = (long long)batch * Hkv * p.n_row_tiles;
-  const long long target = (long long)(num_sms > 0 ? num_sms : 148) * ctas_per_sm * FB_SPLIT_WAVES;
-  max_tiles = max_tiles < 1 ? 1 : max_tiles;
-  long long splits = (target + units - 1) / units;
   if (splits < 1) splits = 1;
   if (splits > max_tiles) splits = max_tiles;
   p.tiles_per_split = ceil_div(max_tiles, splits);
@@ -356,12 +427,7 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
 #define FB_LAUNCH_PERSIST(DD, RGV)                                                       \
   do {                                                                                   \
     auto kfn = attn_bf16_persistent<DD, RGV>;                                            \
-    static bool attr_set = false;                                                        \
-    if (!attr_set) {                                                                     \
-      cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,             \
-                           PersistSmem<DD>::kBytes);                                     \
-      attr_set = true;                                                                   \
-    }                                                                                    \
+    if (int rc_ = set_smem_once((const void*)kfn, PersistSmem<DD>::kBytes)) return rc_;  \
     kfn<<<pp.n_cta, kAttnThreads, PersistSmem<DD>::kBytes, stream>>>(a, tk, tv);         \
   } while (0)
     if (D == 128) {
@@ -418,20 +484,11 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
   do {                                                                                       \
     auto kfn = attn_bf16_kernel<DD, RGV>;                                                    \
     const int smem = Bf16Smem<DD>::kBytes;                                                   \
-    static bool attr_set = false;                                                            \
-    if (!attr_set) {                                                                         \
-      cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);          \
-      attr_set = true;                                                                       \
-    }                                                                                        \
+    if (int rc_ = set_smem_once((const void*)kfn, smem)) return rc_;                       \
     kfn<<<grid, kAttnThreads, smem, stream>>>(a, tk, tv);                                    \
   } while (0)
     if (use_tc(kv->dtype, D, a.R)) {
-      static bool tc_attr = false;
-      if (!tc_attr) {
-        cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             TcSmem::kBytes);
-        tc_attr = true;
-      }
+      if (int rc_ = set_smem_once((const void*)attn_tc_kernel, TcSmem::kBytes)) return rc_;
       attn_tc_kernel<<<grid, kTcThreads, TcSmem::kBytes, stream>>>(a, tk, tv);
     } else if (D == 128) {
       if (p.rg == 1)
@@ -455,10 +512,19 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
   if (p.n_splits > 1) {
     const long long rows = (long long)kv->batch * Hkv * a.R;
     const int blocks = ceil_div(rows * 32, 256);
-    if (D == 128)
-      combine_kernel<128><<<blocks, 256, 0, stream>>>(a);
-    else
-      combine_kernel<64><<<blocks, 256, 0, stream>>>(a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = D == 128 ? cudaLaunchKernelEx(&cfg, combine_kernel<128>, a)
+                                   : cudaLaunchKernelEx(&cfg, combine_kernel<64>, a);
+    if (e != cudaSuccess)
+      return fail(FB_ERR_CUDA, "split combine kernel launch: %s", cudaGetErrorString(e));
     rc = check_launch("split combine kernel");
   }
   return rc;
@@ -690,12 +756,10 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
 #undef FB_LOC_E
 #undef FB_LOC
   } else {
-    if (N2 * 4 > 48 * 1024) {
-      cudaFuncSetAttribute(locality_score_kernel<__nv_bfloat16>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, N2 * 4);
-      cudaFuncSetAttribute(locality_score_kernel<float>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, N2 * 4);
-    }
+    rc = kv->dtype == FB_BF16
+             ? set_smem_once((const void*)locality_score_kernel<__nv_bfloat16>, N2 * 4)
+             : set_smem_once((const void*)locality_score_kernel<float>, N2 * 4);
+    if (rc) return rc;
     if (kv->dtype == FB_BF16)
       locality_score_kernel<__nv_bfloat16><<<g1, 256, N2 * 4, stream>>>(
           static_cast<const __nv_bfloat16*>(q_cur), static_cast<const __nv_bfloat16*>(q_prev), B,
@@ -714,14 +778,14 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
                                        (int)elem_size(kv->dtype);
   if (kv->dtype == FB_BF16) {
     auto kfn = D == 128 ? page_score_kernel<__nv_bfloat16, 128> : page_score_kernel<__nv_bfloat16, 64>;
-    if (psm > 48 * 1024) cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, psm);
+    if ((rc = set_smem_once((const void*)kfn, psm))) return rc;
     kfn<<<g2, 256, psm, stream>>>(static_cast<const __nv_bfloat16*>(q_cur), active_rows, B, Hq, G,
                                   na, static_cast<const __nv_bfloat16*>(page_min),
                                   static_cast<const __nv_bfloat16*>(page_max), v, page_scores,
                                   union_bitmap, words);
   } else {
     auto kfn = D == 128 ? page_score_kernel<float, 128> : page_score_kernel<float, 64>;
-    if (psm > 48 * 1024) cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, psm);
+    if ((rc = set_smem_once((const void*)kfn, psm))) return rc;
     kfn<<<g2, 256, psm, stream>>>(static_cast<const float*>(q_cur), active_rows, B, Hq, G, na,
                                   static_cast<const float*>(page_min),
                                   static_cast<const float*>(page_max), v, page_scores,
@@ -730,8 +794,7 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
   rc = check_launch("page score kernel");
   if (rc) return rc;
   const int ksm = v.max_pages * 4;
-  if (ksm > 48 * 1024)
-    cudaFuncSetAttribute(topk_pages_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ksm);
+  if ((rc = set_smem_once((const void*)topk_pages_kernel, ksm))) return rc;
   topk_pages_kernel<<<dim3(na * Hq, kv->batch), kTopkThreads, ksm, stream>>>(
       page_scores, v, Hq, G, na, topk_pages, union_bitmap, words);
   rc = check_launch("top-k pages kernel");

@@ -85,6 +85,10 @@ typedef struct fb_kv {
  * Bytes of workspace that fb_prefix_attn, losa_select, losa_gather and fb_step
  * need for these shapes (n_active/topk_pages may be 0 when LoSA is unused).
  * num_sms: SM count the split plan targets (0: query the current device).
+ * The split plan may be tuned through the environment (FB_SPLIT_WAVES: waves
+ * of resident CTAs for the streaming kernels; FB_TC_SPLITS: splits per row
+ * tile of the tcgen05 kernel); query the size under the same environment as
+ * the calls that use it.
  * Returns 0 on invalid arguments.
  */
 size_t fb_workspace_size(const fb_kv* kv, int32_t block, int32_t n_heads_q, int32_t n_active,

@@ -60,20 +60,21 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
 
 
 def test_noalloc_rejects_shapes_beyond_its_static_scratch():
-    # 128 stacked rows over a 75776-token prefix split over every SM: their
-    # partials (39 MB on 148 SMs) exceed the 32 MiB static array, so the call is
-    # refused on the host. The buffers are real and sized for the shapes, so
-    # even a launch would only read memory it owns.
-    assert torch.cuda.get_device_properties(0).multi_processor_count >= 140
-    L, B = 75776, 128
-    k = torch.zeros(L, 1, 128, dtype=torch.bfloat16, device="cuda")
+    # A video-shaped request (24 heads, 1664 block rows, 4096-token prefix) is
+    # split twice per 128-row tile on 140-148 SMs: its partials (41 MB) exceed
+    # the 32 MiB static array, so the call is refused on the host. The buffers
+    # are real and sized for the shapes, so even a launch would only read memory
+    # it owns.
+    assert 140 <= torch.cuda.get_device_properties(0).multi_processor_count <= 148
+    L, B, H = 4096, 1664, 24
+    k = torch.zeros(L, H, 128, dtype=torch.bfloat16, device="cuda")
     v = torch.zeros_like(k)
-    q = torch.zeros(1, B, 1, 128, dtype=torch.bfloat16, device="cuda")
-    A = torch.full((1, B, 1, 128), 5.0, device="cuda")
-    Lo = torch.full((1, B, 1), 5.0, device="cuda")
+    q = torch.zeros(1, B, H, 128, dtype=torch.bfloat16, device="cuda")
+    A = torch.full((1, B, H, 128), 5.0, device="cuda")
+    Lo = torch.full((1, B, H), 5.0, device="cuda")
     kv = fb.KV(k, v, seq_len=None, page_table=None, page_size=16, max_seq_len=L)
     lib = fb.load_library()
-    rc = lib.fb_prefix_attn_noalloc(q.data_ptr(), B, 1, ctypes.c_float(1.0), ctypes.byref(kv.c),
+    rc = lib.fb_prefix_attn_noalloc(q.data_ptr(), B, H, ctypes.c_float(1.0), ctypes.byref(kv.c),
                                     None, A.data_ptr(), Lo.data_ptr(),
                                     torch.cuda.current_stream().cuda_stream)
     assert rc == fb.FB_ERR_WORKSPACE, rc
