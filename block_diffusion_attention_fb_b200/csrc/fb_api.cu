@@ -19,6 +19,7 @@
 #include "attn.cuh"
 #include "attn_persistent.cuh"
 #include "attn_tc.cuh"
+#include "block_attn.cuh"
 #include "cosine.cuh"
 #include "losa.cuh"
 
@@ -563,6 +564,64 @@ KvView kv_view(const fb_kv* kv) {
   return v;
 }
 
+// Short blocks (bf16, B <= 64): the latency-built kernel of block_attn.cuh.
+// Rows per CTA: 16 per warp, 1 to 4 warps, fewer warps while that keeps the
+// grid within two CTAs per SM (more CTAs = more of the block's loads in flight).
+int block_attn_short(const void* q, const void* k_in, const void* v_in, int batch, int B, int Hq,
+                     int Hkv, int D, float scale, float* a_out, float* l_out, const float* mrg_a,
+                     const float* mrg_l, cudaStream_t stream) {
+  BlockArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k_in);
+  a.v = static_cast<const __nv_bfloat16*>(v_in);
+  a.mrg_a = mrg_a;
+  a.mrg_l = mrg_l;
+  a.a_out = a_out;
+  a.l_out = l_out;
+  a.batch = batch;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.R = B * a.G;
+  a.scale_log2 = scale * kLog2e;
+  if (batch == 0 || B == 0) return FB_OK;
+  if (!aligned16(mrg_a)) return fail(FB_ERR_ALIGN, "merge partner rows not 16-byte aligned");
+  const int tiles16 = ceil_div(a.R, 16);
+  const long long groups = (long long)batch * Hkv;
+  const int slots = 2 * (sm_count() > 0 ? sm_count() : 148);
+  int warps = 1;
+  while (warps < 4 && warps < tiles16 && groups * ceil_div(tiles16, warps) > slots) warps *= 2;
+  const int kt = ceil_div(B, 16);
+  const int smem = BlockSmem<128>::bytes(warps, kt, mrg_a != nullptr);
+  const int smem_d = D == 128 ? smem : BlockSmem<64>::bytes(warps, kt, mrg_a != nullptr);
+  const dim3 grid(ceil_div(a.R, 16 * warps), Hkv, batch);
+  if (grid.y > 65535 || grid.z > 65535) return fail(FB_ERR_SHAPE, "too many heads or sequences");
+#define FB_BLOCK_LAUNCH(DD, KTV)                                                       \
+  do {                                                                                 \
+    auto kfn = block_attn_kernel<DD, KTV>;                                             \
+    if (int rc_ = set_smem_once((const void*)kfn, smem_d)) return rc_;                \
+    kfn<<<grid, 32 * warps, smem_d, stream>>>(a);                                      \
+  } while (0)
+  if (D == 128) {
+    switch (kt) {
+      case 1: FB_BLOCK_LAUNCH(128, 1); break;
+      case 2: FB_BLOCK_LAUNCH(128, 2); break;
+      case 3: FB_BLOCK_LAUNCH(128, 3); break;
+      default: FB_BLOCK_LAUNCH(128, 4); break;
+    }
+  } else {
+    switch (kt) {
+      case 1: FB_BLOCK_LAUNCH(64, 1); break;
+      case 2: FB_BLOCK_LAUNCH(64, 2); break;
+      case 3: FB_BLOCK_LAUNCH(64, 3); break;
+      default: FB_BLOCK_LAUNCH(64, 4); break;
+    }
+  }
+#undef FB_BLOCK_LAUNCH
+  return check_launch("block attention kernel");
+}
+
 int block_attn_impl(const void* q, const void* k_in, const void* v_in, int batch, int B, int Hq,
                     int Hkv, int D, float scale, fb_dtype dt, float* a_in, float* l_in,
                     cudaStream_t stream, const float* mrg_a = nullptr,
@@ -582,6 +641,9 @@ int block_attn_impl(const void* q, const void* k_in, const void* v_in, int batch
   rc = validate_q(q, B, Hq, &kv);
   if (rc) return rc;
   if (!a_in || !l_in) return fail(FB_ERR_ARG, "a_in / l_in is NULL");
+  if (mrg_a && !mrg_l) return fail(FB_ERR_ARG, "merge partner without its L");
+  if (dt == FB_BF16 && (D == 64 || D == 128) && B <= 64) return block_attn_short(
+      q, k_in, v_in, batch, B, Hq, Hkv, D, scale, a_in, l_in, mrg_a, mrg_l, stream);
   PartialCall c{};
   c.q = q;
   c.B = B;

@@ -107,6 +107,15 @@ def test_prefix_attn_empty_and_short_sequences():
     ("gqa", dict(block=64, batch=2, n_heads_q=8, n_heads_kv=2, prefix_min=64, prefix_max=64)),
     ("video", dict(block=130, n_heads_q=2, n_heads_kv=2, prefix_min=64, prefix_max=64)),
     ("dllm", dict(block=5, n_heads_q=2, n_heads_kv=2, prefix_min=64, prefix_max=64)),
+    # short-block kernel: every key-tile count (B padded to 16, 32, 48, 64), GQA row
+    # stacking with a ragged last row tile, head_dim 64, a single-token block
+    ("dllm", dict(block=1, n_heads_q=3, n_heads_kv=3, prefix_min=64, prefix_max=64)),
+    ("dllm", dict(block=17, n_heads_q=2, n_heads_kv=2, prefix_min=64, prefix_max=64)),
+    ("gqa", dict(block=45, batch=3, n_heads_q=12, n_heads_kv=3, prefix_min=64, prefix_max=64)),
+    ("gqa", dict(block=64, batch=2, n_heads_q=32, n_heads_kv=8, prefix_min=64, prefix_max=64)),
+    ("dllm", dict(block=33, head_dim=64, n_heads_q=4, n_heads_kv=2, prefix_min=64,
+                  prefix_max=64)),
+    ("video", dict(block=65, n_heads_q=2, n_heads_kv=2, prefix_min=64, prefix_max=64)),
 ])
 def test_block_attn_matches_oracle(name, ov):
     wl = make_workload(name, **ov)

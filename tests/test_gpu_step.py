@@ -53,6 +53,27 @@ def test_threshold_steps_match_oracle(name, ov, tau):
         assert n_rec == sp.steps * sp.batch
 
 
+def test_threshold_steps_with_an_empty_prefix_side():
+    """A sequence with no prefix tokens has L_out = -inf: the fused merge must
+    return its in-block partial alone (FlashBlock merge with one empty side)."""
+    wl = make_workload("gqa", prefix_min=20, prefix_max=300, batch=3, block=24, n_heads_q=8,
+                       n_heads_kv=2, steps=4)
+    wl.prefix.seq_len[1] = 0
+    sp = wl.spec
+    kv = make_kv(wl.prefix, sp.dtype)
+    blk = BlockAttention(kv, sp.block, sp.n_heads_q, "threshold", tau=2)
+    ctl = ThresholdController(wl.prefix, sp.dtype, 2)
+    A, L = _out(sp)
+    for st in wl.steps():
+        blk.step(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L,
+                 m_updated=st.m_updated)
+        ref = ctl.step(st.step, st.q, st.k_in, st.v_in, st.m_updated)
+        sync()
+        assert np.isfinite(cpu(L)[1]).all()
+        assert_close_A(cpu(A), ref["A_full"], sp.dtype, f"step {st.step}")
+        assert_close_L(cpu(L), ref["L_full"], f"step {st.step}")
+
+
 def test_per_head_steps_match_oracle_with_bit_exact_cosine_replay():
     wl = make_workload("video", prefix_min=700, prefix_max=700, block=90, n_heads_q=6,
                        n_heads_kv=6, steps=8)
