@@ -18,7 +18,7 @@
 #include "../../include/fb.h"
 #include "attn.cuh"
 #include "attn_persistent.cuh"
-#include "attn_tc.cuh"
+#include "attn_tc2.cuh"
 #include "block_attn.cuh"
 #include "cosine.cuh"
 #include "losa.cuh"
@@ -168,10 +168,16 @@ Plan make_plan(fb_dtype dt, int batch, int Hkv, int R, int max_tiles, int num_sm
   max_tiles = max_tiles < 1 ? 1 : max_tiles;
   long long splits;
   if (use_tc(dt, D, R)) {
-    p.row_tile = kTcRows;
+    // two 128-row Q tiles per CTA; key ranges in whole 128-key tiles (an even
+    // number of 64-key metadata tiles)
+    p.row_tile = kT2Rows;
     p.rg = 0;
     p.n_row_tiles = ceil_div(R, p.row_tile);
-    splits = tc_splits((long long)batch * Hkv * p.n_row_tiles, sms, max_tiles, batch);
+    const int tiles128 = ceil_div(max_tiles, 2);
+    const int s = tc_splits((long long)batch * Hkv * p.n_row_tiles, sms, tiles128, batch);
+    p.tiles_per_split = 2 * ceil_div(tiles128, s);
+    p.n_splits = ceil_div(max_tiles, p.tiles_per_split);
+    return p;
   } else {
     if (dt == FB_F32) {
       p.row_tile = kF32Rows;
@@ -489,8 +495,8 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
     kfn<<<grid, kAttnThreads, smem, stream>>>(a, tk, tv);                                    \
   } while (0)
     if (use_tc(kv->dtype, D, a.R)) {
-      if (int rc_ = set_smem_once((const void*)attn_tc_kernel, TcSmem::kBytes)) return rc_;
-      attn_tc_kernel<<<grid, kTcThreads, TcSmem::kBytes, stream>>>(a, tk, tv);
+      if (int rc_ = set_smem_once((const void*)attn_tc2_kernel, Tc2Smem::kBytes)) return rc_;
+      attn_tc2_kernel<<<grid, kT2Threads, Tc2Smem::kBytes, stream>>>(a, tk, tv);
     } else if (D == 128) {
       if (p.rg == 1)
         FB_LAUNCH_BF16(128, 1);
