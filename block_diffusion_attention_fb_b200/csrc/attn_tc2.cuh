@@ -49,7 +49,7 @@ constexpr int kT2Rows = 2 * kT2TileRows;
 constexpr int kT2Producer = 0, kT2Mma = 1, kT2SoftA = 4, kT2SoftB = 8;
 constexpr uint32_t kT2Cols = 512;
 constexpr float kT2Rescale = 8.f;  // log2 of the largest P value before O is rescaled
-constexpr int kT2LowRegs = 80, kT2HighRegs = 208;
+constexpr int kT2LowRegs = 72, kT2HighRegs = 216;
 static_assert(4 * 32 * kT2LowRegs + 8 * 32 * kT2HighRegs <= kT2Threads * 168,
               "register split exceeds the launch's registers");
 
@@ -121,8 +121,8 @@ __global__ void __launch_bounds__(kT2Threads, 1)
   const uint32_t tmem = tmem_base_sh;
 
   // Register split (launch: 384 threads x 168 = 64512): warps 0-3 give theirs
-  // down to 80 (10240), the softmax warps take 208 (8 warps: 53248); the sum,
-  // 63488, fits, so the increase never waits for registers that cannot come.
+  // down to 72 (9216), the softmax warps take 216 (8 warps: 55296); the sum,
+  // 64512, fits, so the increase never waits for registers that cannot come.
   // Each role changes its budget inside its own branch, so the compiler knows
   // the budget of every region.
   if (warp == kT2Producer) {
@@ -132,7 +132,28 @@ __global__ void __launch_bounds__(kT2Threads, 1)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       int issued = 0;  // loads issued (K_0 = 0, V_0 = 1, K_1 = 2, ...)
-      long long slots[2 * kMaxChunks];
+      // Slots and valid counts of the chunks of tile `it` (chunk c covers keys
+      // [c * chunk, (c + 1) * chunk) of the 128-key tile; a sub-tile past the
+      // split's range gives valid = 0, a zero-filled box). Unrolled over the
+      // fixed maximum, so the page-table reads of a tile are independent
+      // loads in flight together; tile it + 1's are issued right after tile
+      // it's copies, ahead of the wait for a free slot.
+      constexpr int kC = 2 * kMaxChunks;
+      int sl_cur[kC], va_cur[kC], sl_nxt[kC], va_nxt[kC];
+      auto tile_slots = [&](int it, int (&sl)[kC], int (&va)[kC]) {
+#pragma unroll
+        for (int c = 0; c < kC; ++c) {
+          long long s_ = a.n_slots;
+          int v_ = 0;
+          if (c < 2 * n_chunks) {
+            const int sub = c / n_chunks, cc = c - sub * n_chunks;
+            if (2 * it + sub < n64) chunk_slot(a, b, hk, tile0 + 2 * it + sub, cc, s_, v_);
+          }
+          sl[c] = (int)s_;
+          va[c] = v_;
+        }
+      };
+      if (n_it > 0) tile_slots(0, sl_cur, va_cur);
       for (int n = 0; n < 2 * n_it; ++n) {
         const int it = n >> 1, is_v = n & 1;
         const int sl = n % kT2Slots;
@@ -140,15 +161,12 @@ __global__ void __launch_bounds__(kT2Threads, 1)
         if (!is_v) {
           const int me = it % kT2Meta;
           int all_full = 1;
-          for (int c = 0; c < 2 * n_chunks; ++c) {
-            // chunk c covers keys [c * chunk, (c + 1) * chunk) of the 128-key tile;
-            // a sub-tile past the split's range yields valid = 0 (zero-filled box)
-            const int sub = c / n_chunks, cc = c - sub * n_chunks;
-            int valid = 0;
-            slots[c] = a.n_slots;
-            if (2 * it + sub < n64) chunk_slot(a, b, hk, tile0 + 2 * it + sub, cc, slots[c], valid);
-            meta[me][c] = valid;
-            all_full &= (valid == a.chunk);
+#pragma unroll
+          for (int c = 0; c < kC; ++c) {
+            if (c < 2 * n_chunks) {
+              meta[me][c] = va_cur[c];
+              all_full &= (va_cur[c] == a.chunk);
+            }
           }
           meta_full[me] = all_full;
           mbar_arrive(&meta_bar[me]);  // release: the entry is written
@@ -156,12 +174,23 @@ __global__ void __launch_bounds__(kT2Threads, 1)
         mbar_arrive_expect_tx(&full_bar[sl], S::kKVTile);
         uint8_t* dst = base_ptr + (sKV0 - base) + sl * S::kKVTile;
         const CUtensorMap* tm = is_v ? &tmV : &tmK;
-        for (int c = 0; c < 2 * n_chunks; ++c) {
-          const int z = (int)slots[c];
-          tma_load_3d(dst + c * a.chunk * 128, tm, 0, hk, z, &full_bar[sl]);
-          tma_load_3d(dst + S::kKVHalf + c * a.chunk * 128, tm, 64, hk, z, &full_bar[sl]);
+#pragma unroll
+        for (int c = 0; c < kC; ++c) {
+          if (c < 2 * n_chunks) {
+            tma_load_3d(dst + c * a.chunk * 128, tm, 0, hk, sl_cur[c], &full_bar[sl]);
+            tma_load_3d(dst + S::kKVHalf + c * a.chunk * 128, tm, 64, hk, sl_cur[c],
+                        &full_bar[sl]);
+          }
         }
         ++issued;
+        if (is_v && it + 1 < n_it) {
+          tile_slots(it + 1, sl_nxt, va_nxt);
+#pragma unroll
+          for (int c = 0; c < kC; ++c) {
+            sl_cur[c] = sl_nxt[c];
+            va_cur[c] = va_nxt[c];
+          }
+        }
       }
       if (abort_flag) {
         // let copies already in flight land before the CTA's memory goes away
@@ -291,16 +320,26 @@ __global__ void __launch_bounds__(kT2Threads, 1)
       mbar_wait(&meta_bar[st], (j / kT2Meta) & 1, &abort_flag);  // acquire tile j's metadata
       const bool tile_full = meta_full[st] != 0;
       const int chunk = a.chunk;
-      float mx = -INFINITY;
+      if (!tile_full) {  // keys outside the key set: raw score -inf
 #pragma unroll
-      for (int k = 0; k < kT2Keys; ++k) {
-        float v = sv[k] * a.scale_log2;
-        if (!tile_full) {
+        for (int k = 0; k < kT2Keys; ++k) {
           const int ci = k / chunk;
-          if (k - ci * chunk >= meta[st][ci]) v = -INFINITY;
+          if (k - ci * chunk >= meta[st][ci]) sv[k] = -INFINITY;
         }
-        sv[k] = v;
-        mx = fmaxf(mx, v);
+      }
+      // Row maximum of the raw scores (scale > 0 keeps the order): eight
+      // independent three-input chains, then a short tree.
+      float mx;
+      {
+        float m8[8];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) m8[g] = sv[g];
+#pragma unroll
+        for (int k = 8; k < kT2Keys; k += 16)
+#pragma unroll
+          for (int g = 0; g < 8; ++g) m8[g] = fmax3(m8[g], sv[k + g], sv[k + 8 + g]);
+        mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+        mx *= a.scale_log2;
       }
       if (!tile_full && x == 0) {
         // the V row of a key outside the key set may hold any bits: zero it
@@ -346,17 +385,36 @@ __global__ void __launch_bounds__(kT2Threads, 1)
         }
       }
       const float bse = (m_used == -INFINITY) ? 0.f : m_used;
+      // P = 2^(s * scale_log2 - m): one packed FMA per key pair; 3 of every 8
+      // pairs take 2^x on the FMA pipe (exp2_poly2), the rest on the MUFU, so
+      // neither unit alone bounds the tile. Row sums in four packed chains.
+      const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+      const float2 nb2 = make_float2(-bse, -bse);
+      float2 lacc[4];
 #pragma unroll
       for (int c = 0; c < kT2Keys / 32; ++c) {
         uint32_t pk[16];
+        float2 lc = make_float2(0.f, 0.f);
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          const float p0 = fast_exp2(sv[c * 32 + 2 * k] - bse);
-          const float p1 = fast_exp2(sv[c * 32 + 2 * k + 1] - bse);
-          l_sum += p0 + p1;
-          pk[k] = pack_bf16(p0, p1);
+          const float2 xx = ffma2(make_float2(sv[c * 32 + 2 * k], sv[c * 32 + 2 * k + 1]), sc2, nb2);
+          float2 pp;
+          if ((k & 7) >= 5) {
+            pp = exp2_poly2(xx);
+          } else {
+            pp.x = fast_exp2(xx.x);
+            pp.y = fast_exp2(xx.y);
+          }
+          lc = fadd2(lc, pp);
+          pk[k] = pack_bf16(pp.x, pp.y);
         }
+        lacc[c] = lc;
         tmem_st16(t_s + c * 16, pk);  // P over the first 64 columns of S_X
+      }
+      {
+        const float2 l01 = fadd2(lacc[0], lacc[1]), l23 = fadd2(lacc[2], lacc[3]);
+        const float2 l4 = fadd2(l01, l23);
+        l_sum += l4.x + l4.y;
       }
       tmem_wait_st();
       tc_fence_before();

@@ -363,7 +363,16 @@ struct PartialCall {
   const float* mrg_l;
 };
 
+// The kernels order keys by raw score when forming the row maximum, which
+// needs a positive scale.
+int validate_scale(float scale) {
+  if (!(scale > 0.f) || !std::isfinite(scale))
+    return fail(FB_ERR_ARG, "scale must be positive and finite (got %g)", (double)scale);
+  return FB_OK;
+}
+
 int launch_partial(const PartialCall& c, cudaStream_t stream) {
+  if (int rc_ = validate_scale(c.scale)) return rc_;
   const fb_kv* kv = c.kv;
   const int D = kv->head_dim, Hkv = kv->n_heads_kv, G = c.Hq / Hkv;
   AttnArgs a{};
@@ -576,6 +585,7 @@ KvView kv_view(const fb_kv* kv) {
 int block_attn_short(const void* q, const void* k_in, const void* v_in, int batch, int B, int Hq,
                      int Hkv, int D, float scale, float* a_out, float* l_out, const float* mrg_a,
                      const float* mrg_l, cudaStream_t stream) {
+  if (int rc_ = validate_scale(scale)) return rc_;
   BlockArgs a{};
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.k = static_cast<const __nv_bfloat16*>(k_in);

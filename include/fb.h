@@ -26,6 +26,8 @@
  *  - Every call validates its arguments on the host before launching and
  *    returns FB_OK (0) or a negative FB_ERR_* code; the text of the last error
  *    of the calling thread is returned by fb_last_error().
+ *  - `scale` (the softmax scale applied to <q, k>) must be positive and
+ *    finite; anything else is FB_ERR_ARG.
  *  - Supported: head_dim 128 (bf16 and f32) or 64; page_size a power of two in
  *    [16, 128] for paged caches; 16-byte aligned tensors. Anything else is
  *    FB_ERR_SHAPE / FB_ERR_ALIGN.

@@ -275,4 +275,12 @@ def test_invalid_arguments_are_rejected_on_the_host():
     with pytest.raises(fb.FbError) as e:
         fb.fb_prefix_attn(q3, kv, A, L, ws)  # 3 q heads cannot share 2 kv heads
     assert e.value.code == fb.FB_ERR_SHAPE
+    big = torch.empty(fb.fb_workspace_size(kv, 32, 2), dtype=torch.uint8, device="cuda")
+    for bad_scale in (0.0, -1.0, float("nan"), float("inf")):
+        with pytest.raises(fb.FbError) as e:
+            fb.fb_prefix_attn(q, kv, A, L, big, scale=bad_scale)
+        assert e.value.code == fb.FB_ERR_ARG
+        with pytest.raises(fb.FbError) as e:
+            fb.fb_block_attn(q, q, q, A, L, scale=bad_scale)
+        assert e.value.code == fb.FB_ERR_ARG
     fb.fb_device_status()
