@@ -33,7 +33,7 @@ FB_LOSA = 2
 # Every entry point include/fb.h declares.
 EXPORTS = ("fb_workspace_size", "fb_prefix_attn", "fb_block_attn", "fb_merge", "fb_page_summary",
            "losa_select", "losa_gather", "fb_step", "fb_device_status", "fb_last_error",
-           "fb_kernel_launches", "fb_prefix_attn_noalloc")
+           "fb_kernel_launches", "fb_prefix_attn_noalloc", "fb_block_commit")
 
 
 class FbError(RuntimeError):
@@ -95,6 +95,7 @@ def load_library() -> ctypes.CDLL:
         "fb_last_error": (ctypes.c_char_p, []),
         "fb_kernel_launches": (ctypes.c_uint64, []),
         "fb_prefix_attn_noalloc": (ctypes.c_int, [P, I32, I32, F32, KV, P, P, P, P]),
+        "fb_block_commit": (ctypes.c_int, [KV, P, P, P, I32, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -258,6 +259,20 @@ def fb_prefix_attn_noalloc(q, kv: KV, a_out, l_out, scale: float = 1.0, head_mas
     _check(load_library().fb_prefix_attn_noalloc(_ptr(q), B, Hq, scale, ctypes.byref(kv.c),
                                                  _ptr(head_mask), _ptr(a_out), _ptr(l_out),
                                                  _stream(stream)))
+
+
+def fb_block_commit(kv: KV, seq_len_host, k_in, v_in, page_min=None, page_max=None,
+                    stream=None) -> None:
+    """Appends the block k_in / v_in [batch, B, Hkv, d] to the cache at the
+    positions given by seq_len_host (host int32 lengths before the call) and
+    updates the device lengths and, if given, the page summaries in place."""
+    import numpy as _np
+    lens = _np.ascontiguousarray(_np.asarray(seq_len_host, dtype=_np.int32))
+    if lens.shape != (kv.batch,):
+        raise ValueError("seq_len_host must hold one length per sequence")
+    _check(load_library().fb_block_commit(
+        ctypes.byref(kv.c), lens.ctypes.data_as(ctypes.c_void_p), _ptr(k_in), _ptr(v_in),
+        int(k_in.shape[1]), _ptr(page_min), _ptr(page_max), _stream(stream)))
 
 
 def fb_kernel_launches() -> int:

@@ -20,6 +20,7 @@
 #include "attn_persistent.cuh"
 #include "attn_tc2.cuh"
 #include "block_attn.cuh"
+#include "commit.cuh"
 #include "cosine.cuh"
 #include "losa.cuh"
 
@@ -691,8 +692,69 @@ int fb_device_status(void) {
   if (cudaMemcpyFromSymbol(&word, g_fb_error_word, sizeof(int)) != cudaSuccess)
     return fail(FB_ERR_CUDA, "reading the device error word failed");
   cudaMemcpyToSymbol(g_fb_error_word, &zero, sizeof(int));
+  if (word & kErrBadPage)
+    return fail(FB_ERR_ARG, "fb_block_commit met a page-table entry outside the pool (that page "
+                            "was left unwritten)");
   if (word) return fail(FB_ERR_TIMEOUT, "a device-side wait exceeded its budget");
   return FB_OK;
+}
+
+int fb_block_commit(const fb_kv* kv, const int32_t* seq_len_host, const void* k_in,
+                    const void* v_in, int32_t B, void* page_min, void* page_max,
+                    cudaStream_t stream) {
+  int rc = validate_kv(kv);
+  if (rc) return rc;
+  if (!kv->seq_len) return fail(FB_ERR_ARG, "kv->seq_len is NULL: the lengths are updated in place");
+  if (!seq_len_host) return fail(FB_ERR_ARG, "seq_len_host is NULL");
+  if (B < 0) return fail(FB_ERR_ARG, "B must be >= 0");
+  if (B > 0 && (!k_in || !v_in)) return fail(FB_ERR_ARG, "k_in / v_in is NULL");
+  if ((page_min == nullptr) != (page_max == nullptr))
+    return fail(FB_ERR_ARG, "page_min and page_max must both be given or both be NULL");
+  if (!aligned16(k_in) || !aligned16(v_in)) return fail(FB_ERR_ALIGN, "k_in / v_in not 16-byte aligned");
+  const KvView v = kv_view(kv);
+  CommitArgs a{};
+  int max_touched = 0;
+  for (int b = 0; b < kv->batch; ++b) {
+    const int n = seq_len_host[b];
+    if (n < 0 || (long long)n + B > kv->max_seq_len)
+      return fail(FB_ERR_ARG, "sequence %d: %d + %d tokens exceed max_seq_len %d", b, n, B,
+                  kv->max_seq_len);
+    a.n_old[b] = n;
+    if (B > 0) {
+      const int touched = (n + B - 1) / v.page_size - n / v.page_size + 1;
+      max_touched = touched > max_touched ? touched : max_touched;
+    }
+  }
+  if (B == 0) return FB_OK;
+  a.k_in = k_in;
+  a.v_in = v_in;
+  a.k = const_cast<void*>(kv->k);
+  a.v = const_cast<void*>(kv->v);
+  a.page_table = kv->page_table;
+  a.seq_len = const_cast<int32_t*>(kv->seq_len);
+  a.pmin = page_min;
+  a.pmax = page_max;
+  a.n_slots = kv->n_slots;
+  a.batch = kv->batch;
+  a.B = B;
+  a.Hkv = kv->n_heads_kv;
+  a.page_size = v.page_size;
+  a.max_pages = v.max_pages;
+  a.max_seq_len = kv->max_seq_len;
+  const dim3 grid(max_touched, kv->n_heads_kv, kv->batch);
+  if (grid.y > 65535) return fail(FB_ERR_SHAPE, "too many kv heads");
+  if (kv->dtype == FB_BF16) {
+    if (v.D == 128)
+      block_commit_kernel<__nv_bfloat16, 128><<<grid, 128, 0, stream>>>(a);
+    else
+      block_commit_kernel<__nv_bfloat16, 64><<<grid, 64, 0, stream>>>(a);
+  } else {
+    if (v.D == 128)
+      block_commit_kernel<float, 128><<<grid, 128, 0, stream>>>(a);
+    else
+      block_commit_kernel<float, 64><<<grid, 64, 0, stream>>>(a);
+  }
+  return check_launch("block commit kernel");
 }
 
 size_t fb_workspace_size(const fb_kv* kv, int32_t block, int32_t n_heads_q, int32_t n_active,

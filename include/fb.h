@@ -267,8 +267,37 @@ int fb_step(const fb_policy* policy, fb_cache* cache, const void* q, const void*
             float* l_full, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Block commit: the finished block joins the block-external cache. Block
+ * diffusion is causal between blocks ([FB] abstract, section 2), so once a
+ * block's tokens are final they belong to J_out of every later block; the
+ * LoSA page summaries ([LoSA] step 3) then have to cover them too.
+ * For every sequence b with n_b = seq_len_host[b] tokens before the call:
+ *  - block row j of k_in / v_in [batch, B, n_heads_kv, head_dim] (kv->dtype)
+ *    is written to the cache slot of position n_b + j (page table, or row
+ *    b * max_seq_len + t of a contiguous cache);
+ *  - kv->seq_len[b] (device, required) becomes n_b + B;
+ *  - if page_min / page_max (fb_page_summary layout) are given, the summary
+ *    of every page receiving tokens is brought up to date: a page that held
+ *    tokens before folds the new keys into its min / max, a fresh page is
+ *    summarised from the new keys alone (bit-exact with a full recompute).
+ * seq_len_host: HOST [batch] int32 lengths before the call; it must equal the
+ *   device lengths (the caller tracks them to map pages). Every n_b + B must
+ *   stay within kv->max_seq_len (FB_ERR_ARG otherwise); kv->max_seq_len in turn
+ *   bounds the lengths that the attention calls plan for.
+ * Paged caches: the caller maps the pages of positions up to n_b + B - 1 in
+ *   the page table before the call. An entry outside the pool is not written
+ *   through; the kernel flags it and fb_device_status() then returns
+ *   FB_ERR_ARG.
+ * B = 0 is a no-op.
+ */
+int fb_block_commit(const fb_kv* kv, const int32_t* seq_len_host, const void* k_in,
+                    const void* v_in, int32_t B, void* page_min, void* page_max,
+                    cudaStream_t stream);
+
+/*
  * Reads and clears the device-side error word that bounded waits set when they
- * give up (SYNCHRONISES the current device). Returns FB_OK or FB_ERR_TIMEOUT.
+ * give up (SYNCHRONISES the current device). Returns FB_OK, FB_ERR_TIMEOUT, or
+ * FB_ERR_ARG when fb_block_commit met a page-table entry outside the pool.
  */
 int fb_device_status(void);
 

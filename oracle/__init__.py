@@ -11,9 +11,10 @@ Modules:
   losa         locality score, active set, page summaries and scores, top-k
                pages, union, sparse partial
   controllers  threshold (tau), per-head (gamma) and LoSA step procedures
+  cache        block commit: a finished block's K/V appended to the cache
 """
 
-from . import attention, controllers, losa  # noqa: F401
+from . import attention, cache, controllers, losa  # noqa: F401
 from .attention import (  # noqa: F401
     block_partial,
     dense_attention,

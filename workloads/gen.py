@@ -142,6 +142,45 @@ class Prefix:
         return pages * self.page_size + t % self.page_size
 
 
+def grow_capacity(prefix: Prefix, extra_tokens: int, seed: int = 0) -> Prefix:
+    """A copy of `prefix` with room for `extra_tokens` more tokens per sequence
+    (layout only: no value is computed). Paged pools get the extra logical
+    pages of every sequence mapped to new physical pages appended to the pool
+    in a seeded permutation; contiguous pools get a longer per-sequence stride.
+    New slots hold NaN (f32) / the bf16 NaN pattern, so a write that misses its
+    slot is caught by any comparison."""
+    P = int(prefix.page_size)
+    batch = len(prefix.seq_len)
+    new_max = int(prefix.max_seq_len) + int(extra_tokens)
+    hd = prefix.k.shape[1:]
+    fill = np.float32(np.nan) if prefix.k.dtype == np.float32 else np.uint16(BF16_NAN_BITS)
+    if prefix.page_table is None:
+        k = np.full((batch * new_max,) + hd, fill, dtype=prefix.k.dtype)
+        v = np.full((batch * new_max,) + hd, fill, dtype=prefix.v.dtype)
+        for b in range(batch):
+            n = int(prefix.seq_len[b])
+            src = b * int(prefix.max_seq_len)
+            k[b * new_max: b * new_max + n] = prefix.k[src: src + n]
+            v[b * new_max: b * new_max + n] = prefix.v[src: src + n]
+        return Prefix(k, v, prefix.seq_len.copy(), None, P, new_max)
+    old_pages = prefix.k.shape[0] // P
+    have = [-(-int(n) // P) for n in prefix.seq_len]
+    need = [-(-(int(n) + int(extra_tokens)) // P) for n in prefix.seq_len]
+    total_new = int(sum(nd - hv for nd, hv in zip(need, have)))
+    perm = old_pages + np.random.default_rng([seed, 11]).permutation(total_new).astype(np.int32)
+    max_pages = -(-new_max // P)
+    table = np.full((batch, max_pages), -1, dtype=np.int32)
+    table[:, : prefix.page_table.shape[1]] = prefix.page_table
+    off = 0
+    for b in range(batch):
+        cnt = need[b] - have[b]
+        table[b, have[b]: need[b]] = perm[off: off + cnt]
+        off += cnt
+    pad = np.full((total_new * P,) + hd, fill, dtype=prefix.k.dtype)
+    return Prefix(np.concatenate([prefix.k, pad]), np.concatenate([prefix.v, pad]),
+                  prefix.seq_len.copy(), table, P, new_max)
+
+
 @dataclass
 class StepInputs:
     step: int
