@@ -29,6 +29,7 @@ FB_BF16 = 1
 FB_THRESHOLD = 0
 FB_PER_HEAD = 1
 FB_LOSA = 2
+FB_SPARSE_RESIDUAL = 3
 
 # Every entry point include/fb.h declares.
 EXPORTS = ("fb_workspace_size", "fb_prefix_attn", "fb_block_attn", "fb_merge", "fb_page_summary",
@@ -64,7 +65,9 @@ class fb_cache(ctypes.Structure):
                 ("active_rows", ctypes.c_void_p), ("row_scores", ctypes.c_void_p),
                 ("union_bitmap", ctypes.c_void_p), ("union_list", ctypes.c_void_p),
                 ("union_count", ctypes.c_void_p), ("step", ctypes.c_int32),
-                ("recomputed", ctypes.c_int32)]
+                ("recomputed", ctypes.c_int32), ("a_res", ctypes.c_void_p),
+                ("l_res", ctypes.c_void_p), ("comp_list", ctypes.c_void_p),
+                ("comp_count", ctypes.c_void_p)]
 
 
 _lib = None

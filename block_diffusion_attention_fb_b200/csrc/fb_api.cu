@@ -678,6 +678,55 @@ int block_attn_impl(const void* q, const void* k_in, const void* v_in, int batch
   return launch_partial(c, stream);
 }
 
+// Selection of the sparse-residual mode: per (sequence, kv head) the top-k
+// pages by head score (max over block rows and the kv head's q heads of the
+// QUEST-style bound) into bitmap / list / count, the other pages of the
+// sequence into comp_list / comp_count.
+int sr_select(const void* q, int B, int Hq, const void* page_min, const void* page_max,
+              const fb_kv* kv, int topk, uint32_t* bitmap, int32_t* list, int32_t* count,
+              int32_t* comp_list, int32_t* comp_count, float* head_scores,
+              cudaStream_t stream) {
+  const KvView v = kv_view(kv);
+  const int D = v.D, G = Hq / v.Hkv, RQ = B * G;
+  const int words = ceil_div(v.max_pages, 32);
+  if (RQ > 64) return fail(FB_ERR_SHAPE, "sparse residual supports <= 64 rows per kv head");
+  if (v.max_pages > 32768) return fail(FB_ERR_SHAPE, "sparse residual supports <= 32768 pages");
+  if (!aligned16(page_min) || !aligned16(page_max))
+    return fail(FB_ERR_ALIGN, "page summaries not 16-byte aligned");
+  const dim3 g2(ceil_div(v.max_pages, kPsPages), v.Hkv, kv->batch);
+  const int es = (int)elem_size(kv->dtype);
+  const int psm = RQ * D * 4 + 2 * kPsPages * (D + 4 / es) * es;
+  int rc;
+#define FB_HPS(TT, DD)                                                                       \
+  do {                                                                                       \
+    auto kfn = head_page_score_kernel<TT, DD>;                                               \
+    if ((rc = set_smem_once((const void*)kfn, psm))) return rc;                            \
+    kfn<<<g2, 256, psm, stream>>>(static_cast<const TT*>(q), B, Hq, G,                       \
+                                  static_cast<const TT*>(page_min),                          \
+                                  static_cast<const TT*>(page_max), v, head_scores, bitmap,  \
+                                  words);                                                    \
+  } while (0)
+  if (kv->dtype == FB_BF16) {
+    if (D == 128) FB_HPS(__nv_bfloat16, 128); else FB_HPS(__nv_bfloat16, 64);
+  } else {
+    if (D == 128) FB_HPS(float, 128); else FB_HPS(float, 64);
+  }
+#undef FB_HPS
+  if ((rc = check_launch("head page score kernel"))) return rc;
+  const int ksm = v.max_pages * 4;
+  if ((rc = set_smem_once((const void*)topk_pages_kernel, ksm))) return rc;
+  // one "row" per kv head: scores [batch, 1, Hkv, pages], G = 1
+  topk_pages_kernel<<<dim3(v.Hkv, kv->batch), kTopkThreads, ksm, stream>>>(
+      head_scores, v, v.Hkv, 1, 1, topk, bitmap, words);
+  if ((rc = check_launch("top-k pages kernel"))) return rc;
+  union_compact_kernel<<<dim3(v.Hkv, kv->batch), 256, 0, stream>>>(bitmap, words, v.Hkv,
+                                                                   v.max_pages, list, count);
+  if ((rc = check_launch("selection compaction kernel"))) return rc;
+  complement_compact_kernel<<<dim3(v.Hkv, kv->batch), 256, 0, stream>>>(
+      bitmap, words, v, v.max_pages, comp_list, comp_count);
+  return check_launch("complement compaction kernel");
+}
+
 }  // namespace
 
 extern "C" {
@@ -992,8 +1041,9 @@ int fb_step(const fb_policy* policy, fb_cache* cache, const void* q, const void*
   const int batch = prefix->batch, Hq = n_heads_q, Hkv = prefix->n_heads_kv, D = prefix->head_dim;
   const int s = cache->step;
   const int num_sms = sm_count();
-  const int na = policy->mode == FB_LOSA ? policy->n_active : 0;
-  const int tk = policy->mode == FB_LOSA ? policy->topk_pages : 0;
+  const bool sr = policy->mode == FB_SPARSE_RESIDUAL;
+  const int na = policy->mode == FB_LOSA ? policy->n_active : (sr ? B : 0);
+  const int tk = policy->mode == FB_LOSA ? policy->topk_pages : (sr ? logical_pages(prefix) : 0);
   const WsLayout w = ws_layout(prefix, B, Hq, na, tk, num_sms);
   if (!workspace || workspace_bytes < w.total)
     return fail(FB_ERR_WORKSPACE, "workspace too small: need %zu, have %zu", w.total,
@@ -1053,6 +1103,42 @@ int fb_step(const fb_policy* policy, fb_cache* cache, const void* q, const void*
       rc = check_launch("cosine stage 2");
       if (rc) return rc;
     }
+  } else if (sr) {
+    if (!page_min || !page_max || !cache->union_bitmap || !cache->union_list ||
+        !cache->union_count || !cache->comp_list || !cache->comp_count || !cache->a_res ||
+        !cache->l_res)
+      return fail(FB_ERR_ARG, "SPARSE_RESIDUAL needs the page summaries, the selection and "
+                              "complement buffers and a_res / l_res");
+    if (policy->topk_pages < 0) return fail(FB_ERR_ARG, "topk_pages < 0");
+    bool refresh = s == 0 || policy->tau <= 0;
+    for (int b = 0; b < batch && !refresh; ++b)
+      refresh = m_updated && m_updated[b] >= policy->tau;
+    cache->recomputed = refresh ? batch : 0;
+    const int np = logical_pages(prefix);
+    if (refresh) {
+      rc = sr_select(q, B, Hq, page_min, page_max, prefix, policy->topk_pages,
+                     cache->union_bitmap, cache->union_list, cache->union_count, cache->comp_list,
+                     cache->comp_count, reinterpret_cast<float*>(ws + w.scores), stream);
+      if (rc) return rc;
+      PartialCall cr = c;  // residual: every row over the unselected pages
+      cr.page_list = cache->comp_list;
+      cr.page_count = cache->comp_count;
+      cr.page_list_stride = np;
+      cr.max_list_entries = np;
+      cr.a_out = cache->a_res;
+      cr.l_out = cache->l_res;
+      rc = launch_partial(cr, stream);
+      if (rc) return rc;
+    }
+    PartialCall cs = c;  // fresh sparse partial over the selected pages, merged with the residual
+    cs.page_list = cache->union_list;
+    cs.page_count = cache->union_count;
+    cs.page_list_stride = np;
+    cs.max_list_entries = policy->topk_pages < np ? policy->topk_pages : np;
+    cs.mrg_a = cache->a_res;
+    cs.mrg_l = cache->l_res;
+    rc = launch_partial(cs, stream);
+    if (rc) return rc;
   } else if (policy->mode == FB_LOSA) {
     if (!cache->q_prev || !cache->active_rows || !cache->union_bitmap || !cache->union_list ||
         !cache->union_count)

@@ -428,4 +428,134 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// ---------------------------------------------------------------------------
+// FlashBlock + sparse attention (FlashBlock technical summary §2, compatibility
+// with sparse attention): the sparse selector scores pages per kv head by the
+// same QUEST-style bound, taking the maximum over every block row and every q
+// head of the kv head: head score of page p = max_{i,g} tree_sum_c
+// max(q_c kmin_c, q_c kmax_c). The per-(row, head) bound is formed exactly as in
+// page_score_kernel (single-rounded products, stride-halving tree); the maximum
+// is order-free, taken on order-preserving keys with shared-memory atomics.
+// scores: [batch, Hkv, max_pages]. Block (0, hk, b) clears the (b, hk) bitmap.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float order_key_inv(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+    head_page_score_kernel(const T* __restrict__ q, int B, int Hq, int G,
+                           const T* __restrict__ pmin, const T* __restrict__ pmax,
+                           const KvView kv, float* __restrict__ scores,
+                           uint32_t* __restrict__ bitmap, int words) {
+  constexpr int PS = D + 4 / (int)sizeof(T);
+  constexpr int VE = 16 / (int)sizeof(T);
+  extern __shared__ float sm[];
+  __shared__ uint32_t best[kPsPages];
+  const int RQ = B * G;
+  float* qs = sm;                              // [RQ][D], row r = i * G + g
+  T* smn = reinterpret_cast<T*>(qs + RQ * D);  // [kPsPages][PS]
+  T* smx = smn + kPsPages * PS;
+  const int hk = blockIdx.y, b = blockIdx.z;
+  const int p0 = blockIdx.x * kPsPages;
+  if (blockIdx.x == 0)
+    for (int w = threadIdx.x; w < words; w += blockDim.x)
+      bitmap[((long long)b * kv.Hkv + hk) * words + w] = 0u;
+  const int n_pages = (kv_tokens(kv, b) + kv.page_size - 1) / kv.page_size;
+  if (p0 >= n_pages) return;
+  for (int pg = threadIdx.x; pg < kPsPages; pg += blockDim.x) best[pg] = 0u;  // below every key
+  for (int idx = threadIdx.x; idx < RQ * D; idx += blockDim.x) {
+    const int rq = idx / D, c = idx - (idx / D) * D;
+    const int i = rq / G, g = rq - (rq / G) * G;
+    qs[idx] = ld_f32<T>(q + (((long long)b * B + i) * Hq + hk * G + g) * D + c);
+  }
+  for (int idx = threadIdx.x; idx < kPsPages * (D / VE); idx += blockDim.x) {
+    const int pg = idx / (D / VE), cv = idx - (idx / (D / VE)) * (D / VE);
+    const int p = p0 + pg;
+    uint4 mn = make_uint4(0u, 0u, 0u, 0u), mx = make_uint4(0u, 0u, 0u, 0u);
+    if (p < n_pages) {
+      const long long so = (((long long)b * kv.max_pages + p) * kv.Hkv + hk) * D + cv * VE;
+      mn = *reinterpret_cast<const uint4*>(pmin + so);
+      mx = *reinterpret_cast<const uint4*>(pmax + so);
+    }
+    uint32_t* dn = reinterpret_cast<uint32_t*>(smn + pg * PS + cv * VE);
+    uint32_t* dx = reinterpret_cast<uint32_t*>(smx + pg * PS + cv * VE);
+    dn[0] = mn.x; dn[1] = mn.y; dn[2] = mn.z; dn[3] = mn.w;
+    dx[0] = mx.x; dx[1] = mx.y; dx[2] = mx.z; dx[3] = mx.w;
+  }
+  __syncthreads();
+  for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
+    const int pg = task % kPsPages, rq = task / kPsPages;
+    const int p = p0 + pg;
+    if (p >= n_pages) continue;
+    const float* qr = qs + rq * D;
+    const T* mnr = smn + pg * PS;
+    const T* mxr = smx + pg * PS;
+    float y[D / 2];
+#pragma unroll
+    for (int c = 0; c < D / 2; ++c) {
+      const float q0 = qr[c], q1 = qr[c + D / 2];
+      const float x0 = fmaxf(__fmul_rn(q0, ld_f32<T>(mnr + c)), __fmul_rn(q0, ld_f32<T>(mxr + c)));
+      const float x1 = fmaxf(__fmul_rn(q1, ld_f32<T>(mnr + c + D / 2)),
+                             __fmul_rn(q1, ld_f32<T>(mxr + c + D / 2)));
+      y[c] = __fadd_rn(x0, x1);
+    }
+#pragma unroll
+    for (int st = D / 4; st >= 1; st >>= 1)
+#pragma unroll
+      for (int c = 0; c < st; ++c) y[c] = __fadd_rn(y[c], y[c + st]);
+    atomicMax(&best[pg], order_key(y[0]));
+  }
+  __syncthreads();
+  for (int pg = threadIdx.x; pg < kPsPages; pg += blockDim.x) {
+    const int p = p0 + pg;
+    if (p < n_pages)
+      scores[((long long)b * kv.Hkv + hk) * kv.max_pages + p] = order_key_inv(best[pg]);
+  }
+}
+
+// Complement of a selection bitmap within a sequence's pages: ascending list of
+// the pages p < n_pages(b) whose bit is clear, and their count, per (b, hk).
+__global__ void __launch_bounds__(256)
+    complement_compact_kernel(const uint32_t* __restrict__ bitmap, int words, const KvView kv,
+                              int stride, int32_t* __restrict__ list,
+                              int32_t* __restrict__ count) {
+  __shared__ int wsum[256];
+  const int hk = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int n_pages = (kv_tokens(kv, b) + kv.page_size - 1) / kv.page_size;
+  const uint32_t* bm = bitmap + ((long long)b * kv.Hkv + hk) * words;
+  int32_t* out = list + ((long long)b * kv.Hkv + hk) * stride;
+  const int per = (words + 255) / 256;
+  const int w0 = tid * per, w1 = min(words, w0 + per);
+  auto clear_bits = [&](int w) -> uint32_t {
+    const int lo = w * 32;
+    if (lo >= n_pages) return 0u;
+    const uint32_t valid = (n_pages - lo >= 32) ? 0xFFFFFFFFu : ((1u << (n_pages - lo)) - 1u);
+    return ~bm[w] & valid;
+  };
+  int c = 0;
+  for (int w = w0; w < w1; ++w) c += __popc(clear_bits(w));
+  wsum[tid] = c;
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int t = 0; t < 256; ++t) {
+      const int x = wsum[t];
+      wsum[t] = run;
+      run += x;
+    }
+    count[b * kv.Hkv + hk] = run;
+  }
+  __syncthreads();
+  int pos = wsum[tid];
+  for (int w = w0; w < w1; ++w) {
+    uint32_t bits = clear_bits(w);
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      out[pos++] = w * 32 + bit;
+    }
+  }
+}
+
 }  // namespace fb

@@ -10,16 +10,18 @@ from typing import Optional, Sequence
 
 import torch
 
-from . import (FB_LOSA, FB_PER_HEAD, FB_THRESHOLD, KV, fb_cache, fb_page_summary, fb_policy,
-               fb_step, fb_workspace_size)
+from . import (FB_LOSA, FB_PER_HEAD, FB_SPARSE_RESIDUAL, FB_THRESHOLD, KV, fb_cache,
+               fb_page_summary, fb_policy, fb_step, fb_workspace_size)
 
-_MODES = {"threshold": FB_THRESHOLD, "per_head": FB_PER_HEAD, "losa": FB_LOSA}
+_MODES = {"threshold": FB_THRESHOLD, "per_head": FB_PER_HEAD, "losa": FB_LOSA,
+          "sparse_residual": FB_SPARSE_RESIDUAL}
 
 
 class BlockAttention:
     """Attention of one block across its denoise steps (FlashBlock / LoSA).
 
-    mode: "threshold" (tau), "per_head" (gamma) or "losa" (n_active, topk_pages).
+    mode: "threshold" (tau), "per_head" (gamma), "losa" (n_active, topk_pages) or
+    "sparse_residual" (tau, topk_pages: pages selected per kv head).
     """
 
     def __init__(self, kv: KV, block: int, n_heads_q: int, mode: str, tau: int = 0,
@@ -39,13 +41,9 @@ class BlockAttention:
             self.t["head_cos"] = torch.full((batch, n_heads_q), float("nan"), dtype=torch.float64,
                                             device=dev)
         self.page_min = self.page_max = None
-        if mode == "losa":
-            na = min(n_active, block)
-            hkv = kv.c.n_heads_kv
-            npg = kv.n_pages
-            self.t["q_prev"] = torch.zeros(batch, block, n_heads_q, d, dtype=kv.k.dtype, device=dev)
-            self.t["active_rows"] = torch.zeros(batch, max(na, 1), dtype=torch.int32, device=dev)
-            self.t["row_scores"] = torch.zeros(batch, block, **f32)
+        hkv = kv.c.n_heads_kv
+        npg = kv.n_pages
+        if mode in ("losa", "sparse_residual"):
             self.t["union_bitmap"] = torch.zeros(batch, hkv, -(-npg // 32), dtype=torch.int32,
                                                  device=dev)
             self.t["union_list"] = torch.zeros(batch, hkv, npg, dtype=torch.int32, device=dev)
@@ -53,14 +51,29 @@ class BlockAttention:
             self.page_min = torch.empty(batch, npg, hkv, d, dtype=kv.k.dtype, device=dev)
             self.page_max = torch.empty_like(self.page_min)
             fb_page_summary(kv, self.page_min, self.page_max)
-        ws = fb_workspace_size(kv, block, n_heads_q, n_active if mode == "losa" else 0,
-                               topk_pages if mode == "losa" else 0)
+        if mode == "losa":
+            na = min(n_active, block)
+            self.t["q_prev"] = torch.zeros(batch, block, n_heads_q, d, dtype=kv.k.dtype, device=dev)
+            self.t["active_rows"] = torch.zeros(batch, max(na, 1), dtype=torch.int32, device=dev)
+            self.t["row_scores"] = torch.zeros(batch, block, **f32)
+        if mode == "sparse_residual":
+            self.t["a_res"] = torch.zeros_like(self.a_out)
+            self.t["l_res"] = torch.zeros_like(self.l_out)
+            self.t["comp_list"] = torch.zeros(batch, hkv, npg, dtype=torch.int32, device=dev)
+            self.t["comp_count"] = torch.zeros(batch, hkv, dtype=torch.int32, device=dev)
+        if mode == "losa":
+            ws = fb_workspace_size(kv, block, n_heads_q, n_active, topk_pages)
+        elif mode == "sparse_residual":  # every row scored, every page a possible list entry
+            ws = fb_workspace_size(kv, block, n_heads_q, block, npg)
+        else:
+            ws = fb_workspace_size(kv, block, n_heads_q)
         self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
         p = {k: v.data_ptr() for k, v in self.t.items()}
         self.cache = fb_cache(p.get("a_out"), p.get("l_out"), p.get("a_out_prev"), p.get("head_mask"),
                               p.get("head_cos"), p.get("q_prev"), p.get("active_rows"),
                               p.get("row_scores"), p.get("union_bitmap"), p.get("union_list"),
-                              p.get("union_count"), 0, 0)
+                              p.get("union_count"), 0, 0, p.get("a_res"), p.get("l_res"),
+                              p.get("comp_list"), p.get("comp_count"))
 
     def reset(self) -> None:
         """Start a new block (the next step computes the prefix partial)."""

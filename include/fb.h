@@ -210,17 +210,20 @@ int losa_gather(const void* q, int32_t B, int32_t n_heads_q, const int32_t* acti
 /* ---------------------------------------------------------------------------
  * Step controller ([FB] "Adaptive reuse strategies"; [LoSA] steps 1-4).
  * ------------------------------------------------------------------------- */
-typedef enum { FB_THRESHOLD = 0, FB_PER_HEAD = 1, FB_LOSA = 2 } fb_mode;
+typedef enum { FB_THRESHOLD = 0, FB_PER_HEAD = 1, FB_LOSA = 2, FB_SPARSE_RESIDUAL = 3 } fb_mode;
 
 typedef struct fb_policy {
   fb_mode mode;
   int32_t tau;        /* THRESHOLD: recompute sequence b when m_updated[b] >= tau
-                         (tau <= 0: recompute every step, i.e. dense) */
+                         (tau <= 0: recompute every step, i.e. dense).
+                         SPARSE_RESIDUAL: refresh the selection and the residual
+                         when any sequence has m_updated[b] >= tau */
   double gamma;       /* PER_HEAD: a head that computed at steps s-1 and s stops
                          computing for the rest of the block once
                          cos(A_out^s, A_out^{s-1}) >= gamma (gamma > 1: dense) */
   int32_t n_active;   /* LOSA: active rows per step */
-  int32_t topk_pages; /* LOSA: pages kept per active row and q head */
+  int32_t topk_pages; /* LOSA: pages kept per active row and q head;
+                         SPARSE_RESIDUAL: pages selected per kv head */
   float scale;        /* softmax scale applied to <q, k> */
 } fb_policy;
 
@@ -242,7 +245,12 @@ typedef struct fb_cache {
   int32_t* union_list;    /* LOSA: [batch, Hkv, max_pages] */
   int32_t* union_count;   /* LOSA: [batch, Hkv] */
   int32_t step;           /* host: index of the next step (0 = block start); fb_step advances it */
-  int32_t recomputed;     /* host: sequences (THRESHOLD) whose prefix partial the last step recomputed */
+  int32_t recomputed;     /* host: sequences (THRESHOLD) whose prefix partial the last step
+                             recomputed; SPARSE_RESIDUAL: batch on a refresh step, else 0 */
+  float* a_res;           /* SPARSE_RESIDUAL: cached partial over the unselected pages */
+  float* l_res;           /* SPARSE_RESIDUAL: its log normaliser */
+  int32_t* comp_list;     /* SPARSE_RESIDUAL: [batch, Hkv, max_pages] unselected pages */
+  int32_t* comp_count;    /* SPARSE_RESIDUAL: [batch, Hkv] */
 } fb_cache;
 
 /*
@@ -254,12 +262,26 @@ typedef struct fb_cache {
  *              device (no host round trip);
  *   LOSA:      step 0 computes the dense prefix partial; later steps run
  *              losa_select + losa_gather; q is copied into q_prev.
+ *   SPARSE_RESIDUAL ([FB] section 2, compatibility with sparse attention: the
+ *              keys a sparse method leaves out are treated as block-external and
+ *              their contribution is cached): on a refresh step (step 0, tau <= 0,
+ *              or any m_updated[b] >= tau) every kv head selects topk_pages pages
+ *              by the head score max over block rows i and its q heads h of
+ *              tree_sum_c max(q_c kmin_c, q_c kmax_c) (float32, LoSA's order;
+ *              ties: lower page) into union_bitmap / union_list / union_count,
+ *              the other pages into comp_list / comp_count, and the partial
+ *              over the unselected pages is stored in a_res / l_res. Every step
+ *              computes the partial over the selected pages with the current q
+ *              and merges it with the cached residual into a_out / l_out. At
+ *              most 64 stacked rows (B * Hq / Hkv) per kv head (FB_ERR_SHAPE).
+ *              Workspace: fb_workspace_size with n_active = B and topk_pages =
+ *              the logical page count.
  * Then the block-internal partial is computed and merged:
  *   a_full [batch, B, Hq, d] float32, l_full [batch, B, Hq] float32 (may be NULL).
  *  q, k_in, v_in: this step's block tensors (dtype of prefix->dtype).
- *  page_min / page_max: fb_page_summary output (LOSA only).
+ *  page_min / page_max: fb_page_summary output (LOSA, SPARSE_RESIDUAL).
  *  m_updated: HOST [batch] int32 rows updated since the previous step
- *             (THRESHOLD only; may be NULL at step 0).
+ *             (THRESHOLD, SPARSE_RESIDUAL; may be NULL at step 0).
  */
 int fb_step(const fb_policy* policy, fb_cache* cache, const void* q, const void* k_in,
             const void* v_in, int32_t B, int32_t n_heads_q, const fb_kv* prefix,

@@ -12,9 +12,10 @@ Modules:
                pages, union, sparse partial
   controllers  threshold (tau), per-head (gamma) and LoSA step procedures
   cache        block commit: a finished block's K/V appended to the cache
+  residual     FlashBlock + sparse attention: cached residual of unselected pages
 """
 
-from . import attention, cache, controllers, losa  # noqa: F401
+from . import attention, cache, controllers, losa, residual  # noqa: F401
 from .attention import (  # noqa: F401
     block_partial,
     dense_attention,

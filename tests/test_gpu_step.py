@@ -12,6 +12,7 @@ import torch
 from block_diffusion_attention_fb_b200.runtime import BlockAttention
 from oracle.controllers import (LosaController, PerHeadController, ThresholdController,
                                 head_cosine)
+from oracle.residual import SparseResidualController
 from tests.gpu_util import assert_close_A, assert_close_L, cpu, dev, make_kv, sync
 from workloads import make_workload
 
@@ -157,3 +158,57 @@ def test_losa_steps_match_oracle(ov, n_active, topk):
                 np.testing.assert_array_equal(cpu(blk.t["union_list"])[b, hk, :cnt], pages)
         assert_close_A(cpu(A), ref["A_full"], sp.dtype, f"step {st.step}")
         assert_close_L(cpu(L), ref["L_full"], f"step {st.step}")
+
+
+@pytest.mark.parametrize("name,ov,tau,topk", [
+    ("dllm", dict(prefix_min=1500, prefix_max=1500, n_heads_q=4, n_heads_kv=4, block=32,
+                  steps=8), 2, 12),
+    # paged, ragged lengths, GQA (16 rows x 4 q heads = 64 stacked rows per kv head)
+    ("gqa", dict(prefix_min=100, prefix_max=900, batch=3, block=16, n_heads_q=8, n_heads_kv=2,
+                 steps=6), 3, 5),
+    ("tiny", dict(steps=6), 2, 9),  # float32, head_dim 64
+    # every page selected: the complement is empty and every step is dense
+    ("dllm", dict(prefix_min=700, prefix_max=700, n_heads_q=2, n_heads_kv=2, block=8, steps=4),
+     2, 1000),
+    # no page selected: plain threshold reuse of the cached residual
+    ("dllm", dict(prefix_min=700, prefix_max=700, n_heads_q=2, n_heads_kv=2, block=8, steps=5),
+     2, 0),
+])
+def test_sparse_residual_steps_match_oracle(name, ov, tau, topk):
+    """FlashBlock with sparse attention (technical summary §2): fresh partial over
+    the selected pages merged with the cached residual of the unselected ones."""
+    wl = make_workload(name, **ov)
+    sp = wl.spec
+    kv = make_kv(wl.prefix, sp.dtype)
+    blk = BlockAttention(kv, sp.block, sp.n_heads_q, "sparse_residual", tau=tau, topk_pages=topk)
+    ctl = SparseResidualController(wl.prefix, sp.dtype, tau, topk)
+    A, L = _out(sp)
+    for st in wl.steps():
+        blk.step(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L,
+                 m_updated=st.m_updated)
+        ref = ctl.step(st.step, st.q, st.k_in, st.v_in, st.m_updated)
+        sync()
+        assert blk.recomputed == (sp.batch if ref["refresh"] else 0), f"step {st.step}"
+        if ref["refresh"]:  # the selection is bit-exact
+            ul, uc = cpu(blk.t["union_list"]), cpu(blk.t["union_count"])
+            cl, cc = cpu(blk.t["comp_list"]), cpu(blk.t["comp_count"])
+            for (b, hk), (S, C) in ref["selection"].items():
+                assert uc[b, hk] == len(S) and np.array_equal(ul[b, hk, :len(S)], S), (b, hk)
+                assert cc[b, hk] == len(C) and np.array_equal(cl[b, hk, :len(C)], C), (b, hk)
+        assert_close_A(cpu(A), ref["A_full"], sp.dtype, f"step {st.step}")
+        assert_close_L(cpu(L), ref["L_full"], f"step {st.step}")
+
+
+def test_sparse_residual_rejects_more_than_64_rows_per_kv_head():
+    import block_diffusion_attention_fb_b200 as fb
+    wl = make_workload("gqa", prefix_min=100, prefix_max=300, batch=2, block=32, n_heads_q=8,
+                       n_heads_kv=2, steps=1)
+    sp = wl.spec
+    kv = make_kv(wl.prefix, sp.dtype)
+    blk = BlockAttention(kv, sp.block, sp.n_heads_q, "sparse_residual", tau=2, topk_pages=4)
+    A, L = _out(sp)
+    st = next(wl.steps(1))
+    with pytest.raises(fb.FbError) as e:
+        blk.step(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L,
+                 m_updated=st.m_updated)
+    assert e.value.code == fb.FB_ERR_SHAPE
