@@ -14,6 +14,9 @@ Modes, each timed over the same K blocks:
   reuse  FlashBlock threshold reuse (tau=4) through fb_step: the headline value
   dense  prefix partial every step (fb_prefix_attn + fb_block_attn + fb_merge)
   losa   LoSA (4 active rows, top-256 of 2048 pages) through fb_step
+  sparse_residual  FlashBlock + sparse attention (20% of pages per kv head,
+         residual of the rest cached, tau=4) through fb_step
+  block_commit     fb_block_commit of one block's rows (into a separate cache)
 
 value = microseconds per denoise step of the whole job (max over ranks of the
 device time / denoise steps of all ranks). With N GPUs every rank runs its own
@@ -43,6 +46,7 @@ WORKLOAD = ("dllm: bf16, batch 1, 32 heads MHA, head_dim 128, prefix 32768 token
             "32 denoise steps per block, Poisson(2) updates, tau 4; LoSA 4 active rows, top-256 pages")
 FLUSH_BYTES = 256 << 20
 LOSA_ACTIVE, LOSA_TOPK = 4, 256
+SR_DENSITY_PCT = 20  # sparse-residual mode: selected pages per kv head, percent
 ORACLE_HEADS = 4  # oracle sample: this many of the 32 heads, scaled to all heads
 BASELINE_HEADS, BASELINE_BLOCKS = 8, 2  # CPU baseline sample of our arm (about 10 s)
 
@@ -54,7 +58,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=3, help="untimed blocks before timing")
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--mode", choices=["all", "reuse", "dense", "losa", "prefix", "block"],
+    p.add_argument("--mode", choices=["all", "reuse", "dense", "losa", "sparse_residual",
+                                      "prefix", "block"],
                    default="all",
                    help="all: the contract line; one mode: time only that mode (for profiling)")
     p.add_argument("--workload", choices=["dllm", "tiny", "gqa", "video", "losa"],
@@ -247,6 +252,27 @@ def run_ours(args, rank, world, local):
     n_act = sp.n_active or LOSA_ACTIVE
     topk = sp.topk_pages or LOSA_TOPK
     losa = BlockAttention(kv, B, Hq, "losa", n_active=n_act, topk_pages=topk)
+    # FlashBlock + sparse residual: 20% page density (the pages pair FlashBlock
+    # with SparseD at 20-40%); supported up to 64 stacked rows per kv head
+    sr_topk = max(1, -(-kv.n_pages * SR_DENSITY_PCT // 100))
+    sr_tau = sp.tau if sp.tau is not None else 4
+    sres = (BlockAttention(kv, B, Hq, "sparse_residual", tau=sr_tau, topk_pages=sr_topk)
+            if B * (Hq // sp.n_heads_kv) <= 64 else None)
+    # block commit: a separate contiguous cache with room for every timed
+    # commit (the commit reads only the block rows, so its content is not needed)
+    commit = None
+    if wl.prefix.page_table is None:
+        n_commits = max(1, args.warmup) + args.steps
+        cap = int(wl.prefix.max_seq_len) + n_commits * S * B
+        ck = torch.empty(batch * cap, sp.n_heads_kv, d, dtype=dk[0].dtype, device="cuda")
+        cv = torch.empty_like(ck)
+        clen = torch.from_numpy(wl.prefix.seq_len.astype("int32")).cuda()
+        ckv = fb.KV(ck, cv, seq_len=clen, page_table=None, page_size=t["page_size"],
+                    max_seq_len=cap)
+        cmin = torch.empty(batch, ckv.n_pages, sp.n_heads_kv, d, dtype=dk[0].dtype, device="cuda")
+        cmax = torch.empty_like(cmin)
+        commit = {"kv": ckv, "min": cmin, "max": cmax,
+                  "len": wl.prefix.seq_len.astype("int32").copy()}
     a_out = torch.zeros(batch, B, Hq, d, device="cuda")
     l_out = torch.zeros(batch, B, Hq, device="cuda")
     a_in = torch.zeros_like(a_out)
@@ -272,6 +298,15 @@ def run_ours(args, rank, world, local):
         if s == 0:
             losa.reset()
         losa.step(dq[s], dk[s], dv[s], A, L)
+
+    def sres_step(s):
+        if s == 0:
+            sres.reset()
+        sres.step(dq[s], dk[s], dv[s], A, L, m_updated=ms[s])
+
+    def commit_call(s):
+        fb.fb_block_commit(commit["kv"], commit["len"], dk[s], dv[s], commit["min"], commit["max"])
+        commit["len"] += B
 
     hA = torch.empty(batch, B, Hq, d, dtype=torch.float32).pin_memory()
     hL = torch.empty(batch, B, Hq, dtype=torch.float32).pin_memory()
@@ -308,6 +343,10 @@ def run_ours(args, rank, world, local):
             prefix_call(s)
             dense_rest(s)
             losa_step(s)
+            if sres is not None:
+                sres_step(s)
+            if commit is not None:
+                commit_call(s)
             e2e_step(s)
     torch.cuda.synchronize()
 
@@ -328,6 +367,7 @@ def run_ours(args, rank, world, local):
     g_prefix = capture(prefix_call)
     g_rest = capture(dense_rest)
     g_losa = capture(losa_step)
+    g_sres = capture(sres_step) if sres is not None else None
     rec = sum(1 for s in range(S) if s == 0 or (sp.gamma is None and ms[s][0] >= reuse.policy.tau))
 
     def timed(graph_lists, n_blocks, timed_flag=True):
@@ -364,7 +404,8 @@ def run_ours(args, rank, world, local):
         timed([gl], 1)
     timed([g_prefix, g_rest], 1)
     if args.mode != "all":
-        lists = {"reuse": [g_reuse], "dense": [g_prefix, g_rest], "losa": [g_losa]}[args.mode]
+        lists = {"reuse": [g_reuse], "dense": [g_prefix, g_rest], "losa": [g_losa],
+                 "sparse_residual": [g_sres]}[args.mode]
         barrier(world)
         tot, _ = timed(lists, K)
         barrier(world)
@@ -383,6 +424,11 @@ def run_ours(args, rank, world, local):
     barrier(world)
     (t_losa,), _ = timed([g_losa], K)
     barrier(world)
+    t_sres = timed([g_sres], K)[0][0] if g_sres is not None else None
+    barrier(world)
+    # block commit: one call per denoise step's block rows, eager, L2 flushed before
+    t_commit = eager(commit_call, K) if commit is not None else None
+    barrier(world)
     t_e2e = eager(e2e_step, K)
     barrier(world)
     # the roofline's kernel time: the prefix call launched eagerly (attention
@@ -398,6 +444,8 @@ def run_ours(args, rank, world, local):
     t_reuse_max = max_over_ranks(t_reuse, world)
     t_dense_max = max_over_ranks(t_dense, world)
     t_losa_max = max_over_ranks(t_losa, world)
+    t_sres_max = max_over_ranks(t_sres, world) if t_sres is not None else None
+    t_commit_max = max_over_ranks(t_commit, world) if t_commit is not None else None
     t_e2e_max = max_over_ranks(t_e2e, world)
     us = lambda ms_total: ms_total * 1000.0 / n_steps_all  # noqa: E731
 
@@ -450,6 +498,12 @@ def run_ours(args, rank, world, local):
                       "prefix_call_us": round(prefix_avg_ms * 1000, 3),
                       "prefix_gbs": round(achieved, 1),
                       "prefix_tflops": round(flops / (prefix_avg_ms * 1e-3) / 1e12, 1)},
+            "sparse_residual": ({"us_per_step": round(us(t_sres_max), 3), "tau": sr_tau,
+                                 "topk_pages": sr_topk, "of_pages": kv.n_pages}
+                                if t_sres_max is not None else None),
+            "block_commit": ({"us_per_call": round(us(t_commit_max), 3),
+                              "bytes_per_call": 2 * batch * B * sp.n_heads_kv * d * dk[0].element_size()}
+                             if t_commit_max is not None else None),
             "losa": {"us_per_step": round(us(t_losa_max), 3), "n_active": n_act,
                      "topk_pages": topk},
         },

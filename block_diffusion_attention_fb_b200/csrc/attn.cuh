@@ -61,7 +61,6 @@ struct AttnArgs {
   float* a_out;     // [batch, B, Hq, D]
   float* l_out;     // [batch, B, Hq] natural log
   float* a_prev;    // optional: old a_out rows are copied here before overwrite
-  int* tickets;        // persistent kernel: [batch * Hkv], zero at launch
   const float* mrg_a;  // optional second partial merged into every final row (FlashBlock merge)
   const float* mrg_l;
 };

@@ -11,9 +11,9 @@
 // the new keys alone. min and max are exact, so the incremental result equals
 // a summary recomputed from scratch bit for bit.
 //
-// One CTA per (touched page of a sequence, kv head, sequence), one thread per
-// channel: it copies the page's new K and V rows (coalesced across channels)
-// and folds the new keys into the summary in registers. The new lengths come
+// One CTA per (touched page of a sequence, kv head, sequence) copies the
+// page's new K and V rows with 16-byte loads, all issued before any store,
+// then folds the new keys into the summary per channel. The new lengths come
 // from the host (the caller tracks them to map pages), so nothing here reads
 // the device lengths that it updates.
 #pragma once
@@ -63,41 +63,75 @@ __device__ __forceinline__ __nv_bfloat16 commit_from_f32<__nv_bfloat16>(float x)
   return __float2bfloat16_rn(x);  // exact: x is a bf16 value
 }
 
+// One CTA of 256 threads per (touched page, kv head, sequence). Thread
+// (token slot u, 16-byte chunk v) moves one chunk of K and one of V; every
+// load of the page is issued before any store (one memory round trip). The
+// summary is then folded per channel from the K rows staged in shared memory.
+constexpr int kCommitThreads = 256;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(D) block_commit_kernel(const __grid_constant__ CommitArgs a) {
-  const int pi = blockIdx.x, hk = blockIdx.y, b = blockIdx.z, c = threadIdx.x;
+__global__ void __launch_bounds__(kCommitThreads)
+    block_commit_kernel(const __grid_constant__ CommitArgs a) {
+  constexpr int VE = 16 / (int)sizeof(T);  // elements per 16-byte chunk
+  constexpr int CH = D / VE;               // chunks per row
+  extern __shared__ uint4 srows[];         // [page tokens][CH] new K rows
+  const int pi = blockIdx.x, hk = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int n = a.n_old[b], P = a.page_size;
   const int p = n / P + pi;  // logical page
   const int t0 = max(n, p * P), t1 = min(n + a.B, (p + 1) * P);
-  if (pi == 0 && hk == 0 && c == 0 && a.seq_len) a.seq_len[b] = n + a.B;
+  if (pi == 0 && hk == 0 && tid == 0 && a.seq_len) a.seq_len[b] = n + a.B;
   if (t0 >= t1) return;
   long long page_slot = (long long)b * a.max_seq_len + (long long)p * P;
   if (a.page_table) {
     const int pg = a.page_table[(long long)b * a.max_pages + p];
     if (pg < 0 || ((long long)pg + 1) * P > a.n_slots) {  // unmapped or outside the pool
-      if (c == 0) atomicOr(&g_fb_error_word, kErrBadPage);
+      if (tid == 0) atomicOr(&g_fb_error_word, kErrBadPage);
       return;
     }
     page_slot = (long long)pg * P;
   }
-  const T* kin = static_cast<const T*>(a.k_in);
-  const T* vin = static_cast<const T*>(a.v_in);
-  T* kc = static_cast<T*>(a.k);
-  T* vc = static_cast<T*>(a.v);
-  float mn = INFINITY, mx = -INFINITY;
-  for (int t = t0; t < t1; ++t) {
-    const long long src = (((long long)b * a.B + (t - n)) * a.Hkv + hk) * D + c;
-    const long long dst = ((page_slot + (t - p * P)) * a.Hkv + hk) * D + c;
-    const T kx = kin[src];
-    kc[dst] = kx;
-    vc[dst] = vin[src];
-    const float f = commit_f32<T>(kx);
-    mn = fminf(mn, f);
-    mx = fmaxf(mx, f);
+  const uint4* __restrict__ kin = static_cast<const uint4*>(a.k_in);
+  const uint4* __restrict__ vin = static_cast<const uint4*>(a.v_in);
+  uint4* __restrict__ kc = static_cast<uint4*>(a.k);
+  uint4* __restrict__ vc = static_cast<uint4*>(a.v);
+  const int nt = t1 - t0, total = nt * CH;
+  // at most 4 chunks of K and V per thread in flight at once
+  for (int base = 0; base < total; base += 4 * kCommitThreads) {
+    uint4 kx[4], vx[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int idx = base + r * kCommitThreads + tid;
+      if (idx < total) {
+        const int u = idx / CH, v = idx - u * CH;
+        const long long src = (((long long)b * a.B + (t0 + u - n)) * a.Hkv + hk) * CH + v;
+        kx[r] = kin[src];
+        vx[r] = vin[src];
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int idx = base + r * kCommitThreads + tid;
+      if (idx < total) {
+        const int u = idx / CH, v = idx - u * CH;
+        const long long dst = ((page_slot + (t0 + u - p * P)) * a.Hkv + hk) * CH + v;
+        kc[dst] = kx[r];
+        vc[dst] = vx[r];
+        srows[u * CH + v] = kx[r];
+      }
+    }
   }
-  if (a.pmin) {
-    T* smin = static_cast<T*>(a.pmin);
-    T* smax = static_cast<T*>(a.pmax);
+  if (!a.pmin) return;
+  __syncthreads();
+  const T* sk = reinterpret_cast<const T*>(srows);
+  T* smin = static_cast<T*>(a.pmin);
+  T* smax = static_cast<T*>(a.pmax);
+  for (int c = tid; c < D; c += kCommitThreads) {
+    float mn = INFINITY, mx = -INFINITY;
+    for (int u = 0; u < nt; ++u) {
+      const float f = commit_f32<T>(sk[u * D + c]);
+      mn = fminf(mn, f);
+      mx = fmaxf(mx, f);
+    }
     const long long o = (((long long)b * a.max_pages + p) * a.Hkv + hk) * D + c;
     if (n > p * P) {  // the page already held tokens: fold in its summary
       mn = fminf(mn, commit_f32<T>(smin[o]));

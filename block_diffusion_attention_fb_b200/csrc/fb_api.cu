@@ -17,7 +17,6 @@
 
 #include "../../include/fb.h"
 #include "attn.cuh"
-#include "attn_persistent.cuh"
 #include "attn_tc2.cuh"
 #include "block_attn.cuh"
 #include "commit.cuh"
@@ -206,41 +205,14 @@ size_t partial_bytes(const Plan& p, int batch, int Hkv, int R, int D) {
   return round_up(rows * D * 4, 256) + round_up(rows * 4, 256);
 }
 
-// The persistent kernel serves the LoSA gather (bf16, page lists, at most one
-// 64-row tile per kv head): union sizes are known only on the device, and it
-// balances the tiles actually present over the SMs. Dense prefixes run on the
-// grid kernel, whose three-stage pipeline streams faster (measured: dllm prefix
-// 135 us against 156 us).
-bool use_persistent(fb_dtype dt, int batch, int Hkv, int R, bool page_list) {
-  return dt == FB_BF16 && page_list && R <= 64 && (long long)batch * Hkv <= kMaxGroupsP;
-}
-
-// Persistent launch: CTAs (two per SM, at most one per tile) and workspace
-// (two partial slots per CTA + one ticket per group).
-struct PersistPlan {
-  int n_cta;
-  size_t o_off, l_off, t_off, bytes;
-};
-
-PersistPlan persist_plan(int batch, int Hkv, int R, int D, int max_tiles, int num_sms) {
-  PersistPlan p{};
-  const long long upper = (long long)batch * Hkv * (max_tiles < 1 ? 1 : max_tiles);
-  const long long slots = (long long)(num_sms > 0 ? num_sms : 148) * kPersistCtasPerSm;
-  p.n_cta = (int)(upper < slots ? upper : slots);
-  if (p.n_cta < 1) p.n_cta = 1;
-  const size_t rows = (size_t)p.n_cta * 2 * R;
-  p.o_off = 0;
-  p.l_off = round_up(rows * D * 4, 256);
-  p.t_off = p.l_off + round_up(rows * 4, 256);
-  p.bytes = p.t_off + round_up((size_t)batch * Hkv * 4, 256);
-  return p;
-}
-
-// Workspace bytes of one attention-partial launch, whichever kernel serves it.
+// Workspace bytes of one attention-partial launch (split partials).
+// Page-list attention (LoSA gather, sparse residual) runs on the same split grid
+// kernels as dense prefixes: measured against a persistent stream-K kernel it
+// was faster on every page-list workload (dllm LoSA 108.6 vs 122.8 us per step,
+// sparse residual 96.6 vs 159.0; L = 131072: 180.9 vs 205.2 and 245.0 vs 343.5),
+// whose short per-CTA tile runs were latency-bound on group merges.
 size_t partial_ws_bytes(fb_dtype dt, int batch, int Hkv, int R, int D, int max_tiles,
-                        int num_sms, bool page_list = false) {
-  if (use_persistent(dt, batch, Hkv, R, page_list))
-    return persist_plan(batch, Hkv, R, D, max_tiles, num_sms).bytes;
+                        int num_sms) {
   return partial_bytes(make_plan(dt, batch, Hkv, R, max_tiles, num_sms, D), batch, Hkv, R, D);
 }
 
@@ -271,7 +243,7 @@ WsLayout ws_layout(const fb_kv* kv, int B, int Hq, int n_active, int topk, int n
     const int per_tile = kTK / (kv->page_size < kTK ? kv->page_size : kTK);
     const int ent = max_union_entries(kv, G, na, topk);
     const size_t pgb = partial_ws_bytes(kv->dtype, kv->batch, kv->n_heads_kv, na * G, D,
-                                        ceil_div(ent, per_tile), num_sms, true);
+                                        ceil_div(ent, per_tile), num_sms);
     part = part > pgb ? part : pgb;
     scores = round_up((size_t)kv->batch * na * Hq * logical_pages(kv) * 4, 256) +
              round_up((size_t)kv->batch * B * 4, 256);
@@ -417,53 +389,6 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
   } else {
     a.chunk = kv->page_table ? (kv->page_size < kTK ? kv->page_size : kTK) : kTK;
     max_tiles = ceil_div(kv->max_seq_len, kTK);
-  }
-  if (use_persistent(kv->dtype, kv->batch, Hkv, a.R, c.page_list != nullptr)) {
-    const PersistPlan pp = persist_plan(kv->batch, Hkv, a.R, D, max_tiles, c.num_sms);
-    if (!c.ws || c.ws_offset + pp.bytes > c.ws_bytes)
-      return fail(FB_ERR_WORKSPACE, "workspace too small: need %zu bytes at offset %zu, have %zu",
-                  pp.bytes, c.ws_offset, c.ws_bytes);
-    if (!aligned16(c.ws)) return fail(FB_ERR_ALIGN, "workspace not 16-byte aligned");
-    char* w = static_cast<char*>(c.ws) + c.ws_offset;
-    a.o_part = reinterpret_cast<float*>(w + pp.o_off);
-    a.lse_part = reinterpret_cast<float*>(w + pp.l_off);
-    a.tickets = reinterpret_cast<int*>(w + pp.t_off);
-    // tickets count a group's partials in; they start at zero on every call
-    if (cudaMemsetAsync(a.tickets, 0, (size_t)kv->batch * Hkv * 4, stream) != cudaSuccess)
-      return fail(FB_ERR_CUDA, "ticket reset failed");
-    a.row_tile = 64;
-    a.n_row_tiles = 1;
-    a.n_splits = 1;
-    a.tiles_per_split = max_tiles;
-    CUtensorMap tk, tv;
-    int rc = make_tmap(&tk, kv->k, D, Hkv, kv->n_slots, a.chunk);
-    if (rc) return rc;
-    rc = make_tmap(&tv, kv->v, D, Hkv, kv->n_slots, a.chunk);
-    if (rc) return rc;
-    const int rg = a.R <= 16 ? 1 : (a.R <= 32 ? 2 : 4);
-#define FB_LAUNCH_PERSIST(DD, RGV)                                                       \
-  do {                                                                                   \
-    auto kfn = attn_bf16_persistent<DD, RGV>;                                            \
-    if (int rc_ = set_smem_once((const void*)kfn, PersistSmem<DD>::kBytes)) return rc_;  \
-    kfn<<<pp.n_cta, kAttnThreads, PersistSmem<DD>::kBytes, stream>>>(a, tk, tv);         \
-  } while (0)
-    if (D == 128) {
-      if (rg == 1)
-        FB_LAUNCH_PERSIST(128, 1);
-      else if (rg == 2)
-        FB_LAUNCH_PERSIST(128, 2);
-      else
-        FB_LAUNCH_PERSIST(128, 4);
-    } else {
-      if (rg == 1)
-        FB_LAUNCH_PERSIST(64, 1);
-      else if (rg == 2)
-        FB_LAUNCH_PERSIST(64, 2);
-      else
-        FB_LAUNCH_PERSIST(64, 4);
-    }
-#undef FB_LAUNCH_PERSIST
-    return check_launch("persistent attention kernel");
   }
   Plan p = make_plan(kv->dtype, kv->batch, Hkv, a.R, max_tiles, c.num_sms, D);
   if (c.single_split) {
@@ -695,7 +620,7 @@ int sr_select(const void* q, int B, int Hq, const void* page_min, const void* pa
     return fail(FB_ERR_ALIGN, "page summaries not 16-byte aligned");
   const dim3 g2(ceil_div(v.max_pages, kPsPages), v.Hkv, kv->batch);
   const int es = (int)elem_size(kv->dtype);
-  const int psm = RQ * D * 4 + 2 * kPsPages * (D + 4 / es) * es;
+  const int psm = RQ * D * 4 + 2 * kPsPages * (D + 16 / es) * es;
   int rc;
 #define FB_HPS(TT, DD)                                                                       \
   do {                                                                                       \
@@ -792,17 +717,22 @@ int fb_block_commit(const fb_kv* kv, const int32_t* seq_len_host, const void* k_
   a.max_seq_len = kv->max_seq_len;
   const dim3 grid(max_touched, kv->n_heads_kv, kv->batch);
   if (grid.y > 65535) return fail(FB_ERR_SHAPE, "too many kv heads");
+  if (!aligned16(kv->k) || !aligned16(kv->v)) return fail(FB_ERR_ALIGN, "k / v not 16-byte aligned");
+  // shared memory: the new K rows of one page
+  const int sm = v.page_size * v.D * (int)elem_size(kv->dtype);
+  if (sm > 160 * 1024) return fail(FB_ERR_SHAPE, "page_size %d too large for the commit", v.page_size);
+#define FB_COMMIT(TT, DD)                                                          \
+  do {                                                                             \
+    auto kfn = block_commit_kernel<TT, DD>;                                        \
+    if (int rc_ = set_smem_once((const void*)kfn, sm)) return rc_;                \
+    kfn<<<grid, kCommitThreads, sm, stream>>>(a);                                  \
+  } while (0)
   if (kv->dtype == FB_BF16) {
-    if (v.D == 128)
-      block_commit_kernel<__nv_bfloat16, 128><<<grid, 128, 0, stream>>>(a);
-    else
-      block_commit_kernel<__nv_bfloat16, 64><<<grid, 64, 0, stream>>>(a);
+    if (v.D == 128) FB_COMMIT(__nv_bfloat16, 128); else FB_COMMIT(__nv_bfloat16, 64);
   } else {
-    if (v.D == 128)
-      block_commit_kernel<float, 128><<<grid, 128, 0, stream>>>(a);
-    else
-      block_commit_kernel<float, 64><<<grid, 64, 0, stream>>>(a);
+    if (v.D == 128) FB_COMMIT(float, 128); else FB_COMMIT(float, 64);
   }
+#undef FB_COMMIT
   return check_launch("block commit kernel");
 }
 
@@ -963,7 +893,7 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
   rc = check_launch("active rows kernel");
   if (rc) return rc;
   const dim3 g2(ceil_div(v.max_pages, kPsPages), v.Hkv, kv->batch);
-  const int psm = na * G * D * 4 + 2 * kPsPages * (D + 4 / (int)elem_size(kv->dtype)) *
+  const int psm = na * G * D * 4 + 2 * kPsPages * (D + 16 / (int)elem_size(kv->dtype)) *
                                        (int)elem_size(kv->dtype);
   if (kv->dtype == FB_BF16) {
     auto kfn = D == 128 ? page_score_kernel<__nv_bfloat16, 128> : page_score_kernel<__nv_bfloat16, 64>;

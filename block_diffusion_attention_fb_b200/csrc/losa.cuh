@@ -196,15 +196,69 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------------------------
 constexpr int kPsPages = 64;
 
+// Shared-memory row stride (elements) of the staged page summaries: rows stay
+// 16-byte aligned for vector loads, and consecutive pages start 4 banks apart,
+// so the 8 lanes of a quarter warp reading 16 bytes each hit distinct banks.
+template <typename T, int D>
+__host__ __device__ constexpr int ps_stride() {
+  return D + 16 / (int)sizeof(T);
+}
+
+// 8 consecutive elements as float (exact for bf16 and f32) from shared memory.
+__device__ __forceinline__ void load8_f32(const __nv_bfloat16* p, float (&o)[8]) {
+  const uint4 v = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    o[2 * j] = __uint_as_float(w[j] << 16);
+    o[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void load8_f32(const float* p, float (&o)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+  o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+}
+
+// QUEST-style bound of one q row over one staged page:
+//   tree_sum_c max(q_c * kmin_c, q_c * kmax_c)
+// single-rounded products, then the stride-halving tree over c (level 1 pairs
+// c with c + D/2). Operands are read 8 channels per shared-memory load; the
+// arithmetic and its order are those of the definition.
+template <typename T, int D>
+__device__ __forceinline__ float page_bound(const float* qr, const T* mnr, const T* mxr) {
+  float y[D / 2];
+#pragma unroll
+  for (int c8 = 0; c8 < D / 2; c8 += 8) {
+    float q0[8], q1[8], n0[8], n1[8], x0[8], x1[8];
+    load8_f32(qr + c8, q0);
+    load8_f32(qr + c8 + D / 2, q1);
+    load8_f32(mnr + c8, n0);
+    load8_f32(mnr + c8 + D / 2, n1);
+    load8_f32(mxr + c8, x0);
+    load8_f32(mxr + c8 + D / 2, x1);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float a0 = fmaxf(__fmul_rn(q0[j], n0[j]), __fmul_rn(q0[j], x0[j]));
+      const float a1 = fmaxf(__fmul_rn(q1[j], n1[j]), __fmul_rn(q1[j], x1[j]));
+      y[c8 + j] = __fadd_rn(a0, a1);
+    }
+  }
+#pragma unroll
+  for (int st = D / 4; st >= 1; st >>= 1)
+#pragma unroll
+    for (int c = 0; c < st; ++c) y[c] = __fadd_rn(y[c], y[c + st]);
+  return y[0];
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
     page_score_kernel(const T* __restrict__ q, const int32_t* __restrict__ active, int B, int Hq,
                       int G, int n_act, const T* __restrict__ pmin, const T* __restrict__ pmax,
                       const KvView kv, float* __restrict__ scores, uint32_t* __restrict__ bitmap,
                       int words) {
-  // rows padded by one 32-bit word: threads reading the same channel of
-  // consecutive pages hit different banks
-  constexpr int PS = D + 4 / (int)sizeof(T);
+  constexpr int PS = ps_stride<T, D>();
   constexpr int VE = 16 / (int)sizeof(T);  // elements per 16-byte global load
   extern __shared__ float sm[];
   const int RQ = n_act * G;
@@ -234,34 +288,17 @@ __global__ void __launch_bounds__(256)
       mn = *reinterpret_cast<const uint4*>(pmin + so);
       mx = *reinterpret_cast<const uint4*>(pmax + so);
     }
-    uint32_t* dn = reinterpret_cast<uint32_t*>(smn + pg * PS + cv * VE);  // 4-byte aligned
-    uint32_t* dx = reinterpret_cast<uint32_t*>(smx + pg * PS + cv * VE);
-    dn[0] = mn.x; dn[1] = mn.y; dn[2] = mn.z; dn[3] = mn.w;
-    dx[0] = mx.x; dx[1] = mx.y; dx[2] = mx.z; dx[3] = mx.w;
+    *reinterpret_cast<uint4*>(smn + pg * PS + cv * VE) = mn;
+    *reinterpret_cast<uint4*>(smx + pg * PS + cv * VE) = mx;
   }
   __syncthreads();
   for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
     const int pg = task % kPsPages, rq = task / kPsPages;
     const int p = p0 + pg;
     if (p >= n_pages) continue;
-    const float* qr = qs + rq * D;
-    const T* mnr = smn + pg * PS;
-    const T* mxr = smx + pg * PS;
-    float y[D / 2];
-#pragma unroll
-    for (int c = 0; c < D / 2; ++c) {
-      const float q0 = qr[c], q1 = qr[c + D / 2];
-      const float x0 = fmaxf(__fmul_rn(q0, ld_f32<T>(mnr + c)), __fmul_rn(q0, ld_f32<T>(mxr + c)));
-      const float x1 = fmaxf(__fmul_rn(q1, ld_f32<T>(mnr + c + D / 2)),
-                             __fmul_rn(q1, ld_f32<T>(mxr + c + D / 2)));
-      y[c] = __fadd_rn(x0, x1);
-    }
-#pragma unroll
-    for (int st = D / 4; st >= 1; st >>= 1)
-#pragma unroll
-      for (int c = 0; c < st; ++c) y[c] = __fadd_rn(y[c], y[c + st]);
+    const float yb = page_bound<T, D>(qs + rq * D, smn + pg * PS, smx + pg * PS);
     const int a_i = rq / G, g = rq - (rq / G) * G;
-    scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = y[0];
+    scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = yb;
   }
 }
 
@@ -448,7 +485,7 @@ __global__ void __launch_bounds__(256)
                            const T* __restrict__ pmin, const T* __restrict__ pmax,
                            const KvView kv, float* __restrict__ scores,
                            uint32_t* __restrict__ bitmap, int words) {
-  constexpr int PS = D + 4 / (int)sizeof(T);
+  constexpr int PS = ps_stride<T, D>();
   constexpr int VE = 16 / (int)sizeof(T);
   extern __shared__ float sm[];
   __shared__ uint32_t best[kPsPages];
@@ -478,33 +515,16 @@ __global__ void __launch_bounds__(256)
       mn = *reinterpret_cast<const uint4*>(pmin + so);
       mx = *reinterpret_cast<const uint4*>(pmax + so);
     }
-    uint32_t* dn = reinterpret_cast<uint32_t*>(smn + pg * PS + cv * VE);
-    uint32_t* dx = reinterpret_cast<uint32_t*>(smx + pg * PS + cv * VE);
-    dn[0] = mn.x; dn[1] = mn.y; dn[2] = mn.z; dn[3] = mn.w;
-    dx[0] = mx.x; dx[1] = mx.y; dx[2] = mx.z; dx[3] = mx.w;
+    *reinterpret_cast<uint4*>(smn + pg * PS + cv * VE) = mn;
+    *reinterpret_cast<uint4*>(smx + pg * PS + cv * VE) = mx;
   }
   __syncthreads();
   for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
     const int pg = task % kPsPages, rq = task / kPsPages;
     const int p = p0 + pg;
     if (p >= n_pages) continue;
-    const float* qr = qs + rq * D;
-    const T* mnr = smn + pg * PS;
-    const T* mxr = smx + pg * PS;
-    float y[D / 2];
-#pragma unroll
-    for (int c = 0; c < D / 2; ++c) {
-      const float q0 = qr[c], q1 = qr[c + D / 2];
-      const float x0 = fmaxf(__fmul_rn(q0, ld_f32<T>(mnr + c)), __fmul_rn(q0, ld_f32<T>(mxr + c)));
-      const float x1 = fmaxf(__fmul_rn(q1, ld_f32<T>(mnr + c + D / 2)),
-                             __fmul_rn(q1, ld_f32<T>(mxr + c + D / 2)));
-      y[c] = __fadd_rn(x0, x1);
-    }
-#pragma unroll
-    for (int st = D / 4; st >= 1; st >>= 1)
-#pragma unroll
-      for (int c = 0; c < st; ++c) y[c] = __fadd_rn(y[c], y[c + st]);
-    atomicMax(&best[pg], order_key(y[0]));
+    const float yb = page_bound<T, D>(qs + rq * D, smn + pg * PS, smx + pg * PS);
+    atomicMax(&best[pg], order_key(yb));
   }
   __syncthreads();
   for (int pg = threadIdx.x; pg < kPsPages; pg += blockDim.x) {
