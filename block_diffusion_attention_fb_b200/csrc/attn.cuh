@@ -28,6 +28,8 @@ constexpr int kStages = 3;   // TMA pipeline depth
 constexpr int kNWC = 4;      // consumer warps per CTA (bf16)
 constexpr int kAttnThreads = (kNWC + 1) * 32;
 constexpr int kMaxChunks = kTK / 16;  // TMA boxes per tile and half (page >= 16)
+constexpr int kSlotAhead = 3;  // tiles whose chunk slots a producer fetches ahead
+constexpr int kSlotRing = kSlotAhead + 1;
 
 struct AttnArgs {
   const void* q;  // [batch, B, Hq, D]
@@ -348,6 +350,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   __shared__ int meta[kStages][kMaxChunks];
   __shared__ int meta_full[kStages];
   __shared__ int abort_flag;
+  // chunk slots / valid counts of upcoming tiles, filled by the producer warp
+  __shared__ int ring_slot[kSlotRing][kMaxChunks];
+  __shared__ int ring_valid[kSlotRing][kMaxChunks];
   extern __shared__ uint8_t dyn_smem[];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -379,46 +384,73 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 
   if (warp == kNWC) {
     // ----------------------------- producer -----------------------------
+    // Lane 0 waits for free stages and issues the copies; all lanes fetch the
+    // chunk slots of the tile kSlotAhead tiles ahead (one chunk per lane) into
+    // a shared ring, so page-list / page-table reads overlap earlier copies.
+    auto fill = [&](int it) {  // tile `it` -> ring entry it % kSlotRing (all lanes)
+      if (lane < n_chunks) {
+        long long s_ = a.n_slots;
+        int v_ = 0;
+        chunk_slot(a, b, hk, tile0 + it, lane, s_, v_);
+        ring_slot[it % kSlotRing][lane] = (int)s_;
+        ring_valid[it % kSlotRing][lane] = v_;
+      }
+    };
+    for (int it = 0; it < kSlotAhead && it < n_it; ++it) fill(it);
+    __syncwarp();
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      int issued = 0;
-      for (int it = 0; it < n_it; ++it) {
+    }
+    int issued = 0;
+    for (int it = 0; it < n_it; ++it) {
+      // entry (it + kSlotAhead) % kSlotRing last served tile it - 1
+      if (it + kSlotAhead < n_it) fill(it + kSlotAhead);
+      int ok = 1;
+      if (lane == 0) {
         const int st = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
-        if (!mbar_wait(&empty_bar[st], ph ^ 1, &abort_flag)) break;
-        long long slots[kMaxChunks];
-        int all_full = 1;
-        for (int c = 0; c < n_chunks; ++c) {
-          int valid;
-          chunk_slot(a, b, hk, tile0 + it, c, slots[c], valid);
-          meta[st][c] = valid;
-          all_full &= (valid == a.chunk);
-        }
-        meta_full[st] = all_full;
-        mbar_arrive_expect_tx(&full_bar[st], S::kStageBytes);
-        uint8_t* sk = base_ptr + st * S::kStageBytes;
-        uint8_t* sv = sk + S::kTileBytes;
-        for (int c = 0; c < n_chunks; ++c) {
-          const int z = (int)slots[c];
+        const int re = it % kSlotRing;
+        ok = mbar_wait(&empty_bar[st], ph ^ 1, &abort_flag);
+        if (ok) {
+          int all_full = 1;
 #pragma unroll
-          for (int hf = 0; hf < S::kHalves; ++hf) {
-            uint8_t* dk = sk + hf * S::kHalfBytes + c * a.chunk * 128;
-            uint8_t* dv = sv + hf * S::kHalfBytes + c * a.chunk * 128;
-            tma_load_3d(dk, &tmK, hf * 64, hk, z, &full_bar[st]);
-            tma_load_3d(dv, &tmV, hf * 64, hk, z, &full_bar[st]);
+          for (int c = 0; c < kMaxChunks; ++c) {
+            if (c < n_chunks) {
+              meta[st][c] = ring_valid[re][c];
+              all_full &= (ring_valid[re][c] == a.chunk);
+            }
           }
+          meta_full[st] = all_full;
+          mbar_arrive_expect_tx(&full_bar[st], S::kStageBytes);
+          uint8_t* sk = base_ptr + st * S::kStageBytes;
+          uint8_t* sv = sk + S::kTileBytes;
+#pragma unroll
+          for (int c = 0; c < kMaxChunks; ++c) {
+            if (c < n_chunks) {
+              const int z = ring_slot[re][c];
+#pragma unroll
+              for (int hf = 0; hf < S::kHalves; ++hf) {
+                uint8_t* dk = sk + hf * S::kHalfBytes + c * a.chunk * 128;
+                uint8_t* dv = sv + hf * S::kHalfBytes + c * a.chunk * 128;
+                tma_load_3d(dk, &tmK, hf * 64, hk, z, &full_bar[st]);
+                tma_load_3d(dv, &tmV, hf * 64, hk, z, &full_bar[st]);
+              }
+            }
+          }
+          ++issued;
         }
-        ++issued;
       }
-      if (abort_flag) {
-        // let copies already in flight land before the CTA's memory goes away
-        const long long t0 = clock64();
-        for (int it = max(0, issued - kStages); it < issued; ++it) {
-          const int st = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
-          while (!mbar_try_wait(&full_bar[st], ph) && clock64() - t0 < kWaitBudgetCycles) {
-          }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      __syncwarp();  // ring entries written this iteration are visible to lane 0 next time
+    }
+    if (lane == 0 && abort_flag) {
+      // let copies already in flight land before the CTA's memory goes away
+      const long long t0 = clock64();
+      for (int it = max(0, issued - kStages); it < issued; ++it) {
+        const int st = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        while (!mbar_try_wait(&full_bar[st], ph) && clock64() - t0 < kWaitBudgetCycles) {
         }
       }
     }

@@ -77,6 +77,9 @@ __global__ void __launch_bounds__(kT2Threads, 1)
   // barrier advance twice.
   __shared__ int meta[kT2Meta][2 * kMaxChunks];
   __shared__ int meta_full[kT2Meta];
+  // chunk slots / valid counts of upcoming tiles, filled by the producer warp
+  __shared__ int ring_slot[kSlotRing][2 * kMaxChunks];
+  __shared__ int ring_valid[kSlotRing][2 * kMaxChunks];
   __shared__ int abort_flag;
   __shared__ uint32_t tmem_base_sh;
   extern __shared__ uint8_t dyn_smem[];
@@ -128,77 +131,78 @@ __global__ void __launch_bounds__(kT2Threads, 1)
   if (warp == kT2Producer) {
     reg_dealloc<kT2LowRegs>();
     // ------------------------------ TMA producer ------------------------------
+    // Lane 0 waits for free slots and issues the copies; all 32 lanes fetch the
+    // chunk slots of the tile kSlotAhead tiles ahead (one chunk per lane, the
+    // page-list / page-table reads of a tile in flight together) into a small
+    // shared ring, so those reads overlap the copies of the tiles before it.
+    constexpr int kC = 2 * kMaxChunks;
+    const int nc2 = 2 * n_chunks;  // chunks per 128-key tile
+    auto fill = [&](int it) {      // tile `it` -> ring entry it % kSlotRing (all lanes)
+      if (lane < nc2) {
+        // chunk c covers keys [c * chunk, (c + 1) * chunk) of the 128-key tile; a
+        // sub-tile past the split's range gives valid = 0 (a zero-filled box)
+        const int sub = lane / n_chunks, cc = lane - sub * n_chunks;
+        long long s_ = a.n_slots;
+        int v_ = 0;
+        if (2 * it + sub < n64) chunk_slot(a, b, hk, tile0 + 2 * it + sub, cc, s_, v_);
+        ring_slot[it % kSlotRing][lane] = (int)s_;
+        ring_valid[it % kSlotRing][lane] = v_;
+      }
+    };
+    for (int it = 0; it < kSlotAhead && it < n_it; ++it) fill(it);
+    __syncwarp();
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      int issued = 0;  // loads issued (K_0 = 0, V_0 = 1, K_1 = 2, ...)
-      // Slots and valid counts of the chunks of tile `it` (chunk c covers keys
-      // [c * chunk, (c + 1) * chunk) of the 128-key tile; a sub-tile past the
-      // split's range gives valid = 0, a zero-filled box). Unrolled over the
-      // fixed maximum, so the page-table reads of a tile are independent
-      // loads in flight together; tile it + 1's are issued right after tile
-      // it's copies, ahead of the wait for a free slot.
-      constexpr int kC = 2 * kMaxChunks;
-      int sl_cur[kC], va_cur[kC], sl_nxt[kC], va_nxt[kC];
-      auto tile_slots = [&](int it, int (&sl)[kC], int (&va)[kC]) {
-#pragma unroll
-        for (int c = 0; c < kC; ++c) {
-          long long s_ = a.n_slots;
-          int v_ = 0;
-          if (c < 2 * n_chunks) {
-            const int sub = c / n_chunks, cc = c - sub * n_chunks;
-            if (2 * it + sub < n64) chunk_slot(a, b, hk, tile0 + 2 * it + sub, cc, s_, v_);
-          }
-          sl[c] = (int)s_;
-          va[c] = v_;
-        }
-      };
-      if (n_it > 0) tile_slots(0, sl_cur, va_cur);
-      for (int n = 0; n < 2 * n_it; ++n) {
-        const int it = n >> 1, is_v = n & 1;
+    }
+    int issued = 0;  // loads issued (K_0 = 0, V_0 = 1, K_1 = 2, ...)
+    for (int n = 0; n < 2 * n_it; ++n) {
+      const int it = n >> 1, is_v = n & 1;
+      // ring entry (it + kSlotAhead) % kSlotRing last served tile it - 1, whose
+      // copies were issued in the previous iterations
+      if (!is_v && it + kSlotAhead < n_it) fill(it + kSlotAhead);
+      int ok = 1;
+      if (lane == 0) {
         const int sl = n % kT2Slots;
-        if (!mbar_wait(&empty_bar[sl], ((n / kT2Slots) & 1) ^ 1, &abort_flag)) break;
-        if (!is_v) {
-          const int me = it % kT2Meta;
-          int all_full = 1;
+        const int re = it % kSlotRing;
+        ok = mbar_wait(&empty_bar[sl], ((n / kT2Slots) & 1) ^ 1, &abort_flag);
+        if (ok) {
+          if (!is_v) {
+            const int me = it % kT2Meta;
+            int all_full = 1;
+#pragma unroll
+            for (int c = 0; c < kC; ++c) {
+              if (c < nc2) {
+                meta[me][c] = ring_valid[re][c];
+                all_full &= (ring_valid[re][c] == a.chunk);
+              }
+            }
+            meta_full[me] = all_full;
+            mbar_arrive(&meta_bar[me]);  // release: the entry is written
+          }
+          mbar_arrive_expect_tx(&full_bar[sl], S::kKVTile);
+          uint8_t* dst = base_ptr + (sKV0 - base) + sl * S::kKVTile;
+          const CUtensorMap* tm = is_v ? &tmV : &tmK;
 #pragma unroll
           for (int c = 0; c < kC; ++c) {
-            if (c < 2 * n_chunks) {
-              meta[me][c] = va_cur[c];
-              all_full &= (va_cur[c] == a.chunk);
+            if (c < nc2) {
+              const int z = ring_slot[re][c];
+              tma_load_3d(dst + c * a.chunk * 128, tm, 0, hk, z, &full_bar[sl]);
+              tma_load_3d(dst + S::kKVHalf + c * a.chunk * 128, tm, 64, hk, z, &full_bar[sl]);
             }
           }
-          meta_full[me] = all_full;
-          mbar_arrive(&meta_bar[me]);  // release: the entry is written
-        }
-        mbar_arrive_expect_tx(&full_bar[sl], S::kKVTile);
-        uint8_t* dst = base_ptr + (sKV0 - base) + sl * S::kKVTile;
-        const CUtensorMap* tm = is_v ? &tmV : &tmK;
-#pragma unroll
-        for (int c = 0; c < kC; ++c) {
-          if (c < 2 * n_chunks) {
-            tma_load_3d(dst + c * a.chunk * 128, tm, 0, hk, sl_cur[c], &full_bar[sl]);
-            tma_load_3d(dst + S::kKVHalf + c * a.chunk * 128, tm, 64, hk, sl_cur[c],
-                        &full_bar[sl]);
-          }
-        }
-        ++issued;
-        if (is_v && it + 1 < n_it) {
-          tile_slots(it + 1, sl_nxt, va_nxt);
-#pragma unroll
-          for (int c = 0; c < kC; ++c) {
-            sl_cur[c] = sl_nxt[c];
-            va_cur[c] = va_nxt[c];
-          }
+          ++issued;
         }
       }
-      if (abort_flag) {
-        // let copies already in flight land before the CTA's memory goes away
-        const long long t0 = clock64();
-        for (int n = max(0, issued - kT2Slots); n < issued; ++n) {
-          while (!mbar_try_wait(&full_bar[n % kT2Slots], (n / kT2Slots) & 1) &&
-                 clock64() - t0 < kWaitBudgetCycles) {
-          }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      __syncwarp();  // ring entries written this iteration are visible to lane 0 next time
+    }
+    if (lane == 0 && abort_flag) {
+      // let copies already in flight land before the CTA's memory goes away
+      const long long t0 = clock64();
+      for (int n = max(0, issued - kT2Slots); n < issued; ++n) {
+        while (!mbar_try_wait(&full_bar[n % kT2Slots], (n / kT2Slots) & 1) &&
+               clock64() - t0 < kWaitBudgetCycles) {
         }
       }
     }

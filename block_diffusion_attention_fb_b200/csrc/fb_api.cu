@@ -106,6 +106,7 @@ size_t elem_size(fb_dtype t) { return t == FB_BF16 ? 2 : 4; }
 // Tuning overrides read from the environment (0 or unset: automatic):
 //   FB_SPLIT_WAVES  resident-CTA waves of the streaming (mma.sync / fp32) plan
 //   FB_TC_SPLITS    splits per row tile of the tcgen05 plan
+//   FB_LIST_WAVES   resident-CTA waves of page-list plans (LoSA gather, sparse residual)
 int env_int(const char* name, int lo, int hi) {
   const char* e = getenv(name);
   if (e && *e) {
@@ -162,7 +163,8 @@ int tc_splits(long long units, int slots, int max_tiles, int batch) {
   return best;
 }
 
-Plan make_plan(fb_dtype dt, int batch, int Hkv, int R, int max_tiles, int num_sms, int D = 128) {
+Plan make_plan(fb_dtype dt, int batch, int Hkv, int R, int max_tiles, int num_sms, int D = 128,
+               bool page_list = false) {
   Plan p{};
   const int sms = num_sms > 0 ? num_sms : 148;
   max_tiles = max_tiles < 1 ? 1 : max_tiles;
@@ -188,7 +190,16 @@ Plan make_plan(fb_dtype dt, int batch, int Hkv, int R, int max_tiles, int num_sm
     }
     p.n_row_tiles = ceil_div(R, p.row_tile);
     const long long units = (long long)batch * Hkv * p.n_row_tiles;
-    const int waves = env_int("FB_SPLIT_WAVES", 1, 64);
+    int waves = env_int("FB_SPLIT_WAVES", 1, 64);
+    if (page_list) {
+      // Page lists are planned on their upper bound (the counts live on the
+      // device). Several sequences have unions of different sizes, so a second
+      // wave lets the CTA scheduler balance them (measured, batch-8 GQA LoSA:
+      // 590 us per step at one wave, 400 at two, 409 at four; single-sequence
+      // workloads are fastest at one wave).
+      waves = env_int("FB_LIST_WAVES", 1, 64);
+      if (!waves) waves = batch > 1 ? 2 : 1;
+    }
     splits = (long long)sms * 2 * (waves ? waves : 1) / units;
   }
   if (splits < 1) splits = 1;
@@ -212,8 +223,9 @@ size_t partial_bytes(const Plan& p, int batch, int Hkv, int R, int D) {
 // sparse residual 96.6 vs 159.0; L = 131072: 180.9 vs 205.2 and 245.0 vs 343.5),
 // whose short per-CTA tile runs were latency-bound on group merges.
 size_t partial_ws_bytes(fb_dtype dt, int batch, int Hkv, int R, int D, int max_tiles,
-                        int num_sms) {
-  return partial_bytes(make_plan(dt, batch, Hkv, R, max_tiles, num_sms, D), batch, Hkv, R, D);
+                        int num_sms, bool page_list = false) {
+  return partial_bytes(make_plan(dt, batch, Hkv, R, max_tiles, num_sms, D, page_list), batch, Hkv,
+                       R, D);
 }
 
 // Workspace regions shared by every entry point (offsets in bytes).
@@ -243,7 +255,7 @@ WsLayout ws_layout(const fb_kv* kv, int B, int Hq, int n_active, int topk, int n
     const int per_tile = kTK / (kv->page_size < kTK ? kv->page_size : kTK);
     const int ent = max_union_entries(kv, G, na, topk);
     const size_t pgb = partial_ws_bytes(kv->dtype, kv->batch, kv->n_heads_kv, na * G, D,
-                                        ceil_div(ent, per_tile), num_sms);
+                                        ceil_div(ent, per_tile), num_sms, true);
     part = part > pgb ? part : pgb;
     scores = round_up((size_t)kv->batch * na * Hq * logical_pages(kv) * 4, 256) +
              round_up((size_t)kv->batch * B * 4, 256);
@@ -390,7 +402,8 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
     a.chunk = kv->page_table ? (kv->page_size < kTK ? kv->page_size : kTK) : kTK;
     max_tiles = ceil_div(kv->max_seq_len, kTK);
   }
-  Plan p = make_plan(kv->dtype, kv->batch, Hkv, a.R, max_tiles, c.num_sms, D);
+  Plan p = make_plan(kv->dtype, kv->batch, Hkv, a.R, max_tiles, c.num_sms, D,
+                     c.page_list != nullptr);
   if (c.single_split) {
     p.tiles_per_split = max_tiles < 1 ? 1 : max_tiles;
     p.n_splits = 1;
