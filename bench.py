@@ -62,6 +62,9 @@ def parse_args():
                                       "prefix", "block"],
                    default="all",
                    help="all: the contract line; one mode: time only that mode (for profiling)")
+    p.add_argument("--sweep", action="store_true",
+                   help="long-context sweep instead of the contract line: dense vs reuse per "
+                   "denoise step over prefixes of 32k..800k tokens (one JSON line per length)")
     p.add_argument("--workload", choices=["dllm", "tiny", "gqa", "video", "losa"],
                    default="dllm", help="dllm is the contract workload; the others are for "
                    "the per-configuration table")
@@ -614,6 +617,98 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+SWEEP_LENGTHS = (32768, 65536, 131072, 262144, 524288, 819200)
+
+
+def run_sweep(args, rank, world):
+    """Per-denoise-step attention at growing context, dllm head configuration
+    (32 heads MHA, d=128, block 32, tau=4 schedule of the dllm steps): the dense
+    prefix call, the dense step and the FlashBlock reuse step, each a CUDA graph
+    per denoise step with the L2 flushed before it; prefixes drawn on the GPU
+    (workloads.long_context)."""
+    import torch
+
+    import block_diffusion_attention_fb_b200 as fb
+    from block_diffusion_attention_fb_b200.runtime import BlockAttention
+    from workloads import make_workload
+    from workloads.long_context import long_prefix
+    from workloads.torch_io import to_torch
+
+    fb.load_library()
+    wl = make_workload("dllm", prefix_min=16, prefix_max=16)
+    sp = wl.spec
+    steps = list(wl.steps())
+    S, B, Hq, d = sp.steps, sp.block, sp.n_heads_q, sp.head_dim
+    dq = [to_torch(x.q, "bf16") for x in steps]
+    dk = [to_torch(x.k_in, "bf16") for x in steps]
+    dv = [to_torch(x.v_in, "bf16") for x in steps]
+    ms = [x.m_updated.tolist() for x in steps]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_rd = torch.zeros(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    A = torch.zeros(1, B, Hq, d, device="cuda")
+    L = torch.zeros(1, B, Hq, device="cuda")
+    peaks = measured_peaks()
+    K, W = args.steps, max(1, args.warmup)
+    for n_tok in SWEEP_LENGTHS:
+        k, v, _ = long_prefix(n_tok, sp.n_heads_kv, d, seed=2000 + n_tok)
+        seq_len = torch.tensor([n_tok], dtype=torch.int32, device="cuda")
+        kv = fb.KV(k, v, seq_len=seq_len, page_table=None, page_size=16, max_seq_len=n_tok)
+        reuse = BlockAttention(kv, B, Hq, "threshold", tau=sp.tau)
+        dense = BlockAttention(kv, B, Hq, "threshold", tau=0)
+
+        def run(blk):
+            def step(s):
+                if s == 0:
+                    blk.reset()
+                blk.step(dq[s], dk[s], dv[s], A, L, m_updated=ms[s])
+            return step
+
+        graphs = {}
+        for name, blk in (("reuse", reuse), ("dense", dense)):
+            fn = run(blk)
+            for _ in range(W):
+                for s in range(S):
+                    fn(s)
+            torch.cuda.synchronize()
+            gl = []
+            for s in range(S):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    fn(s)
+                gl.append(g)
+            graphs[name] = gl
+        tot = {}
+        for name, gl in graphs.items():
+            pairs = []
+            for _ in range(K):
+                for s in range(S):
+                    flush.zero_()
+                    flush_rd.max()
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    gl[s].replay()
+                    e1.record()
+                    pairs.append((e0, e1))
+            torch.cuda.synchronize()
+            tot[name] = sum(a.elapsed_time(b) for a, b in pairs) * 1000 / (K * S)
+        kv_bytes = 2 * n_tok * sp.n_heads_kv * d * 2
+        line = {"sweep": "long_context", "prefix_tokens": n_tok,
+                "config": "dllm heads: 32 MHA, head_dim 128, block 32, 32 denoise steps, "
+                          "tau 4 schedule; prefix drawn on the GPU",
+                "dense_us_per_step": round(tot["dense"], 2),
+                "reuse_us_per_step": round(tot["reuse"], 2),
+                "reuse_speedup": round(tot["dense"] / tot["reuse"], 3),
+                "prefix_recomputes_per_block": sum(1 for s in range(S) if s == 0 or ms[s][0] >= sp.tau),
+                "dense_step_kv_gbs": round(kv_bytes / (tot["dense"] * 1e-6) / 1e9, 1),
+                "dense_step_kv_frac_of_hbm": round(kv_bytes / (tot["dense"] * 1e-6) / 1e9 /
+                                                   peaks["gbs"], 4)}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        del graphs, reuse, dense, kv, k, v
+        torch.cuda.empty_cache()
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -623,7 +718,10 @@ def main():
         return
     rank, world, local = dist_init(args.gpus)
     try:
-        run_ours(args, rank, world, local)
+        if args.sweep:
+            run_sweep(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -186,3 +186,32 @@ def test_losa_full_size():
         A_ref, L_ref = _oracle_full_rows(wl, st, samples, A_out_rows, L_out_rows)
         _check_rows(cpu(A), cpu(L), samples, A_ref, L_ref, sp.dtype, f"losa step {st.step}")
         q_prev = st.q
+
+
+def test_long_context_prefix_partial_sampled():
+    """A 262144-token prefix (the long-context sweep's lengths run to 819200):
+    sampled rows of two kv heads against the oracle on CPU copies of those heads."""
+    from oracle.attention import partial, to_f64
+    from workloads.long_context import long_prefix
+    n_tok = 262144
+    k, v, _ = long_prefix(n_tok, 32, 128, seed=2262144)
+    wl = make_workload("dllm", prefix_min=16, prefix_max=16)
+    sp = wl.spec
+    st = next(wl.steps(1))
+    seq_len = torch.tensor([n_tok], dtype=torch.int32, device="cuda")
+    kv = fb.KV(k, v, seq_len=seq_len, page_table=None, page_size=16, max_seq_len=n_tok)
+    q = dev(st.q, sp.dtype)
+    A = torch.zeros(1, sp.block, sp.n_heads_q, sp.head_dim, device="cuda")
+    L = torch.zeros(1, sp.block, sp.n_heads_q, device="cuda")
+    ws = torch.empty(fb.fb_workspace_size(kv, sp.block, sp.n_heads_q), dtype=torch.uint8,
+                     device="cuda")
+    fb.fb_prefix_attn(q, kv, A, L, ws)
+    sync()
+    A, L = cpu(A), cpu(L)
+    for h in (0, 31):
+        K = to_f64(cpu(k[:, h].contiguous().view(torch.int16)).view(np.uint16), "bf16")
+        V = to_f64(cpu(v[:, h].contiguous().view(torch.int16)).view(np.uint16), "bf16")
+        rows = [0, 13, sp.block - 1]
+        a_ref, l_ref = partial(to_f64(st.q[0, rows, h], "bf16"), K, V)
+        assert_close_A(A[0, rows, h], a_ref, "bf16", f"head {h}")
+        assert_close_L(L[0, rows, h], l_ref, f"head {h}")
