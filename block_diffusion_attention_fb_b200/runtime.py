@@ -91,3 +91,97 @@ class BlockAttention:
     @property
     def recomputed(self) -> int:
         return self.cache.recomputed
+
+
+class HostBlockPipeline:
+    """A block's denoise steps fed from pinned host memory and returned to it.
+
+    Each step's q, k_in, v_in arrive as one packed host buffer (one copy in) and
+    its A_full, L_full leave as one packed buffer (one copy out). Copies run on
+    their own streams with `depth` device buffers in rotation, so the input copy
+    of step s+1 and the output copy of step s-1 overlap the attention of step
+    s; a step then costs about the larger of its copies and its attention. All
+    work is enqueued on the current stream and two copy streams that fork from
+    and join back into it, so a whole block can be captured in one CUDA graph.
+    Attention itself is one fb_step call per step, as in BlockAttention.step.
+    """
+
+    def __init__(self, blk: BlockAttention, dtype, depth: int = 3):
+        self.blk = blk
+        self.depth = depth
+        kv = blk.kv
+        dev = kv.k.device
+        batch, B, Hq, d = kv.batch, blk.B, blk.Hq, kv.c.head_dim
+        hkv = kv.c.n_heads_kv
+        self.q_shape = (batch, B, Hq, d)
+        self.kv_shape = (batch, B, hkv, d)
+        self.dtype = dtype
+        esz = torch.empty((), dtype=dtype).element_size()
+        self.nq = batch * B * Hq * d
+        self.nkv = batch * B * hkv * d
+        self.in_bytes = (self.nq + 2 * self.nkv) * esz
+        self.nA = batch * B * Hq * d
+        self.nL = batch * B * Hq
+        self.dev_in = [torch.empty(self.in_bytes, dtype=torch.uint8, device=dev) for _ in range(depth)]
+        self.dev_out = [torch.empty(self.nA + self.nL, dtype=torch.float32, device=dev)
+                        for _ in range(depth)]
+        self.s_in = torch.cuda.Stream(device=dev)
+        self.s_out = torch.cuda.Stream(device=dev)
+        self.in_done = [torch.cuda.Event() for _ in range(depth)]
+        self.comp_done = [torch.cuda.Event() for _ in range(depth)]
+        self.out_done = [torch.cuda.Event() for _ in range(depth)]
+
+    @property
+    def out_floats(self) -> int:
+        return self.nA + self.nL
+
+    def pack_inputs(self, q, k_in, v_in) -> torch.Tensor:
+        """One pinned host buffer holding q, k_in, v_in (in that order)."""
+        parts = [t.contiguous().view(torch.uint8).reshape(-1) for t in (q, k_in, v_in)]
+        buf = torch.empty(self.in_bytes, dtype=torch.uint8).pin_memory()
+        torch.cat(parts, out=buf)
+        return buf
+
+    def new_output(self) -> torch.Tensor:
+        """A pinned host buffer for one step's A_full then L_full (float32)."""
+        return torch.empty(self.out_floats, dtype=torch.float32).pin_memory()
+
+    def unpack_output(self, out: torch.Tensor):
+        return (out[: self.nA].view(*self.q_shape), out[self.nA:].view(*self.q_shape[:3]))
+
+    def _views(self, slot):
+        raw = self.dev_in[slot]
+        esz = torch.empty((), dtype=self.dtype).element_size()
+        q = raw[: self.nq * esz].view(self.dtype).view(*self.q_shape)
+        k = raw[self.nq * esz: (self.nq + self.nkv) * esz].view(self.dtype).view(*self.kv_shape)
+        v = raw[(self.nq + self.nkv) * esz:].view(self.dtype).view(*self.kv_shape)
+        out = self.dev_out[slot]
+        return q, k, v, out[: self.nA].view(*self.q_shape), out[self.nA:].view(*self.q_shape[:3])
+
+    def enqueue_block(self, host_in: Sequence[torch.Tensor], host_out: Sequence[torch.Tensor],
+                      m_updated: Optional[Sequence[Sequence[int]]] = None) -> None:
+        """Enqueues every step of a block (step 0 starts the block)."""
+        main = torch.cuda.current_stream()
+        self.s_in.wait_stream(main)   # fork: the copy streams follow all prior work
+        self.s_out.wait_stream(main)
+        for s in range(len(host_in)):
+            slot = s % self.depth
+            with torch.cuda.stream(self.s_in):
+                if s >= self.depth:  # the step that last read this input buffer is done
+                    self.s_in.wait_event(self.comp_done[slot])
+                self.dev_in[slot].copy_(host_in[s], non_blocking=True)
+                self.in_done[slot].record(self.s_in)
+            main.wait_event(self.in_done[slot])
+            if s >= self.depth:  # the copy out of this output buffer is done
+                main.wait_event(self.out_done[slot])
+            q, k, v, A, L = self._views(slot)
+            if s == 0:
+                self.blk.reset()
+            self.blk.step(q, k, v, A, L, m_updated=None if m_updated is None else m_updated[s])
+            self.comp_done[slot].record(main)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(self.comp_done[slot])
+                host_out[s].copy_(self.dev_out[slot], non_blocking=True)
+                self.out_done[slot].record(self.s_out)
+        main.wait_stream(self.s_in)  # join
+        main.wait_stream(self.s_out)

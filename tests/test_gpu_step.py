@@ -212,3 +212,40 @@ def test_sparse_residual_rejects_more_than_64_rows_per_kv_head():
         blk.step(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L,
                  m_updated=st.m_updated)
     assert e.value.code == fb.FB_ERR_SHAPE
+
+
+@pytest.mark.parametrize("captured", [False, True])
+def test_host_block_pipeline_matches_oracle(captured):
+    """Steps fed from pinned host buffers with overlapped copies (eager, and
+    captured as one CUDA graph per block) return the oracle's A_full / L_full."""
+    from block_diffusion_attention_fb_b200.runtime import HostBlockPipeline
+    from workloads.torch_io import to_torch
+    wl = make_workload("dllm", prefix_min=1200, prefix_max=1200, n_heads_q=4, n_heads_kv=4,
+                       steps=9)
+    sp = wl.spec
+    kv = make_kv(wl.prefix, sp.dtype)
+    blk = BlockAttention(kv, sp.block, sp.n_heads_q, "threshold", tau=2)
+    pipe = HostBlockPipeline(blk, torch.bfloat16, depth=3)
+    steps = list(wl.steps())
+    host_in = [pipe.pack_inputs(to_torch(st.q, sp.dtype, "cpu"), to_torch(st.k_in, sp.dtype, "cpu"),
+                                to_torch(st.v_in, sp.dtype, "cpu")) for st in steps]
+    host_out = [pipe.new_output() for _ in steps]
+    ms = [st.m_updated.tolist() for st in steps]
+    if captured:
+        pipe.enqueue_block(host_in, host_out, ms)  # eager warm-up
+        sync()
+        for o in host_out:
+            o.fill_(7.0)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            pipe.enqueue_block(host_in, host_out, ms)
+        g.replay()
+    else:
+        pipe.enqueue_block(host_in, host_out, ms)
+    sync()
+    ctl = ThresholdController(wl.prefix, sp.dtype, 2)
+    for st, out in zip(steps, host_out):
+        ref = ctl.step(st.step, st.q, st.k_in, st.v_in, st.m_updated)
+        A, L = pipe.unpack_output(out)
+        assert_close_A(A.numpy(), ref["A_full"], sp.dtype, f"step {st.step}")
+        assert_close_L(L.numpy(), ref["L_full"], f"step {st.step}")
