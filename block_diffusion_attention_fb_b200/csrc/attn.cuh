@@ -98,14 +98,28 @@ __device__ __forceinline__ int n_tiles_of(const AttnArgs& a, int b, int hk) {
 
 // Slot of the first token of chunk c of tile tl, and how many of the chunk's
 // tokens are valid (0 => the chunk is loaded out of bounds, i.e. zero-filled).
-__device__ __forceinline__ void chunk_slot(const AttnArgs& a, int b, int hk, int tl, int c,
-                                           long long& slot, int& valid) {
-  const int n_tok = seq_tokens(a, b);
+// Per-(sequence, kv head) values every chunk lookup needs, read once per CTA
+// (a producer would otherwise pay a global load on every tile).
+struct GroupInfo {
+  int n_tok;     // tokens of the sequence
+  int list_cnt;  // entries of the page list (page-list key sets)
+};
+
+__device__ __forceinline__ GroupInfo group_info(const AttnArgs& a, int b, int hk) {
+  GroupInfo g;
+  g.n_tok = seq_tokens(a, b);
+  g.list_cnt = a.page_list ? a.page_count[b * a.Hkv + hk] : 0;
+  return g;
+}
+
+__device__ __forceinline__ void chunk_slot(const AttnArgs& a, const GroupInfo& gi, int b, int hk,
+                                           int tl, int c, long long& slot, int& valid) {
+  const int n_tok = gi.n_tok;
   int t0;
   if (a.page_list) {
     const int per_tile = kTK / a.page_size;
     const int e = tl * per_tile + c;
-    if (e >= a.page_count[b * a.Hkv + hk]) {
+    if (e >= gi.list_cnt) {
       slot = a.n_slots;
       valid = 0;
       return;
@@ -127,6 +141,11 @@ __device__ __forceinline__ void chunk_slot(const AttnArgs& a, int b, int hk, int
   } else {
     slot = (long long)b * a.max_seq_len + t0;
   }
+}
+
+__device__ __forceinline__ void chunk_slot(const AttnArgs& a, int b, int hk, int tl, int c,
+                                           long long& slot, int& valid) {
+  chunk_slot(a, group_info(a, b, hk), b, hk, tl, c, slot, valid);
 }
 
 // Maps row r of (b, hk) to the block row i and q head h.
@@ -387,11 +406,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     // Lane 0 waits for free stages and issues the copies; all lanes fetch the
     // chunk slots of the tile kSlotAhead tiles ahead (one chunk per lane) into
     // a shared ring, so page-list / page-table reads overlap earlier copies.
+    const GroupInfo gi = group_info(a, b, hk);
     auto fill = [&](int it) {  // tile `it` -> ring entry it % kSlotRing (all lanes)
       if (lane < n_chunks) {
         long long s_ = a.n_slots;
         int v_ = 0;
-        chunk_slot(a, b, hk, tile0 + it, lane, s_, v_);
+        chunk_slot(a, gi, b, hk, tile0 + it, lane, s_, v_);
         ring_slot[it % kSlotRing][lane] = (int)s_;
         ring_valid[it % kSlotRing][lane] = v_;
       }

@@ -137,6 +137,7 @@ __global__ void __launch_bounds__(kT2Threads, 1)
     // shared ring, so those reads overlap the copies of the tiles before it.
     constexpr int kC = 2 * kMaxChunks;
     const int nc2 = 2 * n_chunks;  // chunks per 128-key tile
+    const GroupInfo gi = group_info(a, b, hk);
     auto fill = [&](int it) {      // tile `it` -> ring entry it % kSlotRing (all lanes)
       if (lane < nc2) {
         // chunk c covers keys [c * chunk, (c + 1) * chunk) of the 128-key tile; a
@@ -144,7 +145,7 @@ __global__ void __launch_bounds__(kT2Threads, 1)
         const int sub = lane / n_chunks, cc = lane - sub * n_chunks;
         long long s_ = a.n_slots;
         int v_ = 0;
-        if (2 * it + sub < n64) chunk_slot(a, b, hk, tile0 + 2 * it + sub, cc, s_, v_);
+        if (2 * it + sub < n64) chunk_slot(a, gi, b, hk, tile0 + 2 * it + sub, cc, s_, v_);
         ring_slot[it % kSlotRing][lane] = (int)s_;
         ring_valid[it % kSlotRing][lane] = v_;
       }
