@@ -142,28 +142,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair on the FMA pipe (no MUFU), x <= 64. x is clamped to >= -126,
-// split as x = j + f with j = round(x) (added to 1.5 * 2^23, whose low mantissa
-// bits then hold j) and f in [-0.5, 0.5]; 2^f is a degree-3 polynomial whose
-// coefficients are the minimax fit of maximum relative error on that interval
-// (linear program over 4001 points, csrc/fit_exp2_poly.py): max relative
-// error 7.5e-5, against 2^-9 for rounding the result to bf16. The result's
-// exponent field receives j by an integer add.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f, kC3 = 0.05517167f;
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  const float2 t = fadd2(x, make_float2(kMagic, kMagic));
-  const float2 j = fadd2(t, make_float2(-kMagic, -kMagic));
-  const float2 f = ffma2(j, make_float2(-1.f, -1.f), x);
-  float2 p = ffma2(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
-  p = ffma2(p, f, make_float2(kC1, kC1));
-  p = ffma2(p, f, make_float2(kC0, kC0));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
 // Per-warp register budget changes (whole warp, converged): a warp that only
 // issues copies or MMAs gives registers back to the pool; a warp doing the
 // arithmetic takes more. The sum over the CTA must stay within the launch's.
