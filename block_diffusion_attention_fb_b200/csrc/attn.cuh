@@ -298,6 +298,53 @@ __device__ __forceinline__ void combine_row(const AttnArgs& a, int b, int hk, in
   constexpr int D = NV * 32;
   const long long stride = (long long)a.batch * a.Hkv * a.R;  // between splits
   const long long p0 = ((long long)b * a.Hkv + hk) * a.R + r;
+  constexpr int kFast = 16;
+  if (a.n_splits <= kFast) {
+    // Up to 16 splits: every partial and normaliser load is issued before any
+    // of them is used, so a row costs one memory round trip.
+    float v[kFast][NV];
+    const float l = lane < a.n_splits ? __ldcg(a.lse_part + p0 + lane * stride) : -INFINITY;
+#pragma unroll
+    for (int s = 0; s < kFast; ++s) {
+      if (s < a.n_splits) {
+        const float* src = a.o_part + (p0 + (long long)s * stride) * D + lane * NV;
+        if constexpr (NV == 4) {
+          const float4 t = __ldcg(reinterpret_cast<const float4*>(src));
+          v[s][0] = t.x;
+          v[s][1] = t.y;
+          v[s][2] = t.z;
+          v[s][3] = t.w;
+        } else {
+#pragma unroll
+          for (int jj = 0; jj < NV; ++jj) v[s][jj] = __ldcg(src + jj);
+        }
+      }
+    }
+    float M = l;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float bse = (M == -INFINITY) ? 0.f : M;
+    const float wl = l == -INFINITY ? 0.f : fast_exp2(l - bse);
+    float acc[NV], wsum = 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) acc[j] = 0.f;
+#pragma unroll
+    for (int s = 0; s < kFast; ++s) {
+      if (s < a.n_splits) {
+        // empty splits carry weight 0 and zero partials
+        const float w = __shfl_sync(0xffffffffu, wl, s);
+        wsum += w;
+#pragma unroll
+        for (int j = 0; j < NV; ++j) acc[j] += w * v[s][j];
+      }
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) acc[j] *= inv;
+    const float lse2 = wsum > 0.f ? bse + log2f(wsum) : -INFINITY;
+    write_final<NV>(a, b, hk, r, acc, lane * NV, 1, lse2, lane == 0);
+    return;
+  }
   float M = -INFINITY;
   for (int s = lane; s < a.n_splits; s += 32) M = fmaxf(M, __ldcg(a.lse_part + p0 + s * stride));
 #pragma unroll
