@@ -458,6 +458,33 @@ def run_ours(args, rank, world, local):
     t_prefix_kernel = eager(prefix_call, K)
     barrier(world)
     clk = clocks.stop()
+
+    # Quality of the cheap modes against dense attention on the same block
+    # (reported, not asserted: the pages give no number to hold it to). One
+    # untimed block per mode; A_full compared per denoise step.
+    def collect(step_fn):
+        outs = []
+        for s in range(S):
+            step_fn(s)
+            outs.append(A.clone())
+        return outs
+
+    def dense_full(s):
+        prefix_call(s)
+        fb.fb_block_attn(dq[s], dk[s], dv[s], a_in, l_in)
+        fb.fb_merge(a_out, l_out, a_in, l_in, A, L)
+
+    ref_outs = collect(dense_full)
+    quality = {}
+    for qname, fn in (("reuse", reuse_step), ("losa", losa_step),
+                      ("sparse_residual", sres_step if sres is not None else None)):
+        if fn is None:
+            continue
+        outs = collect(fn)
+        diffs = [(o - r).abs() for o, r in zip(outs, ref_outs)]
+        quality[qname] = {"max_abs_vs_dense": round(max(float(x.max()) for x in diffs), 5),
+                          "mean_abs_vs_dense": round(sum(float(x.mean()) for x in diffs) / S, 6)}
+    torch.cuda.synchronize()
     fb.fb_device_status()
 
     n_steps_all = K * S * world
@@ -527,6 +554,7 @@ def run_ours(args, rank, world, local):
             "losa": {"us_per_step": round(us(t_losa_max), 3), "n_active": n_act,
                      "topk_pages": topk},
         },
+        "quality": quality,
         "tokens_per_s": round(world * K * batch * B / (t_reuse_max * 1e-3), 1),
         "roofline": {
             "bound": "tensor" if tensor_bound else "hbm",

@@ -215,3 +215,52 @@ def test_long_context_prefix_partial_sampled():
         a_ref, l_ref = partial(to_f64(st.q[0, rows, h], "bf16"), K, V)
         assert_close_A(A[0, rows, h], a_ref, "bf16", f"head {h}")
         assert_close_L(L[0, rows, h], l_ref, f"head {h}")
+
+
+def test_sparse_residual_full_size_dllm():
+    """FlashBlock + sparse residual over the dllm block (20 % of the 2048 pages per
+    kv head): the selection at every refresh bit-exact, sampled A_full rows within
+    tolerance of the oracle's fresh-sparse + cached-residual merge."""
+    from oracle import residual as ores
+    wl = make_workload("dllm", steps=5)
+    sp = wl.spec
+    kv = make_kv(wl.prefix, sp.dtype)
+    topk = 410
+    blk = BlockAttention(kv, sp.block, sp.n_heads_q, "sparse_residual", tau=sp.tau,
+                         topk_pages=topk)
+    smin, smax = olosa.page_summary(wl.prefix, sp.dtype)
+    samples = _samples(sp, 12, 11)
+    heads = sorted({h for _, _, h in samples})
+    A = torch.zeros(sp.batch, sp.block, sp.n_heads_q, sp.head_dim, device="cuda")
+    L = torch.zeros(sp.batch, sp.block, sp.n_heads_q, device="cuda")
+    res = None
+    for st in wl.steps():
+        blk.step(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L,
+                 m_updated=st.m_updated)
+        sync()
+        refresh = st.step == 0 or int(st.m_updated[0]) >= sp.tau
+        assert blk.recomputed == (1 if refresh else 0)
+        if refresh:  # oracle selection of the sampled heads, bit-exact against the GPU's
+            ul, uc = cpu(blk.t["union_list"]), cpu(blk.t["union_count"])
+            res = {}
+            for h in heads:
+                sc = ores.head_page_scores(wl.prefix, st.q, sp.dtype, 0, h, smin, smax)
+                S_sel = np.sort(olosa.top_indices(sc, topk)).astype(np.int32)
+                assert uc[0, h] == len(S_sel) and np.array_equal(ul[0, h, :len(S_sel)], S_sel)
+                C = np.setdiff1d(np.arange(len(sc), dtype=np.int32), S_sel)
+                res[h] = (S_sel, C, st.q)
+        A_ref, L_ref = [], []
+        for (b, i, h) in samples:
+            S_sel, C, q_ref = res[h]
+            P = wl.prefix.page_size
+            toks = lambda pages: np.asarray([t for p in pages for t in range(p * P, (p + 1) * P)],
+                                            dtype=np.int64)
+            Ks, Vs = oracle.attention.prefix_keys(wl.prefix, 0, h, sp.dtype, tokens=toks(S_sel))
+            Kc, Vc = oracle.attention.prefix_keys(wl.prefix, 0, h, sp.dtype, tokens=toks(C))
+            a_s, l_s = oracle.partial(oracle.to_f64(st.q[0, [i], h], sp.dtype), Ks, Vs)
+            a_c, l_c = oracle.partial(oracle.to_f64(q_ref[0, [i], h], sp.dtype), Kc, Vc)
+            a_o, l_o = oracle.merge(a_s, l_s, a_c, l_c)
+            A_ref.append(a_o[0])
+            L_ref.append(l_o[0])
+        A_full, L_full = _oracle_full_rows(wl, st, samples, np.stack(A_ref), np.array(L_ref))
+        _check_rows(cpu(A), cpu(L), samples, A_full, L_full, sp.dtype, f"step {st.step}")
