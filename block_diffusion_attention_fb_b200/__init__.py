@@ -34,7 +34,8 @@ FB_SPARSE_RESIDUAL = 3
 # Every entry point include/fb.h declares.
 EXPORTS = ("fb_workspace_size", "fb_prefix_attn", "fb_block_attn", "fb_merge", "fb_page_summary",
            "losa_select", "losa_gather", "fb_step", "fb_device_status", "fb_last_error",
-           "fb_kernel_launches", "fb_prefix_attn_noalloc", "fb_block_commit")
+           "fb_kernel_launches", "fb_prefix_attn_noalloc", "fb_block_commit",
+           "fb_selftest_timeout")
 
 
 class FbError(RuntimeError):
@@ -99,6 +100,7 @@ def load_library() -> ctypes.CDLL:
         "fb_kernel_launches": (ctypes.c_uint64, []),
         "fb_prefix_attn_noalloc": (ctypes.c_int, [P, I32, I32, F32, KV, P, P, P, P]),
         "fb_block_commit": (ctypes.c_int, [KV, P, P, P, I32, P, P, P]),
+        "fb_selftest_timeout": (ctypes.c_int, [P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -276,6 +278,11 @@ def fb_block_commit(kv: KV, seq_len_host, k_in, v_in, page_min=None, page_max=No
     _check(load_library().fb_block_commit(
         ctypes.byref(kv.c), lens.ctypes.data_as(ctypes.c_void_p), _ptr(k_in), _ptr(v_in),
         int(k_in.shape[1]), _ptr(page_min), _ptr(page_max), _stream(stream)))
+
+
+def fb_selftest_timeout(gave_up=None, stream=None) -> None:
+    """Launches the failure-path self-test kernel (a wait that must give up)."""
+    _check(load_library().fb_selftest_timeout(_ptr(gave_up), _stream(stream)))
 
 
 def fb_kernel_launches() -> int:

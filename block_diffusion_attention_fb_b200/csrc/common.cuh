@@ -47,13 +47,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Waits for the phase with the given parity; gives up after the budget, sets
 // the error word and *abort, and returns false. Never spins forever.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          long long budget = kWaitBudgetCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitBudgetCycles) {
+    if (clock64() - t0 > budget) {
       *abort = 1;
       atomicExch(&g_fb_error_word, 1);
       return false;
@@ -152,6 +153,23 @@ __device__ __forceinline__ void reg_alloc() {
 template <int N>
 __device__ __forceinline__ void reg_dealloc() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Self-test of the failure path: one CTA waits on an mbarrier that nothing
+// ever arrives at. The bounded wait (the same routine every kernel uses) must
+// give up after `budget` cycles, set the device error word and return, leaving
+// the context usable. No fault, trap or endless loop is involved.
+__global__ void selftest_wait_kernel(long long budget, int* gave_up) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  const bool ok = mbar_wait(&bar, 0, &abort_flag, budget);
+  if (threadIdx.x == 0 && gave_up) *gave_up = ok ? 0 : 1;
 }
 
 constexpr float kLn2 = 0.6931471805599453f;

@@ -686,6 +686,11 @@ int fb_device_status(void) {
   return FB_OK;
 }
 
+int fb_selftest_timeout(int32_t* gave_up, cudaStream_t stream) {
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(2000000LL, gave_up);  // about a millisecond
+  return check_launch("self-test wait kernel");
+}
+
 int fb_block_commit(const fb_kv* kv, const int32_t* seq_len_host, const void* k_in,
                     const void* v_in, int32_t B, void* page_min, void* page_max,
                     cudaStream_t stream) {

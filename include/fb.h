@@ -317,6 +317,16 @@ int fb_block_commit(const fb_kv* kv, const int32_t* seq_len_host, const void* k_
                     cudaStream_t stream);
 
 /*
+ * Self-test of the failure path (no counterpart on the pages): launches one
+ * small kernel whose single wait can never be satisfied (an mbarrier nobody
+ * arrives at). Its bounded wait, the same routine every kernel of this library
+ * uses, gives up after about a millisecond, sets the device error word and
+ * returns; the next fb_device_status() then reports FB_ERR_TIMEOUT and the
+ * context stays usable. gave_up (device int, may be NULL) receives 1.
+ */
+int fb_selftest_timeout(int32_t* gave_up, cudaStream_t stream);
+
+/*
  * Reads and clears the device-side error word that bounded waits set when they
  * give up (SYNCHRONISES the current device). Returns FB_OK, FB_ERR_TIMEOUT, or
  * FB_ERR_ARG when fb_block_commit met a page-table entry outside the pool.

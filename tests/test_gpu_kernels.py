@@ -284,3 +284,26 @@ def test_invalid_arguments_are_rejected_on_the_host():
             fb.fb_block_attn(q, q, q, A, L, scale=bad_scale)
         assert e.value.code == fb.FB_ERR_ARG
     fb.fb_device_status()
+
+
+def test_bounded_wait_gives_up_and_the_context_stays_usable():
+    """A wait that nothing satisfies (an mbarrier nobody arrives at) gives up
+    after its cycle budget, flags FB_ERR_TIMEOUT to the host, and the next
+    attention call on the same context is correct."""
+    fb.fb_device_status()  # start clean
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fb.fb_selftest_timeout(flag)
+    sync()
+    assert int(flag.item()) == 1
+    with pytest.raises(fb.FbError) as e:
+        fb.fb_device_status()
+    assert e.value.code == fb.FB_ERR_TIMEOUT
+    fb.fb_device_status()  # the word was cleared by the read
+    name, ov = PREFIX_CASES["dllm_small_ragged"]
+    wl = make_workload(name, **ov)
+    st = next(wl.steps(1))
+    A, L = run_prefix(wl, st.q)
+    A_ref, L_ref = oracle.prefix_partial(wl.prefix, st.q, wl.spec.dtype)
+    assert_close_A(A, A_ref, wl.spec.dtype)
+    assert_close_L(L, L_ref)
+    fb.fb_device_status()
