@@ -166,7 +166,10 @@ __global__ void __launch_bounds__(256)
 }
 
 // Step 1b: the n_act highest-scoring rows of each sequence, in rank order
-// (score descending, then row ascending). O(B^2) ranks; B is a block size.
+// (score descending, then row ascending). Up to 32 active rows: n_act rounds
+// of a block-wide maximum over the key (order-preserving score bits, ~row), so
+// a higher score wins and equal scores go to the lower row; more active rows:
+// O(B^2) ranks. Scores are sums of squares, never NaN.
 __global__ void __launch_bounds__(256)
     active_rows_kernel(const float* __restrict__ score, int B, int n_act,
                        int32_t* __restrict__ active) {
@@ -174,6 +177,40 @@ __global__ void __launch_bounds__(256)
   const int b = blockIdx.x;
   for (int i = threadIdx.x; i < B; i += blockDim.x) sc[i] = score[(long long)b * B + i];
   __syncthreads();
+  if (n_act <= 32) {
+    __shared__ unsigned long long wbest[8];
+    __shared__ int taken[32];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    for (int r = 0; r < n_act; ++r) {
+      unsigned long long best = 0ull;
+      for (int i = threadIdx.x; i < B; i += blockDim.x) {
+        bool used = false;
+        for (int t = 0; t < r; ++t) used |= (taken[t] == i);
+        if (used) continue;
+        const float f = sc[i] == 0.f ? 0.f : sc[i];  // -0 and +0 rank equal
+        const uint32_t u = __float_as_uint(f);
+        const uint32_t key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+        const unsigned long long k = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)i);
+        best = k > best ? k : best;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+        best = other > best ? other : best;
+      }
+      if (lane == 0) wbest[wid] = best;
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        unsigned long long m = 0ull;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = wbest[w] > m ? wbest[w] : m;
+        const int row = (int)(0xFFFFFFFFu - (uint32_t)(m & 0xFFFFFFFFull));
+        taken[r] = row;
+        active[b * n_act + r] = row;
+      }
+      __syncthreads();
+    }
+    return;
+  }
   for (int i = threadIdx.x; i < B; i += blockDim.x) {
     const float si = sc[i];
     int rank = 0;

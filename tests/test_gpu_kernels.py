@@ -211,6 +211,8 @@ def run_select(wl, q_cur, q_prev, n_active, topk):
     (dict(n_heads_q=4, n_heads_kv=2), 2, 9),
     ({}, 4, 1000),       # top-k larger than the page count: every page
     ({}, 40, 5),         # more active rows than block rows: all rows
+    (dict(block=300), 4, 9),    # more rows than the selection block's threads
+    (dict(block=70), 40, 5),    # more than 32 active rows: the rank path
 ])
 def test_losa_select_is_bit_exact(ov, n_active, topk):
     wl = _losa_small(**ov)
@@ -307,3 +309,19 @@ def test_bounded_wait_gives_up_and_the_context_stays_usable():
     assert_close_A(A, A_ref, wl.spec.dtype)
     assert_close_L(L, L_ref)
     fb.fb_device_status()
+
+
+def test_losa_active_rows_break_ties_by_lower_row():
+    """Rows whose q did not move score exactly 0; the active set takes the moved
+    rows by score, then the lowest-index unmoved rows (LoSA step 1, ties)."""
+    wl = _losa_small(block=40)
+    steps = list(wl.steps(2))
+    q_prev = steps[0].q
+    q_cur = q_prev.copy()
+    q_cur[0, [7, 21, 33]] = steps[1].q[0, [7, 21, 33]]
+    kv, act, rs, *_ = run_select(wl, q_cur, q_prev, 6, 4)
+    score = olosa.locality_score(q_cur, q_prev, "bf16")
+    act_ref = olosa.active_rows(score, 6)
+    np.testing.assert_array_equal(cpu(act)[:, :6], act_ref)
+    assert sorted(act_ref[0, :3].tolist()) == [7, 21, 33]
+    assert act_ref[0, 3:].tolist() == [0, 1, 2]
