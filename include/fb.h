@@ -88,9 +88,9 @@ typedef struct fb_kv {
  * need for these shapes (n_active/topk_pages may be 0 when LoSA is unused).
  * num_sms: SM count the split plan targets (0: query the current device).
  * The split plan may be tuned through the environment (FB_SPLIT_WAVES: waves
- * of resident CTAs for the streaming kernels; FB_TC_SPLITS: splits per row
- * tile of the tcgen05 kernel); query the size under the same environment as
- * the calls that use it.
+ * of resident CTAs for the streaming kernels; FB_LIST_WAVES: the same for
+ * page-list key sets; FB_TC_SPLITS: splits per row tile of the tcgen05
+ * kernel); query the size under the same environment as the calls that use it.
  * Returns 0 on invalid arguments.
  */
 size_t fb_workspace_size(const fb_kv* kv, int32_t block, int32_t n_heads_q, int32_t n_active,
