@@ -518,6 +518,19 @@ KvView kv_view(const fb_kv* kv) {
   return v;
 }
 
+// Page scoring grid: chunks of kPsPages pages per (sequence, kv head), `cpc`
+// consecutive chunks per CTA so that about two CTAs per SM cover the chunks
+// (each CTA's next chunk then loads while it scores the current one).
+dim3 page_score_grid(const KvView& v, int num_sms, int& cpc) {
+  const int chunks = ceil_div(v.max_pages, kPsPages);
+  const long long groups = (long long)v.batch * v.Hkv;
+  const long long slots = 2LL * (num_sms > 0 ? num_sms : 148);
+  cpc = (int)((groups * chunks + slots - 1) / slots);
+  if (cpc < 1) cpc = 1;
+  if (cpc > chunks) cpc = chunks;
+  return dim3(ceil_div(chunks, cpc), v.Hkv, v.batch);
+}
+
 // Short blocks (bf16, B <= 64): the latency-built kernel of block_attn.cuh.
 // Rows per CTA: 16 per warp, 1 to 4 warps, fewer warps while that keeps the
 // grid within two CTAs per SM (more CTAs = more of the block's loads in flight).
@@ -631,9 +644,10 @@ int sr_select(const void* q, int B, int Hq, const void* page_min, const void* pa
   if (v.max_pages > 32768) return fail(FB_ERR_SHAPE, "sparse residual supports <= 32768 pages");
   if (!aligned16(page_min) || !aligned16(page_max))
     return fail(FB_ERR_ALIGN, "page summaries not 16-byte aligned");
-  const dim3 g2(ceil_div(v.max_pages, kPsPages), v.Hkv, kv->batch);
+  int cpc;
+  const dim3 g2 = page_score_grid(v, sm_count(), cpc);
   const int es = (int)elem_size(kv->dtype);
-  const int psm = RQ * D * 4 + 2 * kPsPages * (D + 16 / es) * es;
+  const int psm = RQ * D * 4 + 4 * kPsPages * (D + 16 / es) * es;
   int rc;
 #define FB_HPS(TT, DD)                                                                       \
   do {                                                                                       \
@@ -642,7 +656,7 @@ int sr_select(const void* q, int B, int Hq, const void* page_min, const void* pa
     kfn<<<g2, 256, psm, stream>>>(static_cast<const TT*>(q), B, Hq, G,                       \
                                   static_cast<const TT*>(page_min),                          \
                                   static_cast<const TT*>(page_max), v, head_scores, bitmap,  \
-                                  words);                                                    \
+                                  words, cpc);                                               \
   } while (0)
   if (kv->dtype == FB_BF16) {
     if (D == 128) FB_HPS(__nv_bfloat16, 128); else FB_HPS(__nv_bfloat16, 64);
@@ -910,8 +924,9 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
   active_rows_kernel<<<kv->batch, 256, B * 4, stream>>>(rs, B, na, active_rows);
   rc = check_launch("active rows kernel");
   if (rc) return rc;
-  const dim3 g2(ceil_div(v.max_pages, kPsPages), v.Hkv, kv->batch);
-  const int psm = na * G * D * 4 + 2 * kPsPages * (D + 16 / (int)elem_size(kv->dtype)) *
+  int cpc;
+  const dim3 g2 = page_score_grid(v, num_sms, cpc);
+  const int psm = na * G * D * 4 + 4 * kPsPages * (D + 16 / (int)elem_size(kv->dtype)) *
                                        (int)elem_size(kv->dtype);
   if (kv->dtype == FB_BF16) {
     auto kfn = D == 128 ? page_score_kernel<__nv_bfloat16, 128> : page_score_kernel<__nv_bfloat16, 64>;
@@ -919,14 +934,14 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
     kfn<<<g2, 256, psm, stream>>>(static_cast<const __nv_bfloat16*>(q_cur), active_rows, B, Hq, G,
                                   na, static_cast<const __nv_bfloat16*>(page_min),
                                   static_cast<const __nv_bfloat16*>(page_max), v, page_scores,
-                                  union_bitmap, words);
+                                  union_bitmap, words, cpc);
   } else {
     auto kfn = D == 128 ? page_score_kernel<float, 128> : page_score_kernel<float, 64>;
     if ((rc = set_smem_once((const void*)kfn, psm))) return rc;
     kfn<<<g2, 256, psm, stream>>>(static_cast<const float*>(q_cur), active_rows, B, Hq, G, na,
                                   static_cast<const float*>(page_min),
                                   static_cast<const float*>(page_max), v, page_scores,
-                                  union_bitmap, words);
+                                  union_bitmap, words, cpc);
   }
   rc = check_launch("page score kernel");
   if (rc) return rc;

@@ -223,13 +223,8 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------------------
-// Step 3a: QUEST-style page scores u_p = tree_sum_c max(q_c kmin_c, q_c kmax_c)
-// for every active row a and q head h of kv head hk. A block stages the
-// summaries of kPsPages pages (coalesced) and the active q rows in shared
-// memory; then one thread per (page, row) forms the products and runs the
-// stride-halving tree in registers (level 1 pairs c with c + D/2, ...).
-// scores: [batch, n_act, Hq, max_pages]. Block (0, hk, b) also clears the
-// union bitmap of (b, hk) for the top-k kernel that follows.
+// Page scoring (steps 3a of LoSA and the sparse-residual selector): pages are
+// handled in chunks of kPsPages.
 // ---------------------------------------------------------------------------
 constexpr int kPsPages = 64;
 
@@ -289,53 +284,80 @@ __device__ __forceinline__ float page_bound(const float* qr, const T* mnr, const
   return y[0];
 }
 
+// Stages the summaries of 64-page chunk `chunk` of (b, hk) into one of two
+// shared buffers with cp.async (zero-filled past the sequence's pages).
+template <typename T, int D>
+__device__ __forceinline__ void stage_page_chunk(const T* pmin, const T* pmax, const KvView& kv,
+                                                 int b, int hk, int chunk, int n_pages,
+                                                 T* smn, T* smx) {
+  constexpr int PS = ps_stride<T, D>();
+  constexpr int VE = 16 / (int)sizeof(T);  // elements per 16-byte copy
+  for (int idx = threadIdx.x; idx < kPsPages * (D / VE); idx += blockDim.x) {
+    const int pg = idx / (D / VE), cv = idx - (idx / (D / VE)) * (D / VE);
+    const int p = chunk * kPsPages + pg;
+    const bool ok = p < n_pages;
+    const long long so = (((long long)b * kv.max_pages + (ok ? p : 0)) * kv.Hkv + hk) * D + cv * VE;
+    cp_async16(smem_u32(smn + pg * PS + cv * VE), pmin + so, ok ? 16u : 0u);
+    cp_async16(smem_u32(smx + pg * PS + cv * VE), pmax + so, ok ? 16u : 0u);
+  }
+  cp_async_commit();
+}
+
+// Step 3a: QUEST-style page scores u_p = tree_sum_c max(q_c kmin_c, q_c kmax_c)
+// for every active row a and q head h of kv head hk. A CTA scores `cpc`
+// consecutive chunks of 64 pages of one (b, hk): the active q rows once into
+// shared memory, the summaries chunk by chunk into two buffers with cp.async,
+// the next chunk loading while the current one is scored by one thread per
+// (page, row) (page_bound: single-rounded products, stride-halving tree).
+// scores: [batch, n_act, Hq, max_pages]. Block (0, hk, b) also clears the
+// union bitmap of (b, hk) for the top-k kernel that follows.
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
     page_score_kernel(const T* __restrict__ q, const int32_t* __restrict__ active, int B, int Hq,
                       int G, int n_act, const T* __restrict__ pmin, const T* __restrict__ pmax,
                       const KvView kv, float* __restrict__ scores, uint32_t* __restrict__ bitmap,
-                      int words) {
+                      int words, int cpc) {
   constexpr int PS = ps_stride<T, D>();
-  constexpr int VE = 16 / (int)sizeof(T);  // elements per 16-byte global load
-  extern __shared__ float sm[];
+  extern __shared__ __align__(16) float sm[];
   const int RQ = n_act * G;
-  float* qs = sm;                                   // [RQ][D]
-  T* smn = reinterpret_cast<T*>(qs + RQ * D);       // [kPsPages][PS]
-  T* smx = smn + kPsPages * PS;
+  float* qs = sm;                              // [RQ][D]
+  T* sbuf = reinterpret_cast<T*>(qs + RQ * D);  // 2 x ([kPsPages][PS] min, then max)
   const int hk = blockIdx.y, b = blockIdx.z;
-  const int p0 = blockIdx.x * kPsPages;
   if (blockIdx.x == 0)
     for (int w = threadIdx.x; w < words; w += blockDim.x)
       bitmap[((long long)b * kv.Hkv + hk) * words + w] = 0u;
   const int n_pages = (kv_tokens(kv, b) + kv.page_size - 1) / kv.page_size;
-  if (p0 >= n_pages) return;
+  const int c0 = blockIdx.x * cpc;
+  const int c1 = min(c0 + cpc, (n_pages + kPsPages - 1) / kPsPages);
+  if (c0 >= c1) return;
+  stage_page_chunk<T, D>(pmin, pmax, kv, b, hk, c0, n_pages, sbuf, sbuf + kPsPages * PS);
   for (int idx = threadIdx.x; idx < RQ * D; idx += blockDim.x) {
     const int rq = idx / D, c = idx - (idx / D) * D;
     const int a_i = rq / G, g = rq - (rq / G) * G;
-    const int i = active[b * n_act + a_i];
+    const int i = active ? active[b * n_act + a_i] : a_i;
     qs[idx] = ld_f32<T>(q + (((long long)b * B + i) * Hq + hk * G + g) * D + c);
   }
-  // stage the summaries with 16-byte loads (rows of one head are contiguous)
-  for (int idx = threadIdx.x; idx < kPsPages * (D / VE); idx += blockDim.x) {
-    const int pg = idx / (D / VE), cv = idx - (idx / (D / VE)) * (D / VE);
-    const int p = p0 + pg;
-    uint4 mn = make_uint4(0u, 0u, 0u, 0u), mx = make_uint4(0u, 0u, 0u, 0u);
-    if (p < n_pages) {
-      const long long so = (((long long)b * kv.max_pages + p) * kv.Hkv + hk) * D + cv * VE;
-      mn = *reinterpret_cast<const uint4*>(pmin + so);
-      mx = *reinterpret_cast<const uint4*>(pmax + so);
+  for (int ch = c0; ch < c1; ++ch) {
+    const int buf = (ch - c0) & 1;
+    T* smn = sbuf + buf * 2 * kPsPages * PS;
+    T* smx = smn + kPsPages * PS;
+    if (ch + 1 < c1) {
+      T* nmn = sbuf + (buf ^ 1) * 2 * kPsPages * PS;
+      stage_page_chunk<T, D>(pmin, pmax, kv, b, hk, ch + 1, n_pages, nmn, nmn + kPsPages * PS);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
-    *reinterpret_cast<uint4*>(smn + pg * PS + cv * VE) = mn;
-    *reinterpret_cast<uint4*>(smx + pg * PS + cv * VE) = mx;
-  }
-  __syncthreads();
-  for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
-    const int pg = task % kPsPages, rq = task / kPsPages;
-    const int p = p0 + pg;
-    if (p >= n_pages) continue;
-    const float yb = page_bound<T, D>(qs + rq * D, smn + pg * PS, smx + pg * PS);
-    const int a_i = rq / G, g = rq - (rq / G) * G;
-    scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = yb;
+    __syncthreads();  // chunk ch (and the q rows) visible to every thread
+    for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
+      const int pg = task % kPsPages, rq = task / kPsPages;
+      const int p = ch * kPsPages + pg;
+      if (p >= n_pages) continue;
+      const float yb = page_bound<T, D>(qs + rq * D, smn + pg * PS, smx + pg * PS);
+      const int a_i = rq / G, g = rq - (rq / G) * G;
+      scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = yb;
+    }
+    __syncthreads();  // buffer `buf` is refilled two chunks later
   }
 }
 
@@ -521,53 +543,54 @@ __global__ void __launch_bounds__(256)
     head_page_score_kernel(const T* __restrict__ q, int B, int Hq, int G,
                            const T* __restrict__ pmin, const T* __restrict__ pmax,
                            const KvView kv, float* __restrict__ scores,
-                           uint32_t* __restrict__ bitmap, int words) {
+                           uint32_t* __restrict__ bitmap, int words, int cpc) {
   constexpr int PS = ps_stride<T, D>();
-  constexpr int VE = 16 / (int)sizeof(T);
-  extern __shared__ float sm[];
+  extern __shared__ __align__(16) float sm[];
   __shared__ uint32_t best[kPsPages];
   const int RQ = B * G;
-  float* qs = sm;                              // [RQ][D], row r = i * G + g
-  T* smn = reinterpret_cast<T*>(qs + RQ * D);  // [kPsPages][PS]
-  T* smx = smn + kPsPages * PS;
+  float* qs = sm;                               // [RQ][D], row r = i * G + g
+  T* sbuf = reinterpret_cast<T*>(qs + RQ * D);  // 2 x ([kPsPages][PS] min, then max)
   const int hk = blockIdx.y, b = blockIdx.z;
-  const int p0 = blockIdx.x * kPsPages;
   if (blockIdx.x == 0)
     for (int w = threadIdx.x; w < words; w += blockDim.x)
       bitmap[((long long)b * kv.Hkv + hk) * words + w] = 0u;
   const int n_pages = (kv_tokens(kv, b) + kv.page_size - 1) / kv.page_size;
-  if (p0 >= n_pages) return;
-  for (int pg = threadIdx.x; pg < kPsPages; pg += blockDim.x) best[pg] = 0u;  // below every key
+  const int c0 = blockIdx.x * cpc;
+  const int c1 = min(c0 + cpc, (n_pages + kPsPages - 1) / kPsPages);
+  if (c0 >= c1) return;
+  stage_page_chunk<T, D>(pmin, pmax, kv, b, hk, c0, n_pages, sbuf, sbuf + kPsPages * PS);
   for (int idx = threadIdx.x; idx < RQ * D; idx += blockDim.x) {
     const int rq = idx / D, c = idx - (idx / D) * D;
     const int i = rq / G, g = rq - (rq / G) * G;
     qs[idx] = ld_f32<T>(q + (((long long)b * B + i) * Hq + hk * G + g) * D + c);
   }
-  for (int idx = threadIdx.x; idx < kPsPages * (D / VE); idx += blockDim.x) {
-    const int pg = idx / (D / VE), cv = idx - (idx / (D / VE)) * (D / VE);
-    const int p = p0 + pg;
-    uint4 mn = make_uint4(0u, 0u, 0u, 0u), mx = make_uint4(0u, 0u, 0u, 0u);
-    if (p < n_pages) {
-      const long long so = (((long long)b * kv.max_pages + p) * kv.Hkv + hk) * D + cv * VE;
-      mn = *reinterpret_cast<const uint4*>(pmin + so);
-      mx = *reinterpret_cast<const uint4*>(pmax + so);
+  for (int ch = c0; ch < c1; ++ch) {
+    const int buf = (ch - c0) & 1;
+    T* smn = sbuf + buf * 2 * kPsPages * PS;
+    T* smx = smn + kPsPages * PS;
+    for (int pg = threadIdx.x; pg < kPsPages; pg += blockDim.x) best[pg] = 0u;  // below every key
+    if (ch + 1 < c1) {
+      T* nmn = sbuf + (buf ^ 1) * 2 * kPsPages * PS;
+      stage_page_chunk<T, D>(pmin, pmax, kv, b, hk, ch + 1, n_pages, nmn, nmn + kPsPages * PS);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
-    *reinterpret_cast<uint4*>(smn + pg * PS + cv * VE) = mn;
-    *reinterpret_cast<uint4*>(smx + pg * PS + cv * VE) = mx;
-  }
-  __syncthreads();
-  for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
-    const int pg = task % kPsPages, rq = task / kPsPages;
-    const int p = p0 + pg;
-    if (p >= n_pages) continue;
-    const float yb = page_bound<T, D>(qs + rq * D, smn + pg * PS, smx + pg * PS);
-    atomicMax(&best[pg], order_key(yb));
-  }
-  __syncthreads();
-  for (int pg = threadIdx.x; pg < kPsPages; pg += blockDim.x) {
-    const int p = p0 + pg;
-    if (p < n_pages)
-      scores[((long long)b * kv.Hkv + hk) * kv.max_pages + p] = order_key_inv(best[pg]);
+    __syncthreads();  // chunk ch, the q rows and the cleared maxima visible to every thread
+    for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
+      const int pg = task % kPsPages, rq = task / kPsPages;
+      const int p = ch * kPsPages + pg;
+      if (p >= n_pages) continue;
+      const float yb = page_bound<T, D>(qs + rq * D, smn + pg * PS, smx + pg * PS);
+      atomicMax(&best[pg], order_key(yb));
+    }
+    __syncthreads();
+    for (int pg = threadIdx.x; pg < kPsPages; pg += blockDim.x) {
+      const int p = ch * kPsPages + pg;
+      if (p < n_pages)
+        scores[((long long)b * kv.Hkv + hk) * kv.max_pages + p] = order_key_inv(best[pg]);
+    }
+    __syncthreads();  // maxima read out, buffer `buf` free for chunk ch + 2
   }
 }
 
