@@ -1,7 +1,8 @@
 // C ABI of the block-diffusion attention library (declared in include/fb.h):
 // argument validation, split-KV planning, TMA descriptor creation and kernel
-// launches. Every step of the path runs in the kernels of attn.cuh, losa.cuh
-// and cosine.cuh; this file only decides what to launch.
+// launches. Every step of the path runs in the kernels of attn.cuh,
+// attn_tc2.cuh, block_attn.cuh, commit.cuh, losa.cuh and cosine.cuh; this file
+// only decides what to launch.
 #include <cudaTypedefs.h>
 
 #include <atomic>
@@ -137,11 +138,10 @@ struct Plan {
 };
 
 // Kernel choice for bf16, head_dim 128: the tcgen05 kernel when a kv head has
-// more than 64 stacked query rows (GQA groups, video blocks: its 128-row MMA
-// tiles are full), the mma.sync kernel for up to 64 rows (dLLM blocks: a
-// 128-row tile would be mostly padding and one softmax warpgroup per SM leaves
-// the stream latency-bound; measured dllm prefix 135 us against 191 us).
-// fp32 runs on the CUDA-core kernel.
+// more than 64 stacked query rows (GQA groups, video blocks: its two 128-row
+// Q tiles are mostly full), the mma.sync kernel for up to 64 rows (dLLM
+// blocks: a 128-row MMA tile would be mostly padding while the stream is
+// HBM-bound). fp32 runs on the CUDA-core kernel.
 bool use_tc(fb_dtype dt, int D, int R) { return dt == FB_BF16 && D == 128 && R > 64; }
 
 int tc_splits(long long units, int slots, int max_tiles, int batch) {
