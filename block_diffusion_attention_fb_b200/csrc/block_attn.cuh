@@ -240,4 +240,111 @@ __global__ void __launch_bounds__(128) block_attn_kernel(const __grid_constant__
   }
 }
 
+// ---------------------------------------------------------------------------
+// fp32 inputs (the same short-block role, float32 arithmetic throughout, no
+// tensor cores): one CTA per (sequence, kv head). K (stored transposed, so the
+// lanes of a warp read consecutive keys), V and the stacked Q rows are staged
+// with cp.async in one round trip; warp w takes rows w, w + 8, ...: lane j
+// forms s_j and s_{j+32} by fp32 FMA over the channels, the row maximum and sum
+// come from warp shuffles, and lane j accumulates output channels j, j + 32, ...
+// The FlashBlock merge with the cached partial is fused as in the bf16 kernel.
+// ---------------------------------------------------------------------------
+struct BlockArgsF32 {
+  const float* q;  // [batch, B, Hq, D]
+  const float* k;  // [batch, B, Hkv, D]
+  const float* v;
+  const float* mrg_a;
+  const float* mrg_l;
+  float* a_out;
+  float* l_out;
+  int batch, B, Hq, Hkv, G, R;
+  float scale;
+};
+
+// shared memory of block_attn_f32_kernel for R stacked rows
+constexpr int block_f32_smem(int D, int R) { return 4 * D * (64 + R + 65); }
+
+template <int D>
+__global__ void __launch_bounds__(256) block_attn_f32_kernel(const __grid_constant__ BlockArgsF32 a) {
+  constexpr int NK = 64;       // keys staged (B <= 64)
+  constexpr int KP = NK + 1;   // padded stride of the transposed keys: no bank conflicts
+  extern __shared__ __align__(16) float fsm[];
+  float* vs = fsm;             // [NK][D]
+  float* qs = vs + NK * D;     // [R][D]
+  float* kT = qs + a.R * D;    // [D][KP]
+  const int hk = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+  // V and Q rows by cp.async (16-byte chunks), K through registers into the
+  // transposed layout; keys past the block are zero
+  constexpr int C4 = D / 4;
+  for (int idx = tid; idx < NK * C4; idx += blockDim.x) {
+    const int j = idx / C4, c = idx - j * C4;
+    const bool ok = j < a.B;
+    const long long off = (((long long)b * a.B + (ok ? j : 0)) * a.Hkv + hk) * D + c * 4;
+    cp_async16(smem_u32(vs + j * D + c * 4), a.v + off, ok ? 16u : 0u);
+  }
+  for (int idx = tid; idx < a.R * C4; idx += blockDim.x) {
+    const int r = idx / C4, c = idx - r * C4;
+    const int i = r / a.G, h = hk * a.G + (r - i * a.G);
+    cp_async16(smem_u32(qs + r * D + c * 4), a.q + (((long long)b * a.B + i) * a.Hq + h) * D + c * 4,
+               16u);
+  }
+  cp_async_commit();
+  for (int idx = tid; idx < NK * D; idx += blockDim.x) {
+    const int j = idx / D, c = idx - j * D;
+    kT[c * KP + j] = j < a.B ? a.k[(((long long)b * a.B + j) * a.Hkv + hk) * D + c] : 0.f;
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  constexpr int NV = D / 32;
+  for (int r = warp; r < a.R; r += nw) {
+    const float* qr = qs + r * D;
+    float s0 = 0.f, s1 = 0.f;  // keys lane and lane + 32
+#pragma unroll 8
+    for (int c = 0; c < D; ++c) {
+      const float qc = qr[c];
+      s0 = fmaf(qc, kT[c * KP + lane], s0);
+      s1 = fmaf(qc, kT[c * KP + lane + 32], s1);
+    }
+    s0 = lane < a.B ? s0 * a.scale : -INFINITY;
+    s1 = lane + 32 < a.B ? s1 * a.scale : -INFINITY;
+    float m = fmaxf(s0, s1);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float p0 = expf(s0 - m), p1 = expf(s1 - m);  // the block has >= 1 key: m finite
+    float l = p0 + p1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    float o[NV];
+#pragma unroll
+    for (int t = 0; t < NV; ++t) o[t] = 0.f;
+    for (int j = 0; j < a.B; ++j) {
+      const float pj = __shfl_sync(0xffffffffu, j < 32 ? p0 : p1, j & 31);
+#pragma unroll
+      for (int t = 0; t < NV; ++t) o[t] = fmaf(pj, vs[j * D + lane + 32 * t], o[t]);
+    }
+    const int i = r / a.G, h = hk * a.G + (r - i * a.G);
+    const long long row = ((long long)b * a.B + i) * a.Hq + h;
+    const float Ln = m + logf(l);
+    float wn = 1.f / l, wo = 0.f, L = Ln;
+    if (a.mrg_a) {
+      const float Lo = a.mrg_l[row];
+      const float mm = fmaxf(Lo, Ln);
+      const float eo = expf(Lo - mm), en = expf(Ln - mm);  // Ln finite, so mm is
+      const float inv = 1.f / (eo + en);
+      wn *= en * inv;
+      wo = eo * inv;
+      L = mm + logf(eo + en);
+    }
+#pragma unroll
+    for (int t = 0; t < NV; ++t) {
+      const int col = lane + 32 * t;
+      float x = wn * o[t];
+      if (wo > 0.f) x += wo * a.mrg_a[row * D + col];  // a side with weight 0 is not read
+      a.a_out[row * D + col] = x;
+    }
+    if (lane == 0) a.l_out[row] = L;
+  }
+}
+
 }  // namespace fb

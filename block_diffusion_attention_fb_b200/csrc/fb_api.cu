@@ -590,6 +590,44 @@ int block_attn_short(const void* q, const void* k_in, const void* v_in, int batc
   return check_launch("block attention kernel");
 }
 
+// Short fp32 blocks (B <= 64): one CTA of up to 8 warps per (sequence, kv head).
+int block_attn_short_f32(const void* q, const void* k_in, const void* v_in, int batch, int B,
+                         int Hq, int Hkv, int D, float scale, float* a_out, float* l_out,
+                         const float* mrg_a, const float* mrg_l, cudaStream_t stream) {
+  if (int rc_ = validate_scale(scale)) return rc_;
+  BlockArgsF32 a{};
+  a.q = static_cast<const float*>(q);
+  a.k = static_cast<const float*>(k_in);
+  a.v = static_cast<const float*>(v_in);
+  a.mrg_a = mrg_a;
+  a.mrg_l = mrg_l;
+  a.a_out = a_out;
+  a.l_out = l_out;
+  a.batch = batch;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.R = B * a.G;
+  a.scale = scale;
+  if (batch == 0 || B == 0) return FB_OK;
+  if (batch > 65535) return fail(FB_ERR_SHAPE, "too many sequences");
+  const int warps = a.R < 8 ? a.R : 8;
+  const int smem = block_f32_smem(D, a.R);
+#define FB_BLOCK_F32_LAUNCH(DD)                                          \
+  do {                                                                   \
+    auto kfn = block_attn_f32_kernel<DD>;                                \
+    if (int rc_ = set_smem_once((const void*)kfn, smem)) return rc_;    \
+    kfn<<<dim3(Hkv, batch), 32 * warps, smem, stream>>>(a);              \
+  } while (0)
+  if (D == 128)
+    FB_BLOCK_F32_LAUNCH(128);
+  else
+    FB_BLOCK_F32_LAUNCH(64);
+#undef FB_BLOCK_F32_LAUNCH
+  return check_launch("fp32 block attention kernel");
+}
+
 int block_attn_impl(const void* q, const void* k_in, const void* v_in, int batch, int B, int Hq,
                     int Hkv, int D, float scale, fb_dtype dt, float* a_in, float* l_in,
                     cudaStream_t stream, const float* mrg_a = nullptr,
@@ -612,6 +650,10 @@ int block_attn_impl(const void* q, const void* k_in, const void* v_in, int batch
   if (mrg_a && !mrg_l) return fail(FB_ERR_ARG, "merge partner without its L");
   if (dt == FB_BF16 && (D == 64 || D == 128) && B <= 64) return block_attn_short(
       q, k_in, v_in, batch, B, Hq, Hkv, D, scale, a_in, l_in, mrg_a, mrg_l, stream);
+  if (dt == FB_F32 && (D == 64 || D == 128) && B <= 64 &&
+      block_f32_smem(D, B * (Hq / Hkv)) <= 200 * 1024)
+    return block_attn_short_f32(q, k_in, v_in, batch, B, Hq, Hkv, D, scale, a_in, l_in, mrg_a,
+                                mrg_l, stream);
   PartialCall c{};
   c.q = q;
   c.B = B;

@@ -54,10 +54,11 @@ def test_threshold_steps_match_oracle(name, ov, tau):
         assert n_rec == sp.steps * sp.batch
 
 
-def test_threshold_steps_with_an_empty_prefix_side():
+@pytest.mark.parametrize("name", ["gqa", "tiny"])
+def test_threshold_steps_with_an_empty_prefix_side(name):
     """A sequence with no prefix tokens has L_out = -inf: the fused merge must
     return its in-block partial alone (FlashBlock merge with one empty side)."""
-    wl = make_workload("gqa", prefix_min=20, prefix_max=300, batch=3, block=24, n_heads_q=8,
+    wl = make_workload(name, prefix_min=20, prefix_max=300, batch=3, block=24, n_heads_q=8,
                        n_heads_kv=2, steps=4)
     wl.prefix.seq_len[1] = 0
     sp = wl.spec
