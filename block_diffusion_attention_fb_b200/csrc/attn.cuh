@@ -112,6 +112,15 @@ __device__ __forceinline__ GroupInfo group_info(const AttnArgs& a, int b, int hk
   return g;
 }
 
+// n_tiles_of from the values group_info already read
+__device__ __forceinline__ int n_tiles_of(const AttnArgs& a, const GroupInfo& gi) {
+  if (a.page_list) {
+    const int per_tile = kTK / a.page_size;
+    return (gi.list_cnt + per_tile - 1) / per_tile;
+  }
+  return (gi.n_tok + kTK - 1) / kTK;
+}
+
 __device__ __forceinline__ void chunk_slot(const AttnArgs& a, const GroupInfo& gi, int b, int hk,
                                            int tl, int c, long long& slot, int& valid) {
   const int n_tok = gi.n_tok;
@@ -747,56 +756,82 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 }
 
 // ---------------------------------------------------------------------------
-// fp32 CUDA-core kernel: row tile 16 (4 warps x 4 rows), tiles of kTK keys
-// loaded with plain coalesced loads; lane j of a warp owns key j of a half tile.
+// fp32 CUDA-core kernel: row tile 16 (4 warps x 4 rows), tiles of kTK keys.
+// A tile's K and V arrive by cp.async in one round trip into a two-stage ring
+// (the next tile loads while this one is computed); K rows are padded to
+// D + 4 floats so that lanes reading float4s of different keys hit different
+// banks. Lane j of a warp owns keys j and j + 32 of the tile; the warp's 4 rows
+// share every K load. P goes through shared memory for the PV product.
 // ---------------------------------------------------------------------------
 constexpr int kF32Rows = 16;
 
-template <typename T>
-__device__ __forceinline__ float elem_f32(const T* p, long long i);
-template <>
-__device__ __forceinline__ float elem_f32<float>(const float* p, long long i) {
-  return p[i];
-}
-template <>
-__device__ __forceinline__ float elem_f32<__nv_bfloat16>(const __nv_bfloat16* p, long long i) {
-  return __bfloat162float(p[i]);
-}
+template <int D>
+struct F32Smem {
+  static constexpr int KP = D + 4;
+  static constexpr int bytes =
+      4 * (kF32Rows * D + 2 * kTK * KP + 2 * kTK * D + kF32Rows * kTK);  // Q, K, V, P
+};
 
-// fp32 attention partial (T = float); inputs are read through elem_f32.
-template <typename T, int D>
+template <int D>
 __global__ void __launch_bounds__(128) attn_f32_kernel(const __grid_constant__ AttnArgs a) {
-  constexpr int NV = D / 32;
-  __shared__ float Ks[32][D + 1];  // half a tile; +1: lanes reading different keys hit different banks
-  __shared__ float Vs[32][D];
-  __shared__ float Qs[kF32Rows][D];
-  __shared__ int meta[kMaxChunks];
-  __shared__ long long slots[kMaxChunks];
+  constexpr int NV = D / 32, KP = F32Smem<D>::KP, C4 = D / 4;
+  extern __shared__ __align__(16) float fs[];
+  float* Qs = fs;                   // [kF32Rows][D]
+  float* Ks = Qs + kF32Rows * D;    // [2][kTK][KP]
+  float* Vs = Ks + 2 * kTK * KP;    // [2][kTK][D]
+  float* Ps = Vs + 2 * kTK * D;     // [kF32Rows][kTK]
+  __shared__ long long slots[2][kMaxChunks];
+  __shared__ int meta[2][kMaxChunks];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rt = blockIdx.x % a.n_row_tiles;
   const int split = blockIdx.x / a.n_row_tiles;
   const int hk = blockIdx.y, b = blockIdx.z;
   if (!cta_selected(a, b, hk)) return;
-  const int n_tiles = n_tiles_of(a, b, hk);
+  const GroupInfo gi = group_info(a, b, hk);
+  const int n_tiles = n_tiles_of(a, gi);
   const int tile0 = split * a.tiles_per_split;
   const int n_it = max(0, min(a.tiles_per_split, n_tiles - tile0));
   const int n_chunks = kTK / a.chunk;
-  const T* qf = static_cast<const T*>(a.q);
-  const T* kg = static_cast<const T*>(a.k);
-  const T* vg = static_cast<const T*>(a.v);
+  const float* qf = static_cast<const float*>(a.q);
+  const float* kg = static_cast<const float*>(a.k);
+  const float* vg = static_cast<const float*>(a.v);
 
-  for (int idx = tid; idx < kF32Rows * D; idx += blockDim.x) {
-    const int rl = idx / D, c = idx % D;
+  for (int idx = tid; idx < kF32Rows * C4; idx += blockDim.x) {
+    const int rl = idx / C4, c4 = idx - rl * C4;
     const int r = rt * kF32Rows + rl;
-    float v = 0.f;
     if (r < a.R) {
       int i, h;
       row_of(a, b, hk, r, i, h);
-      v = elem_f32<T>(qf, (((long long)b * a.B + i) * a.Hq + h) * D + c);
+      cp_async16(smem_u32(Qs + rl * D + 4 * c4), qf + (((long long)b * a.B + i) * a.Hq + h) * D + 4 * c4,
+                 16u);
+    } else {
+      *reinterpret_cast<float4*>(Qs + rl * D + 4 * c4) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    Qs[rl][c] = v;
   }
+  cp_async_commit();
+
+  auto fill_meta = [&](int it, int st) {
+    if (tid < n_chunks) {
+      long long sl;
+      int v;
+      chunk_slot(a, gi, b, hk, tile0 + it, tid, sl, v);
+      slots[st][tid] = sl;
+      meta[st][tid] = v;
+    }
+  };
+  // keys outside the key set are zero-filled (and masked below)
+  auto issue = [&](int st) {
+    for (int idx = tid; idx < kTK * C4; idx += blockDim.x) {
+      const int key = idx / C4, c4 = idx - key * C4;
+      const int ci = key / a.chunk, off = key - ci * a.chunk;
+      const bool ok = off < meta[st][ci];
+      const long long e = ok ? ((slots[st][ci] + off) * a.Hkv + hk) * D + 4 * c4 : 0;
+      cp_async16(smem_u32(Ks + (st * kTK + key) * KP + 4 * c4), kg + e, ok ? 16u : 0u);
+      cp_async16(smem_u32(Vs + (st * kTK + key) * D + 4 * c4), vg + e, ok ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
 
   float m_r[4], l_r[4], o[4][NV];
 #pragma unroll
@@ -807,64 +842,88 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const __grid_constant__ A
     for (int j = 0; j < NV; ++j) o[k][j] = 0.f;
   }
 
-  for (int it = 0; it < n_it; ++it) {
+  if (n_it > 0) {
+    fill_meta(0, 0);
     __syncthreads();
-    if (tid < n_chunks) {
-      long long sl;
-      int valid;
-      chunk_slot(a, b, hk, tile0 + it, tid, sl, valid);
-      slots[tid] = sl;
-      meta[tid] = valid;
+    issue(0);
+  }
+  for (int it = 0; it < n_it; ++it) {
+    const int st = it & 1;
+    if (it + 1 < n_it) {
+      fill_meta(it + 1, st ^ 1);
+      __syncthreads();
+      issue(st ^ 1);
+      cp_async_wait<1>();  // Q and this tile have landed
+    } else {
+      cp_async_wait<0>();
     }
     __syncthreads();
-    for (int half = 0; half < kTK / 32; ++half) {
-      if (half) __syncthreads();
-      for (int idx = tid; idx < 32 * D; idx += blockDim.x) {
-        const int kr = idx / D, c = idx - (idx / D) * D;
-        const int key = half * 32 + kr;
-        const int ci = key / a.chunk, off = key - ci * a.chunk;
-        float kv = 0.f, vv = 0.f;
-        if (off < meta[ci]) {  // keys outside the key set stay 0 (and are masked below)
-          const long long e = ((slots[ci] + off) * a.Hkv + hk) * D + c;
-          kv = elem_f32<T>(kg, e);
-          vv = elem_f32<T>(vg, e);
-        }
-        Ks[kr][c] = kv;
-        Vs[kr][c] = vv;
-      }
-      __syncthreads();
-      const int key = half * 32 + lane;
-      const int ci = key / a.chunk;
-      const bool valid = (key - ci * a.chunk) < meta[ci];
+    const float* K = Ks + st * kTK * KP;
+    const float* V = Vs + st * kTK * D;
+    bool valid[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int key = lane + 32 * h, ci = key / a.chunk;
+      valid[h] = key - ci * a.chunk < meta[st][ci];
+    }
+    float s[4][2];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s[k][0] = s[k][1] = 0.f;
+#pragma unroll 4
+    for (int c4 = 0; c4 < C4; ++c4) {
+      const float4 k0 = *reinterpret_cast<const float4*>(K + lane * KP + 4 * c4);
+      const float4 k1 = *reinterpret_cast<const float4*>(K + (lane + 32) * KP + 4 * c4);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const int rl = warp * 4 + k;
-        float s = 0.f;
-#pragma unroll 16
-        for (int c = 0; c < D; ++c) s = fmaf(Qs[rl][c], Ks[lane][c], s);
-        s = valid ? s * a.scale_log2 : -INFINITY;
-        float mx = s;
+        const float4 q = *reinterpret_cast<const float4*>(Qs + (warp * 4 + k) * D + 4 * c4);
+        s[k][0] = fmaf(q.x, k0.x, fmaf(q.y, k0.y, fmaf(q.z, k0.z, fmaf(q.w, k0.w, s[k][0]))));
+        s[k][1] = fmaf(q.x, k1.x, fmaf(q.y, k1.y, fmaf(q.z, k1.z, fmaf(q.w, k1.w, s[k][1]))));
+      }
+    }
+    float* P = Ps + warp * 4 * kTK;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const float mn = fmaxf(m_r[k], mx);
-        const float bse = (mn == -INFINITY) ? 0.f : mn;
-        const float alpha = exp2f(m_r[k] - bse);
-        const float p = exp2f(s - bse);
-        float ps = p;
+    for (int k = 0; k < 4; ++k) {
+      const float s0 = valid[0] ? s[k][0] * a.scale_log2 : -INFINITY;
+      const float s1 = valid[1] ? s[k][1] * a.scale_log2 : -INFINITY;
+      float mx = fmaxf(s0, s1);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
-        l_r[k] = l_r[k] * alpha + ps;
-        m_r[k] = mn;
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      const float mn = fmaxf(m_r[k], mx);
+      const float bse = (mn == -INFINITY) ? 0.f : mn;
+      const float alpha = exp2f(m_r[k] - bse);
+      const float p0 = exp2f(s0 - bse), p1 = exp2f(s1 - bse);
+      float ps = p0 + p1;
 #pragma unroll
-        for (int j = 0; j < NV; ++j) o[k][j] *= alpha;
-        for (int jk = 0; jk < 32; ++jk) {
-          const float pj = __shfl_sync(0xffffffffu, p, jk);
+      for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+      l_r[k] = l_r[k] * alpha + ps;
+      m_r[k] = mn;
 #pragma unroll
-          for (int j = 0; j < NV; ++j) o[k][j] = fmaf(pj, Vs[jk][lane + 32 * j], o[k][j]);
+      for (int j = 0; j < NV; ++j) o[k][j] *= alpha;
+      P[k * kTK + lane] = p0;
+      P[k * kTK + lane + 32] = p1;
+    }
+    __syncwarp();
+#pragma unroll 2
+    for (int jk = 0; jk < kTK; jk += 4) {
+      float4 pk[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) pk[k] = *reinterpret_cast<const float4*>(P + k * kTK + jk);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+          const float vv = V[(jk + u) * D + lane + 32 * j];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float pu = u == 0 ? pk[k].x : (u == 1 ? pk[k].y : (u == 2 ? pk[k].z : pk[k].w));
+            o[k][j] = fmaf(pu, vv, o[k][j]);
+          }
         }
       }
     }
+    __syncthreads();  // stage st, its meta and P are free for the next prefetch
   }
+  if (n_it == 0) cp_async_wait<0>();
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int r = rt * kF32Rows + warp * 4 + k;

@@ -425,10 +425,17 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
   }
   const dim3 grid(p.n_row_tiles * p.n_splits, Hkv, kv->batch);
   if (kv->dtype == FB_F32) {
+#define FB_LAUNCH_F32(DD)                                                         \
+  do {                                                                            \
+    auto kfn = attn_f32_kernel<DD>;                                               \
+    if (int rc_ = set_smem_once((const void*)kfn, F32Smem<DD>::bytes)) return rc_; \
+    kfn<<<grid, 128, F32Smem<DD>::bytes, stream>>>(a);                            \
+  } while (0)
     if (D == 128)
-      attn_f32_kernel<float, 128><<<grid, 128, 0, stream>>>(a);
+      FB_LAUNCH_F32(128);
     else
-      attn_f32_kernel<float, 64><<<grid, 128, 0, stream>>>(a);
+      FB_LAUNCH_F32(64);
+#undef FB_LAUNCH_F32
   } else {
     CUtensorMap tk, tv;
     int rc = make_tmap(&tk, kv->k, D, Hkv, kv->n_slots, a.chunk);

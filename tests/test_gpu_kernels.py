@@ -36,6 +36,12 @@ PREFIX_CASES = {
     # name: (workload, overrides)
     "tiny_full_f32": ("tiny", {}),
     "tiny_ragged_f32": ("tiny", dict(prefix_min=1001, prefix_max=1001, block=13)),
+    # fp32, several tiles per split through the two-stage cp.async ring, ragged tail
+    "tiny_long_f32": ("tiny", dict(prefix_min=20011, prefix_max=20011)),
+    # fp32 paged pool, head_dim 128, GQA stacking over 5 row tiles, varied lengths
+    "tiny_paged_gqa_d128_f32": ("tiny", dict(prefix_min=17, prefix_max=900, batch=3, block=20,
+                                             head_dim=128, n_heads_q=8, n_heads_kv=2,
+                                             paged=True)),
     "dllm_small_ragged": ("dllm", dict(prefix_min=1000, prefix_max=1000, n_heads_q=4,
                                        n_heads_kv=4)),
     "dllm_block16": ("dllm", dict(prefix_min=777, prefix_max=777, block=16, n_heads_q=2,
