@@ -589,6 +589,13 @@ def run_ours(args, rank, world, local):
         },
         "quality": quality,
         "tokens_per_s": round(world * K * batch * B / (t_reuse_max * 1e-3), 1),
+        # context, not a target: the pages' own dense-vs-FlashBlock figures (end to
+        # end in a model, hardware not stated) beside this run's per-step ratio
+        "context": {
+            "dense_over_reuse_attention_time": round(t_dense_max / t_reuse_max, 2),
+            "pages": "FlashBlock vs dense block diffusion: up to 1.6x lower attention time, "
+                     "up to 1.44x token throughput (312 -> 451 tokens/s); hardware not stated",
+        },
         "roofline": {
             "bound": "tensor" if tensor_bound else "hbm",
             "kernel": "fb_prefix_attn (split-KV attention + combine), dense prefix, eager launch",
