@@ -822,6 +822,10 @@ size_t fb_workspace_size(const fb_kv* kv, int32_t block, int32_t n_heads_q, int3
   if (!kv || block <= 0 || n_heads_q <= 0 || kv->n_heads_kv <= 0 || n_heads_q % kv->n_heads_kv ||
       kv->batch <= 0 || kv->max_seq_len < 0 || kv->page_size <= 0)
     return 0;
+  // shapes no call accepts have no workspace size either
+  if ((kv->head_dim != 64 && kv->head_dim != 128) || !pow2(kv->page_size) || kv->page_size < 16 ||
+      (kv->dtype != FB_BF16 && kv->dtype != FB_F32) || n_active < 0 || topk_pages < 0)
+    return 0;
   if (num_sms <= 0) num_sms = sm_count();
   if (num_sms <= 0) return 0;
   return ws_layout(kv, block, n_heads_q, n_active, topk_pages, num_sms).total;
@@ -1217,6 +1221,7 @@ int fb_prefix_attn_noalloc(const void* q, int32_t B, int32_t n_heads_q, float sc
   rc = validate_q(q, B, n_heads_q, kv);
   if (rc) return rc;
   if (!a_out || !l_out) return fail(FB_ERR_ARG, "a_out / l_out is NULL");
+  if ((rc = validate_scale(scale))) return rc;
   const int num_sms = sm_count();
   const int R = B * (n_heads_q / kv->n_heads_kv);
   const size_t need = partial_ws_bytes(kv->dtype, kv->batch, kv->n_heads_kv, R, kv->head_dim,
