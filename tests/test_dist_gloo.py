@@ -58,3 +58,25 @@ def test_reference_arm_other_ranks_exit_without_work():
                        timeout=120)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_collectives_of_our_arm_come_before_the_rank_zero_only_part():
+    """Every rank must take the same collective steps: in run_ours no barrier or
+    max-over-ranks may follow the point where ranks other than 0 return (one
+    there would leave rank 0 waiting for ranks that already left)."""
+    import ast
+    src = open(os.path.join(ROOT, "bench.py")).read()
+    fn = next(n for n in ast.parse(src).body
+              if isinstance(n, ast.FunctionDef) and n.name == "run_ours")
+    split_line = None
+    for node in ast.walk(fn):
+        if (isinstance(node, ast.If) and isinstance(node.test, ast.Compare)
+                and getattr(node.test.left, "id", None) == "rank"
+                and isinstance(node.test.ops[0], ast.NotEq)
+                and any(isinstance(b, ast.Return) for b in node.body)):
+            split_line = node.lineno if split_line is None else min(split_line, node.lineno)
+    assert split_line is not None
+    late = [n.lineno for n in ast.walk(fn)
+            if isinstance(n, ast.Call) and getattr(n.func, "id", None) in ("max_over_ranks", "barrier")
+            and n.lineno > split_line]
+    assert late == [], f"collective calls after the rank-0 split at lines {late}"
