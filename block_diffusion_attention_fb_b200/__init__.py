@@ -239,6 +239,8 @@ def fb_step(policy: fb_policy, cache: fb_cache, q, k_in, v_in, kv: KV, a_full, l
     batch, B, Hq, d = q.shape
     m_arr = None
     if m_updated is not None:
+        if len(m_updated) < kv.batch:  # the library reads one count per sequence
+            raise ValueError(f"m_updated holds {len(m_updated)} counts for {kv.batch} sequences")
         m_arr = (ctypes.c_int32 * len(m_updated))(*[int(x) for x in m_updated])
     _check(load_library().fb_step(ctypes.byref(policy), ctypes.byref(cache), _ptr(q), _ptr(k_in),
                                   _ptr(v_in), B, Hq, ctypes.byref(kv.c), _ptr(page_min),

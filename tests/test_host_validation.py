@@ -221,3 +221,13 @@ def test_workspace_size_covers_the_split_partials_of_a_dllm_prefix(lib):
     # LoSA adds page scores for every active row and head over the prefix's pages
     ws_losa = lib.fb_workspace_size(ctypes.byref(kv), 32, 32, 4, 256, 148)
     assert ws_losa >= ws + 4 * 32 * (32768 // 16) * 4
+
+
+def test_step_binding_rejects_too_few_update_counts():
+    # the library reads m_updated[b] for every sequence b: a short host array is
+    # refused before any pointer is taken
+    import types
+    kv = types.SimpleNamespace(batch=3, c=make_kv())
+    q = torch.zeros(3, 4, 4, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="3 sequences"):
+        fb.fb_step(fb.fb_policy(), fb.fb_cache(), q, q, q, kv, q, m_updated=[1, 2])
