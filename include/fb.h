@@ -62,6 +62,10 @@ typedef enum { FB_F32 = 0, FB_BF16 = 1 } fb_dtype;
  *              is row b * max_seq_len + t.
  *              Paged: token t of sequence b is row
  *                page_table[b][t / page_size] * page_size + t % page_size.
+ *              Entries of pages that hold tokens must lie in
+ *              [0, n_slots / page_size): the read paths trust them (the
+ *              float32 kernels would read outside the pool through a bad
+ *              entry); fb_block_commit checks the entries it writes through.
  *  seq_len     [batch] int32 tokens per sequence (<= max_seq_len), or NULL when
  *              every sequence has max_seq_len tokens.
  *  page_size   tokens per logical page (also the LoSA page granularity).
