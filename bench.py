@@ -61,9 +61,11 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--mode", choices=["all", "reuse", "dense", "losa", "sparse_residual",
-                                      "prefix", "block"],
+                                      "prefix", "block", "losa_step"],
                    default="all",
-                   help="all: the contract line; one mode: time only that mode (for profiling)")
+                   help="all: the contract line; reuse/dense/losa/sparse_residual: time only "
+                   "that mode; prefix/block/losa_step: run only that call eagerly, untimed "
+                   "(for profilers)")
     p.add_argument("--sweep", action="store_true",
                    help="long-context sweep instead of the contract line: dense vs reuse per "
                    "denoise step over prefixes of 32k..800k tokens (one JSON line per length)")
@@ -338,14 +340,16 @@ def run_ours(args, rank, world, local):
         pipe.enqueue_block(host_in, host_out, ms)
 
     K, W = args.steps, args.warmup
-    if args.mode in ("prefix", "block"):  # one call kind only, eager (for profilers)
+    if args.mode in ("prefix", "block", "losa_step"):  # one call kind only, eager (for profilers)
         for _ in range(W + K):
             for s in range(S):
                 flush_l2()
                 if args.mode == "prefix":
                     prefix_call(s)
-                else:
+                elif args.mode == "block":
                     fb.fb_block_attn(dq[s], dk[s], dv[s], a_in, l_in)
+                else:
+                    losa_step(s)
         torch.cuda.synchronize()
         fb.fb_device_status()
         if rank == 0:
