@@ -61,10 +61,10 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--mode", choices=["all", "reuse", "dense", "losa", "sparse_residual",
-                                      "prefix", "block", "losa_step"],
+                                      "prefix", "block", "losa_step", "sr_step"],
                    default="all",
                    help="all: the contract line; reuse/dense/losa/sparse_residual: time only "
-                   "that mode; prefix/block/losa_step: run only that call eagerly, untimed "
+                   "that mode; prefix/block/losa_step/sr_step: run only that call eagerly, untimed "
                    "(for profilers)")
     p.add_argument("--sweep", action="store_true",
                    help="long-context sweep instead of the contract line: dense vs reuse per "
@@ -340,7 +340,10 @@ def run_ours(args, rank, world, local):
         pipe.enqueue_block(host_in, host_out, ms)
 
     K, W = args.steps, args.warmup
-    if args.mode in ("prefix", "block", "losa_step"):  # one call kind only, eager (for profilers)
+    if args.mode in ("prefix", "block", "losa_step", "sr_step"):  # eager, for profilers
+        if args.mode == "sr_step" and sres is None:
+            raise SystemExit("sr_step: the sparse-residual mode takes at most 64 stacked rows "
+                             "per kv head")
         for _ in range(W + K):
             for s in range(S):
                 flush_l2()
@@ -348,8 +351,10 @@ def run_ours(args, rank, world, local):
                     prefix_call(s)
                 elif args.mode == "block":
                     fb.fb_block_attn(dq[s], dk[s], dv[s], a_in, l_in)
-                else:
+                elif args.mode == "losa_step":
                     losa_step(s)
+                else:
+                    sres_step(s)
         torch.cuda.synchronize()
         fb.fb_device_status()
         if rank == 0:
