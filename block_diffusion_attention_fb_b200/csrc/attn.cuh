@@ -146,7 +146,16 @@ __device__ __forceinline__ void chunk_slot(const AttnArgs& a, const GroupInfo& g
   if (a.page_table) {
     const int lp = t0 / a.page_size;
     const int off = t0 - lp * a.page_size;
-    slot = (long long)a.page_table[(long long)b * a.max_pages + lp] * a.page_size + off;
+    const int pg = a.page_table[(long long)b * a.max_pages + lp];
+    if (pg < 0 || ((long long)pg + 1) * a.page_size > a.n_slots) {
+      // an entry outside the pool: the chunk reads as holding no tokens (no
+      // access is made through it) and the error word records it
+      atomicOr(&g_fb_error_word, kErrBadReadPage);
+      slot = a.n_slots;
+      valid = 0;
+      return;
+    }
+    slot = (long long)pg * a.page_size + off;
   } else {
     slot = (long long)b * a.max_seq_len + t0;
   }
@@ -301,7 +310,10 @@ __device__ __forceinline__ void write_final_rows(const AttnArgs& a, int b, int h
 // the final row. One warp, NV contiguous columns per lane. The normalisers of
 // 32 splits are read at once (one per lane) and their weights broadcast by
 // shuffle, so the partial loads of a chunk are independent of each other.
-// Empty splits (lse = -inf) have weight 0 and all-zero partials.
+// Every split writes its partial and normaliser, an empty one zeros and -inf;
+// a split of weight exactly 0 is left out of the sum rather than multiplied by
+// 0, so no value it holds (a NaN left in reused scratch included) reaches the
+// row, while a NaN weight still propagates.
 template <int NV>
 __device__ __forceinline__ void combine_row(const AttnArgs& a, int b, int hk, int r, int lane) {
   constexpr int D = NV * 32;
@@ -340,11 +352,12 @@ __device__ __forceinline__ void combine_row(const AttnArgs& a, int b, int hk, in
 #pragma unroll
     for (int s = 0; s < kFast; ++s) {
       if (s < a.n_splits) {
-        // empty splits carry weight 0 and zero partials
         const float w = __shfl_sync(0xffffffffu, wl, s);
         wsum += w;
+        if (w != 0.f) {
 #pragma unroll
-        for (int j = 0; j < NV; ++j) acc[j] += w * v[s][j];
+          for (int j = 0; j < NV; ++j) acc[j] += w * v[s][j];
+        }
       }
     }
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
@@ -370,19 +383,20 @@ __device__ __forceinline__ void combine_row(const AttnArgs& a, int b, int hk, in
     const int n = min(32, a.n_splits - s0);
 #pragma unroll 8
     for (int j = 0; j < n; ++j) {
-      // empty splits carry weight 0 and zero partials, so every load is issued
       const float w = __shfl_sync(0xffffffffu, wl, j);
       wsum += w;
-      const float* src = a.o_part + (p0 + (long long)(s0 + j) * stride) * D + lane * NV;
-      if constexpr (NV == 4) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
-        acc[0] += w * v.x;
-        acc[1] += w * v.y;
-        acc[2] += w * v.z;
-        acc[3] += w * v.w;
-      } else {
+      if (w != 0.f) {
+        const float* src = a.o_part + (p0 + (long long)(s0 + j) * stride) * D + lane * NV;
+        if constexpr (NV == 4) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
+          acc[0] += w * v.x;
+          acc[1] += w * v.y;
+          acc[2] += w * v.z;
+          acc[3] += w * v.w;
+        } else {
 #pragma unroll
-        for (int jj = 0; jj < NV; ++jj) acc[jj] += w * __ldcg(src + jj);
+          for (int jj = 0; jj < NV; ++jj) acc[jj] += w * __ldcg(src + jj);
+        }
       }
     }
   }

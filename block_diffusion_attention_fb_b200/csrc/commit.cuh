@@ -38,9 +38,8 @@ struct CommitArgs {
   int n_old[kMaxCommitBatch];  // lengths before the call
 };
 
-// Error-word bit set when a page-table entry points outside the pool (the
-// page is then left unwritten); fb_device_status reports it.
-constexpr int kErrBadPage = 2;
+// A page-table entry outside the pool sets kErrBadPage (common.cuh) and the
+// page is left unwritten; fb_device_status reports it.
 
 template <typename T>
 __device__ __forceinline__ float commit_f32(T x);

@@ -9,8 +9,11 @@
 
 namespace fb {
 
-// Error word set by any bounded wait that gives up (read by fb_device_status).
+// Error word read (and cleared) by fb_device_status; bits are OR-ed in.
 __device__ int g_fb_error_word;
+constexpr int kErrTimeout = 1;      // a bounded wait gave up
+constexpr int kErrBadPage = 2;      // block commit: page-table entry outside the pool
+constexpr int kErrBadReadPage = 4;  // a read path met a page-table entry outside the pool
 
 // Budget of a bounded wait: about one second at B200 clocks.
 constexpr long long kWaitBudgetCycles = 2000000000LL;
@@ -56,7 +59,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (*abort) return false;
     if (clock64() - t0 > budget) {
       *abort = 1;
-      atomicExch(&g_fb_error_word, 1);
+      atomicOr(&g_fb_error_word, kErrTimeout);
       return false;
     }
   }

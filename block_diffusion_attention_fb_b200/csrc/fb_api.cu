@@ -516,6 +516,7 @@ KvView kv_view(const fb_kv* kv) {
   v.k = kv->k;
   v.page_table = kv->page_table;
   v.seq_len = kv->seq_len;
+  v.n_slots = kv->n_slots;
   v.batch = kv->batch;
   v.Hkv = kv->n_heads_kv;
   v.D = kv->head_dim;
@@ -745,6 +746,9 @@ int fb_device_status(void) {
   if (word & kErrBadPage)
     return fail(FB_ERR_ARG, "fb_block_commit met a page-table entry outside the pool (that page "
                             "was left unwritten)");
+  if (word & kErrBadReadPage)
+    return fail(FB_ERR_ARG, "a page-table entry outside the pool was read (its tokens were "
+                            "treated as absent)");
   if (word) return fail(FB_ERR_TIMEOUT, "a device-side wait exceeded its budget");
   return FB_OK;
 }
@@ -1192,24 +1196,59 @@ int fb_step(const fb_policy* policy, fb_cache* cache, const void* q, const void*
   return FB_OK;
 }
 
-// Device address of g_fb_noalloc_scratch on the current device, looked up on
-// the first call made with that device current and remembered afterwards.
+// Unique id of the calling thread's current context (false if none is current
+// or the driver has no id query). A context created after cudaDeviceReset may
+// reuse the handle of the one it replaced, so the id, not the handle, tells
+// whether a remembered device address still belongs to the live context.
+static bool current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_fb_noalloc_scratch on the current device. It is looked up
+// with cudaGetSymbolAddress on the first call made with that device current and
+// remembered together with the context it belongs to; a call that finds another
+// context current (the device was reset and the module loaded again) looks it
+// up afresh instead of handing a stale address to the kernels.
 static int noalloc_scratch(void** out) {
+  struct Entry {
+    void* addr;
+    unsigned long long ctx;
+  };
   static std::mutex mu;
-  static void* addr[256] = {};
+  static Entry seen[256] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256)
     return fail(FB_ERR_CUDA, "fb_prefix_attn_noalloc: no current device");
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  unsigned long long ctx = 0;
+  const bool have_ctx = current_context_id(&ctx);
+  if (!seen[dev].addr || !have_ctx || seen[dev].ctx != ctx) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_fb_noalloc_scratch);
     if (e != cudaSuccess || !p)
       return fail(FB_ERR_CUDA, "fb_prefix_attn_noalloc: cudaGetSymbolAddress failed: %s",
                   cudaGetErrorString(e));
-    addr[dev] = p;
+    // the lookup made the device's context current on this thread if it was not
+    seen[dev].addr = p;
+    seen[dev].ctx = current_context_id(&ctx) ? ctx : 0;
   }
-  *out = addr[dev];
+  *out = seen[dev].addr;
   return FB_OK;
 }
 
@@ -1234,8 +1273,9 @@ int fb_prefix_attn_noalloc(const void* q, int32_t B, int32_t n_heads_q, float sc
   void* scratch = nullptr;
   rc = noalloc_scratch(&scratch);
   if (rc) return rc;
-  // Nothing in the scratch has to start at zero: every split writes its partial
-  // (or an empty-partial marker) before the combine reads it.
+  // Nothing in the scratch has to start at zero: every split of every row writes
+  // its partial and normaliser (an empty split: zeros and -inf) before the
+  // combine reads them, and the combine gives an empty split no weight.
   PartialCall c{};
   c.q = q;
   c.B = B;

@@ -37,6 +37,7 @@ struct KvView {
   const void* k;
   const int32_t* page_table;
   const int32_t* seq_len;
+  long long n_slots;
   int batch, Hkv, D, page_size, max_pages, max_seq_len;
 };
 
@@ -44,11 +45,17 @@ __device__ __forceinline__ int kv_tokens(const KvView& kv, int b) {
   return kv.seq_len ? kv.seq_len[b] : kv.max_seq_len;
 }
 
+// Pool row of token t of sequence b, or -1 when the page-table entry lies
+// outside the pool (the error word then records it; no access is made).
 __device__ __forceinline__ long long kv_slot(const KvView& kv, int b, int t) {
   if (kv.page_table) {
     const int lp = t / kv.page_size;
-    return (long long)kv.page_table[(long long)b * kv.max_pages + lp] * kv.page_size +
-           (t - lp * kv.page_size);
+    const int pg = kv.page_table[(long long)b * kv.max_pages + lp];
+    if (pg < 0 || ((long long)pg + 1) * kv.page_size > kv.n_slots) {
+      atomicOr(&g_fb_error_word, kErrBadReadPage);
+      return -1;
+    }
+    return (long long)pg * kv.page_size + (t - lp * kv.page_size);
   }
   return (long long)b * kv.max_seq_len + t;
 }
@@ -80,7 +87,9 @@ __global__ void __launch_bounds__(256)
     mx[j] = -INFINITY;
   }
   for (int t = t0; t < t1; ++t) {
-    const T* row = kg + (kv_slot(kv, b, t) * kv.Hkv + hk) * D;
+    const long long slot = kv_slot(kv, b, t);
+    if (slot < 0) continue;
+    const T* row = kg + (slot * kv.Hkv + hk) * D;
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
       const float x = ld_f32<T>(row + lane + 32 * j);

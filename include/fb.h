@@ -63,9 +63,11 @@ typedef enum { FB_F32 = 0, FB_BF16 = 1 } fb_dtype;
  *              Paged: token t of sequence b is row
  *                page_table[b][t / page_size] * page_size + t % page_size.
  *              Entries of pages that hold tokens must lie in
- *              [0, n_slots / page_size): the read paths trust them (the
- *              float32 kernels would read outside the pool through a bad
- *              entry); fb_block_commit checks the entries it writes through.
+ *              [0, n_slots / page_size). Every kernel that reads through the
+ *              table checks the entry first: a page outside the pool is
+ *              treated as holding no tokens (nothing is read through it) and
+ *              the next fb_device_status() returns FB_ERR_ARG; fb_block_commit
+ *              leaves such a page unwritten and reports it the same way.
  *  seq_len     [batch] int32 tokens per sequence (<= max_seq_len), or NULL when
  *              every sequence has max_seq_len tokens.
  *  page_size   tokens per logical page (also the LoSA page granularity).
@@ -132,7 +134,10 @@ int fb_prefix_attn(const void* q, int32_t B, int32_t n_heads_q, float scale, con
  *    holds until the process exits; shapes whose split plan needs more return
  *    FB_ERR_WORKSPACE with the required size in fb_last_error();
  *  - the array's device address is looked up on the first call made with a
- *    given device current; make that first call before any stream capture;
+ *    given device current and remembered with that device's context; make that
+ *    first call before any stream capture. After cudaDeviceReset the next call
+ *    sees a new context and looks the address up again (also a first call in
+ *    this sense);
  *  - all calls share the one array, so calls that overlap on the GPU (other
  *    streams, other host threads) race and must be serialised by the caller;
  *  - nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
@@ -333,7 +338,8 @@ int fb_selftest_timeout(int32_t* gave_up, cudaStream_t stream);
 /*
  * Reads and clears the device-side error word that bounded waits set when they
  * give up (SYNCHRONISES the current device). Returns FB_OK, FB_ERR_TIMEOUT, or
- * FB_ERR_ARG when fb_block_commit met a page-table entry outside the pool.
+ * FB_ERR_ARG when a kernel met a page-table entry outside the pool (a read
+ * path, or fb_block_commit).
  */
 int fb_device_status(void);
 

@@ -3,7 +3,9 @@ outputs the oracle computes row by row; integer decisions are checked whole.
 
 The sampled rows are fixed by a seed and span the first and last block rows,
 every kv head and, for GQA, every sequence. Steps run through fb_step (or
-fb_prefix_attn for the dense partial), exactly as bench.py calls them.
+fb_prefix_attn for the dense partial), exactly as bench.py calls them, over
+every denoise step of the block; the prefix is frozen, so the float64 keys of
+each sampled (sequence, kv head) are converted once per test.
 """
 
 import numpy as np
@@ -30,6 +32,66 @@ def _samples(sp, n, seed):
         out.add((int(rng.integers(sp.batch)), int(rng.integers(sp.block)),
                  int(rng.integers(sp.n_heads_q))))
     return sorted(out)
+
+
+def _grouped_samples(sp, groups, rows_per_group, seed):
+    """Sampled (b, i, h) rows from a few (sequence, kv head) groups: the first
+    and the last group always, then `groups - 2` more (every sequence first)."""
+    rng = np.random.default_rng(seed)
+    G = sp.n_heads_q // sp.n_heads_kv
+    chosen = [(0, 0), (sp.batch - 1, sp.n_heads_kv - 1)]
+    for b in range(sp.batch):
+        if len(chosen) >= groups:
+            break
+        g = (b, int(rng.integers(sp.n_heads_kv)))
+        if g not in chosen:
+            chosen.append(g)
+    while len(chosen) < groups:
+        g = (int(rng.integers(sp.batch)), int(rng.integers(sp.n_heads_kv)))
+        if g not in chosen:
+            chosen.append(g)
+    out = set()
+    for (b, hk) in chosen:
+        rows = [0, sp.block - 1] + [int(x) for x in rng.integers(sp.block, size=rows_per_group)]
+        for i in rows[:rows_per_group]:
+            out.add((b, i, hk * G + int(rng.integers(G))))
+    return sorted(out)
+
+
+class SampledOracle:
+    """Oracle partials of sampled rows. Each sampled (sequence, kv head)'s
+    prefix keys and values are converted to float64 once: the prefix is frozen
+    for the whole block."""
+
+    def __init__(self, prefix, dtype, samples, G):
+        self.dtype, self.G = dtype, G
+        self.kv = {}
+        for (b, _, h) in samples:
+            key = (b, h // G)
+            if key not in self.kv:
+                self.kv[key] = oracle.attention.prefix_keys(prefix, b, h // G, dtype)
+
+    def prefix_rows(self, q, samples):
+        A = np.zeros((len(samples), q.shape[-1]))
+        L = np.zeros(len(samples))
+        for n, (b, i, h) in enumerate(samples):
+            K, V = self.kv[(b, h // self.G)]
+            a, l = oracle.partial(oracle.to_f64(q[b, i, h][None], self.dtype), K, V)
+            A[n], L[n] = a[0], l[0]
+        return A, L
+
+    def full_rows(self, st, samples, A_out_rows, L_out_rows):
+        """A_full of the sampled rows: the cached prefix rows merged with the
+        sampled rows' block partials."""
+        ai = np.zeros_like(A_out_rows)
+        li = np.zeros_like(L_out_rows)
+        for n, (b, i, h) in enumerate(samples):
+            hk = h // self.G
+            a, l = oracle.partial(oracle.to_f64(st.q[b, i, h][None], self.dtype),
+                                  oracle.to_f64(st.k_in[b, :, hk], self.dtype),
+                                  oracle.to_f64(st.v_in[b, :, hk], self.dtype))
+            ai[n], li[n] = a[0], l[0]
+        return oracle.merge(A_out_rows, L_out_rows, ai, li)
 
 
 def _check_rows(A, L, samples, A_ref, L_ref, dtype, what):
@@ -67,58 +129,61 @@ def test_dense_prefix_partial_full_size(name):
     _check_rows(A, L, samples, A_ref, L_ref, sp.dtype, name)
 
 
-@pytest.mark.parametrize("name,n_steps", [("dllm", 32), ("gqa", 10)])
-def test_threshold_block_full_size(name, n_steps):
-    """tau controller over the block's steps: per-sequence decisions exact,
-    sampled A_full within tolerance (oracle rows cached at recompute steps)."""
+@pytest.mark.parametrize("name", ["dllm", "gqa"])
+def test_threshold_block_full_size(name):
+    """tau controller over every step of the block: per-sequence decisions
+    exact, sampled A_full within tolerance (oracle rows cached at recompute
+    steps, as the controller caches them)."""
     wl = make_workload(name)
     sp = wl.spec
     kv = make_kv(wl.prefix, sp.dtype)
     blk = BlockAttention(kv, sp.block, sp.n_heads_q, "threshold", tau=sp.tau)
-    samples = _samples(sp, 24, 11)
+    samples = _grouped_samples(sp, min(sp.batch * sp.n_heads_kv, 8), 3, 11)
+    orc = SampledOracle(wl.prefix, sp.dtype, samples, sp.n_heads_q // sp.n_heads_kv)
     A = torch.zeros(sp.batch, sp.block, sp.n_heads_q, sp.head_dim, device="cuda")
     L = torch.zeros(sp.batch, sp.block, sp.n_heads_q, device="cuda")
-    A_out_rows = L_out_rows = None
-    for st in wl.steps(n_steps):
+    A_out_rows = np.full((len(samples), sp.head_dim), np.nan)
+    L_out_rows = np.full(len(samples), np.nan)
+    n_steps = 0
+    for st in wl.steps():
         blk.step(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L,
                  m_updated=st.m_updated)
         sync()
         rec = [st.step == 0 or int(m) >= sp.tau for m in st.m_updated]
         assert blk.recomputed == sum(rec)
-        fresh = [s for s in samples if rec[s[0]]]
+        fresh = [n for n, s in enumerate(samples) if rec[s[0]]]
         if fresh:
-            a, l = oracle.prefix_partial_samples(wl.prefix, st.q, sp.dtype, fresh)
-            if A_out_rows is None:
-                A_out_rows = np.zeros((len(samples), sp.head_dim))
-                L_out_rows = np.zeros(len(samples))
-            for k, s in enumerate(fresh):
-                j = samples.index(s)
-                A_out_rows[j], L_out_rows[j] = a[k], l[k]
-        A_ref, L_ref = _oracle_full_rows(wl, st, samples, A_out_rows, L_out_rows)
+            a, l = orc.prefix_rows(st.q, [samples[n] for n in fresh])
+            A_out_rows[fresh], L_out_rows[fresh] = a, l
+        A_ref, L_ref = orc.full_rows(st, samples, A_out_rows, L_out_rows)
         _check_rows(cpu(A), cpu(L), samples, A_ref, L_ref, sp.dtype, f"{name} step {st.step}")
+        n_steps += 1
+    assert n_steps == sp.steps
 
 
 def test_per_head_video_full_size():
-    """gamma controller at full video size: the GPU's cosine equals the oracle's
-    cosine on the GPU's own tiles bit for bit, masks follow it, and sampled
-    A_full rows match the oracle with the GPU's decisions (teacher forcing)."""
+    """gamma controller over all 50 steps at full video size: the GPU's cosine
+    equals the oracle's cosine on the GPU's own tiles bit for bit, masks follow
+    it, and sampled A_full rows match the oracle with the GPU's decisions
+    (teacher forcing)."""
     wl = make_workload("video")
     sp = wl.spec
     kv = make_kv(wl.prefix, sp.dtype)
     blk = BlockAttention(kv, sp.block, sp.n_heads_q, "per_head", gamma=sp.gamma)
-    samples = _samples(sp, 24, 13)
+    samples = _grouped_samples(sp, 6, 4, 13)
+    orc = SampledOracle(wl.prefix, sp.dtype, samples, 1)
     A = torch.zeros(sp.batch, sp.block, sp.n_heads_q, sp.head_dim, device="cuda")
     L = torch.zeros(sp.batch, sp.block, sp.n_heads_q, device="cuda")
-    A_out_rows = np.zeros((len(samples), sp.head_dim))
-    L_out_rows = np.zeros(len(samples))
-    reused = 0
-    for st in wl.steps(6):
+    A_out_rows = np.full((len(samples), sp.head_dim), np.nan)
+    L_out_rows = np.full(len(samples), np.nan)
+    reused = n_steps = 0
+    for st in wl.steps():
         mask = cpu(blk.t["head_mask"]).astype(bool)
         blk.step(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L)
         sync()
-        cur, prev = cpu(blk.a_out), cpu(blk.t["a_out_prev"])
         nxt = cpu(blk.t["head_mask"]).astype(bool)
-        if st.step >= 1:
+        if st.step >= 1 and mask.any():
+            cur, prev = cpu(blk.a_out), cpu(blk.t["a_out_prev"])
             cos = cpu(blk.t["head_cos"])
             for h in range(sp.n_heads_q):
                 if mask[0, h]:
@@ -127,21 +192,24 @@ def test_per_head_video_full_size():
                     assert nxt[0, h] == (c < sp.gamma)
                 else:
                     assert not nxt[0, h]
+        elif st.step >= 1:
+            assert not nxt.any()
         reused += int((~mask).sum())
-        fresh = [s for s in samples if mask[s[0], s[2]]]
+        fresh = [n for n, s in enumerate(samples) if mask[s[0], s[2]]]
         if fresh:
-            a, l = oracle.prefix_partial_samples(wl.prefix, st.q, sp.dtype, fresh)
-            for k, s in enumerate(fresh):
-                j = samples.index(s)
-                A_out_rows[j], L_out_rows[j] = a[k], l[k]
-        A_ref, L_ref = _oracle_full_rows(wl, st, samples, A_out_rows, L_out_rows)
+            a, l = orc.prefix_rows(st.q, [samples[n] for n in fresh])
+            A_out_rows[fresh], L_out_rows[fresh] = a, l
+        A_ref, L_ref = orc.full_rows(st, samples, A_out_rows, L_out_rows)
         _check_rows(cpu(A), cpu(L), samples, A_ref, L_ref, sp.dtype, f"video step {st.step}")
-    assert reused > 0, "at gamma = 0.95 some heads reuse within the first steps"
+        n_steps += 1
+    assert n_steps == sp.steps
+    assert reused > 0, "at gamma = 0.95 some heads reuse within the block"
 
 
 def test_losa_full_size():
-    """LoSA at full size: step 0 dense; later steps' active rows and page unions
-    equal the oracle's exactly, and the refreshed rows match its sparse partial."""
+    """LoSA over all 32 steps at full size: step 0 dense; every later step's
+    active rows and page unions equal the oracle's exactly, and the refreshed
+    rows match its sparse partial."""
     wl = make_workload("losa")
     sp = wl.spec
     kv = make_kv(wl.prefix, sp.dtype)
@@ -152,27 +220,28 @@ def test_losa_full_size():
     gmax = cpu(blk.page_max.float())
     np.testing.assert_array_equal(gmin[0], smin[0])
     np.testing.assert_array_equal(gmax[0], smax[0])
-    samples = _samples(sp, 16, 17)
+    samples = _grouped_samples(sp, 4, 4, 17)
+    orc = SampledOracle(wl.prefix, sp.dtype, samples, 1)
     A = torch.zeros(sp.batch, sp.block, sp.n_heads_q, sp.head_dim, device="cuda")
     L = torch.zeros(sp.batch, sp.block, sp.n_heads_q, device="cuda")
     q_prev = None
     A_out_rows = L_out_rows = None
-    for st in wl.steps(4):
+    n_steps = 0
+    for st in wl.steps():
         blk.step(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L)
         sync()
         if st.step == 0:
-            A_out_rows, L_out_rows = oracle.prefix_partial_samples(wl.prefix, st.q, sp.dtype,
-                                                                   samples)
+            A_out_rows, L_out_rows = orc.prefix_rows(st.q, samples)
         else:
             score = olosa.locality_score(st.q, q_prev, sp.dtype)
             act = olosa.active_rows(score, sp.n_active)
             np.testing.assert_array_equal(cpu(blk.t["active_rows"]), act)
             _, union = olosa.select_pages(wl.prefix, st.q, sp.dtype, act, sp.topk_pages, smin,
                                           smax)
+            ul, uc = cpu(blk.t["union_list"]), cpu(blk.t["union_count"])
             for (b, hk), pages in union.items():
-                cnt = int(cpu(blk.t["union_count"])[b, hk])
-                assert cnt == len(pages)
-                np.testing.assert_array_equal(cpu(blk.t["union_list"])[b, hk, :cnt], pages)
+                assert int(uc[b, hk]) == len(pages)
+                np.testing.assert_array_equal(ul[b, hk, :len(pages)], pages)
             fresh = olosa.sparse_partial(wl.prefix, st.q, sp.dtype, act, union)
             a_gpu, l_gpu = cpu(blk.a_out), cpu(blk.l_out)
             keys = list(fresh)
@@ -183,9 +252,11 @@ def test_losa_full_size():
             for j, s in enumerate(samples):
                 if s in fresh:
                     A_out_rows[j], L_out_rows[j] = fresh[s]
-        A_ref, L_ref = _oracle_full_rows(wl, st, samples, A_out_rows, L_out_rows)
+        A_ref, L_ref = orc.full_rows(st, samples, A_out_rows, L_out_rows)
         _check_rows(cpu(A), cpu(L), samples, A_ref, L_ref, sp.dtype, f"losa step {st.step}")
         q_prev = st.q
+        n_steps += 1
+    assert n_steps == sp.steps
 
 
 def test_long_context_prefix_partial_sampled():

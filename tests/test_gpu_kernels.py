@@ -340,3 +340,64 @@ def test_losa_active_rows_break_ties_by_lower_row():
     np.testing.assert_array_equal(cpu(act)[:, :6], act_ref)
     assert sorted(act_ref[0, :3].tolist()) == [7, 21, 33]
     assert act_ref[0, 3:].tolist() == [0, 1, 2]
+
+
+@pytest.mark.parametrize("name,ov", [
+    # bf16 (TMA producer) and fp32 (cp.async) read paths; GQA rows over 64 take the
+    # tcgen05 kernel
+    ("gqa", dict(prefix_min=300, prefix_max=700, batch=2, block=12, n_heads_q=8, n_heads_kv=2)),
+    ("gqa", dict(prefix_min=300, prefix_max=700, batch=2, block=24, n_heads_q=8, n_heads_kv=2)),
+    ("tiny", dict(prefix_min=300, prefix_max=700, batch=2, block=12, head_dim=128,
+                  n_heads_q=8, n_heads_kv=2, paged=True)),
+])
+def test_page_table_entries_outside_the_pool_read_as_absent(name, ov):
+    """A page-table entry outside the pool (past its end, or negative) is
+    checked before any access: its tokens count as absent, the result equals
+    the partial over the remaining tokens, and fb_device_status reports
+    FB_ERR_ARG. The page summary skips the same pages."""
+    wl = make_workload(name, steps=1, **ov)
+    sp = wl.spec
+    pre = wl.prefix
+    n_pool_pages = pre.k.shape[0] // pre.page_size
+    kv = make_kv(pre, sp.dtype)
+    bad = {(0, 1): n_pool_pages + 3, (1, 0): -2}  # (sequence, logical page) -> bad entry
+    for (b, p), e in bad.items():
+        kv.page_table[b, p] = e
+    st = next(wl.steps(1))
+    A = torch.full((sp.batch, sp.block, sp.n_heads_q, sp.head_dim), 7.0, device="cuda")
+    L = torch.full((sp.batch, sp.block, sp.n_heads_q), 7.0, device="cuda")
+    ws = torch.empty(fb.fb_workspace_size(kv, sp.block, sp.n_heads_q), dtype=torch.uint8,
+                     device="cuda")
+    fb.fb_prefix_attn(dev(st.q, sp.dtype), kv, A, L, ws)
+    sync()
+    with pytest.raises(fb.FbError) as e:
+        fb.fb_device_status()
+    assert e.value.code == fb.FB_ERR_ARG
+    fb.fb_device_status()  # the word was cleared
+    A, L = cpu(A), cpu(L)
+    G = sp.n_heads_q // sp.n_heads_kv
+    P = pre.page_size
+    for b in range(sp.batch):
+        keep = [t for t in range(int(pre.seq_len[b])) if (b, t // P) not in bad]
+        for hk in range(sp.n_heads_kv):
+            K, V = oracle.attention.prefix_keys(pre, b, hk, sp.dtype, tokens=keep)
+            for g in range(G):
+                h = hk * G + g
+                a, l = oracle.partial(oracle.to_f64(st.q[b, :, h], sp.dtype), K, V)
+                assert_close_A(A[b, :, h], a, sp.dtype, f"b{b} h{h}")
+                assert_close_L(L[b, :, h], l, f"b{b} h{h}")
+    if sp.dtype == "bf16":
+        pmin = torch.empty(sp.batch, kv.n_pages, sp.n_heads_kv, sp.head_dim, dtype=torch.bfloat16,
+                           device="cuda")
+        pmax = torch.empty_like(pmin)
+        fb.fb_page_summary(kv, pmin, pmax)
+        sync()
+        with pytest.raises(fb.FbError):
+            fb.fb_device_status()
+        smin, smax = olosa.page_summary(pre, sp.dtype)
+        gmin, gmax = cpu(pmin.float()), cpu(pmax.float())
+        for b in range(sp.batch):
+            for p in range(-(-int(pre.seq_len[b]) // P)):
+                if (b, p) not in bad:
+                    np.testing.assert_array_equal(gmin[b, p], smin[b, p])
+                    np.testing.assert_array_equal(gmax[b, p], smax[b, p])

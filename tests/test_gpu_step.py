@@ -136,12 +136,28 @@ def test_per_head_oracle_mask_agrees_away_from_the_threshold():
                     assert (cos_gpu[0, h] >= gamma) == (ref["cos"][0, h] >= gamma)
 
 
-@pytest.mark.parametrize("ov,n_active,topk", [
-    (dict(prefix_min=3000, prefix_max=3000, n_heads_q=4, n_heads_kv=4, steps=6), 4, 16),
-    (dict(prefix_min=2500, prefix_max=2500, n_heads_q=4, n_heads_kv=2, steps=5, block=20), 3, 9),
+@pytest.mark.parametrize("name,ov,n_active,topk", [
+    ("losa", dict(prefix_min=3000, prefix_max=3000, n_heads_q=4, n_heads_kv=4, steps=6), 4, 16),
+    ("losa", dict(prefix_min=2500, prefix_max=2500, n_heads_q=4, n_heads_kv=2, steps=5,
+                  block=20), 3, 9),
+    # paged pool, pages permuted, ragged lengths, batch 3, GQA (G = 4): per-sequence
+    # active sets and per-(sequence, kv head) unions in one launch
+    ("gqa", dict(prefix_min=700, prefix_max=3100, batch=3, block=16, n_heads_q=8, n_heads_kv=2,
+                 steps=5), 4, 12),
+    # 20 active rows x 4 q heads = 80 stacked rows per kv head: the tcgen05
+    # kernel over page lists
+    ("gqa", dict(prefix_min=1500, prefix_max=4000, batch=2, block=32, n_heads_q=8, n_heads_kv=2,
+                 steps=4), 20, 8),
+    # video block (200 of its 1560 rows, reduced prefix): per-head drift, long block
+    # (in-block partial on the tcgen05 kernel), 8 active rows on the mma.sync kernel
+    ("video", dict(prefix_min=2000, prefix_max=2000, block=200, n_heads_q=4, n_heads_kv=4,
+                   steps=4), 8, 10),
+    # 70 active rows of the video block: the tcgen05 kernel over page lists
+    ("video", dict(prefix_min=1800, prefix_max=1800, block=200, n_heads_q=2, n_heads_kv=2,
+                   steps=3), 70, 6),
 ])
-def test_losa_steps_match_oracle(ov, n_active, topk):
-    wl = make_workload("losa", **ov)
+def test_losa_steps_match_oracle(name, ov, n_active, topk):
+    wl = make_workload(name, **ov)
     sp = wl.spec
     kv = make_kv(wl.prefix, sp.dtype)
     blk = BlockAttention(kv, sp.block, sp.n_heads_q, "losa", n_active=n_active, topk_pages=topk)
