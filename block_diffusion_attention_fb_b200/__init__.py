@@ -35,7 +35,8 @@ FB_SPARSE_RESIDUAL = 3
 EXPORTS = ("fb_workspace_size", "fb_prefix_attn", "fb_block_attn", "fb_merge", "fb_page_summary",
            "losa_select", "losa_gather", "fb_step", "fb_device_status", "fb_last_error",
            "fb_kernel_launches", "fb_prefix_attn_noalloc", "fb_block_commit",
-           "fb_selftest_timeout")
+           "fb_selftest_timeout", "fb_prefix_attn_varlen", "fb_block_attn_varlen",
+           "fb_step_varlen")
 
 
 class FbError(RuntimeError):
@@ -101,6 +102,11 @@ def load_library() -> ctypes.CDLL:
         "fb_prefix_attn_noalloc": (ctypes.c_int, [P, I32, I32, F32, KV, P, P, P, P]),
         "fb_block_commit": (ctypes.c_int, [KV, P, P, P, I32, P, P, P]),
         "fb_selftest_timeout": (ctypes.c_int, [P, P]),
+        "fb_prefix_attn_varlen": (ctypes.c_int, [P, P, I32, I32, I32, F32, KV, P, P, P, SZ, P]),
+        "fb_block_attn_varlen": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, I32, F32,
+                                                ctypes.c_int, P, P, P]),
+        "fb_step_varlen": (ctypes.c_int, [ctypes.POINTER(fb_policy), ctypes.POINTER(fb_cache), P, P,
+                                          P, P, I32, I32, I32, KV, P, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -237,17 +243,57 @@ def fb_step(policy: fb_policy, cache: fb_cache, q, k_in, v_in, kv: KV, a_full, l
             m_updated: Optional[Sequence[int]] = None, page_min=None, page_max=None,
             workspace=None, stream=None) -> None:
     batch, B, Hq, d = q.shape
-    m_arr = None
-    if m_updated is not None:
-        if len(m_updated) < kv.batch:  # the library reads one count per sequence
-            raise ValueError(f"m_updated holds {len(m_updated)} counts for {kv.batch} sequences")
-        m_arr = (ctypes.c_int32 * len(m_updated))(*[int(x) for x in m_updated])
+    m_arr = _m_array(m_updated, kv.batch)
     _check(load_library().fb_step(ctypes.byref(policy), ctypes.byref(cache), _ptr(q), _ptr(k_in),
                                   _ptr(v_in), B, Hq, ctypes.byref(kv.c), _ptr(page_min),
                                   _ptr(page_max),
                                   ctypes.cast(m_arr, ctypes.c_void_p) if m_arr is not None else None,
                                   _ptr(a_full), _ptr(l_full), _ptr(workspace),
                                   workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def _m_array(m_updated, batch):
+    if m_updated is None:
+        return None
+    if len(m_updated) < batch:  # the library reads one count per sequence
+        raise ValueError(f"m_updated holds {len(m_updated)} counts for {batch} sequences")
+    return (ctypes.c_int32 * len(m_updated))(*[int(x) for x in m_updated])
+
+
+def fb_prefix_attn_varlen(q, cu_rows, max_rows: int, kv: KV, a_out, l_out, workspace,
+                          scale: float = 1.0, stream=None) -> None:
+    """Packed rows q [total, Hq, d]; cu_rows: device int32 [batch + 1] offsets;
+    max_rows: the most rows any sequence has (host)."""
+    total, Hq, d = q.shape
+    _check(load_library().fb_prefix_attn_varlen(_ptr(q), _ptr(cu_rows), max_rows, total, Hq, scale,
+                                                ctypes.byref(kv.c), _ptr(a_out), _ptr(l_out),
+                                                _ptr(workspace),
+                                                workspace.numel() * workspace.element_size(),
+                                                _stream(stream)))
+
+
+def fb_block_attn_varlen(q, k_in, v_in, cu_rows, max_rows: int, a_in, l_in, scale: float = 1.0,
+                         stream=None) -> None:
+    total, Hq, d = q.shape
+    batch = int(cu_rows.shape[0]) - 1
+    _check(load_library().fb_block_attn_varlen(_ptr(q), _ptr(k_in), _ptr(v_in), _ptr(cu_rows),
+                                               batch, max_rows, total, Hq, int(k_in.shape[1]), d,
+                                               scale, _dtype_code(q), _ptr(a_in), _ptr(l_in),
+                                               _stream(stream)))
+
+
+def fb_step_varlen(policy: fb_policy, cache: fb_cache, q, k_in, v_in, cu_rows, max_rows: int,
+                   kv: KV, a_full, l_full=None, m_updated: Optional[Sequence[int]] = None,
+                   workspace=None, stream=None) -> None:
+    total, Hq, d = q.shape
+    m_arr = _m_array(m_updated, kv.batch)
+    _check(load_library().fb_step_varlen(ctypes.byref(policy), ctypes.byref(cache), _ptr(q),
+                                         _ptr(k_in), _ptr(v_in), _ptr(cu_rows), max_rows, total,
+                                         Hq, ctypes.byref(kv.c),
+                                         ctypes.cast(m_arr, ctypes.c_void_p) if m_arr is not None
+                                         else None, _ptr(a_full), _ptr(l_full), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(),
+                                         _stream(stream)))
 
 
 def fb_device_status() -> None:

@@ -32,10 +32,17 @@ constexpr int kSlotAhead = 3;  // tiles whose chunk slots a producer fetches ahe
 constexpr int kSlotRing = kSlotAhead + 1;
 
 struct AttnArgs {
-  const void* q;  // [batch, B, Hq, D]
+  const void* q;  // [batch, B, Hq, D], or [q_total, Hq, D] packed (q_cu)
   const void* k;  // [n_slots, Hkv, D] (f32 path; the bf16 path reads through TMA)
   const void* v;
-  int batch, B, Hq, Hkv, G;
+  int batch, B, Hq, Hkv, G;  // B: rows per sequence (packed rows: the most any sequence has)
+  // Packed (variable-length) rows: sequence b's query rows are rows
+  // q_cu[b] .. q_cu[b+1]-1 of q and of the outputs; NULL: rows b * B + i.
+  const int32_t* q_cu;
+  int q_total;  // rows of the packed buffers
+  // Packed contiguous key set (a varlen block's own keys): sequence b's tokens
+  // are rows kv_cu[b] .. kv_cu[b+1]-1 of k / v; NULL: the cache layout below.
+  const int32_t* kv_cu;
   const int32_t* row_list;  // [batch, n_list] block rows taking part, or NULL (all B)
   int n_list;
   int R;  // rows per (b, hk): (row_list ? n_list : B) * G; row r = i_idx * G + g
@@ -68,7 +75,24 @@ struct AttnArgs {
 };
 
 __device__ __forceinline__ int seq_tokens(const AttnArgs& a, int b) {
+  if (a.kv_cu) {
+    long long t0;
+    return packed_range(a.kv_cu, b, (int)a.n_slots, a.max_seq_len, t0);
+  }
   return a.seq_len ? a.seq_len[b] : a.max_seq_len;
+}
+
+// First output row of sequence b and its stacked row count (block rows x G).
+__device__ __forceinline__ long long q_row0(const AttnArgs& a, int b) {
+  if (!a.q_cu) return (long long)b * a.B;
+  long long r0;
+  packed_range(a.q_cu, b, a.q_total, a.B, r0);
+  return r0;
+}
+__device__ __forceinline__ int rows_of(const AttnArgs& a, int b) {
+  if (!a.q_cu) return a.R;
+  long long r0;
+  return packed_range(a.q_cu, b, a.q_total, a.B, r0) * a.G;
 }
 
 __device__ __forceinline__ bool cta_selected(const AttnArgs& a, int b, int hk) {
@@ -101,13 +125,18 @@ __device__ __forceinline__ int n_tiles_of(const AttnArgs& a, int b, int hk) {
 // Per-(sequence, kv head) values every chunk lookup needs, read once per CTA
 // (a producer would otherwise pay a global load on every tile).
 struct GroupInfo {
-  int n_tok;     // tokens of the sequence
-  int list_cnt;  // entries of the page list (page-list key sets)
+  int n_tok;       // tokens of the sequence
+  int list_cnt;    // entries of the page list (page-list key sets)
+  long long base;  // contiguous key sets: pool row of the sequence's first token
 };
 
 __device__ __forceinline__ GroupInfo group_info(const AttnArgs& a, int b, int hk) {
   GroupInfo g;
-  g.n_tok = seq_tokens(a, b);
+  g.base = (long long)b * a.max_seq_len;
+  if (a.kv_cu)
+    g.n_tok = packed_range(a.kv_cu, b, (int)a.n_slots, a.max_seq_len, g.base);
+  else
+    g.n_tok = a.seq_len ? a.seq_len[b] : a.max_seq_len;
   g.list_cnt = a.page_list ? a.page_count[b * a.Hkv + hk] : 0;
   return g;
 }
@@ -157,7 +186,7 @@ __device__ __forceinline__ void chunk_slot(const AttnArgs& a, const GroupInfo& g
     }
     slot = (long long)pg * a.page_size + off;
   } else {
-    slot = (long long)b * a.max_seq_len + t0;
+    slot = gi.base + t0;
   }
 }
 
@@ -185,7 +214,7 @@ __device__ __forceinline__ void write_final(const AttnArgs& a, int b, int hk, in
   int i, h;
   row_of(a, b, hk, r, i, h);
   if (!row_selected(a, b, h)) return;
-  const long long row = ((long long)b * a.B + i) * a.Hq + h;
+  const long long row = (q_row0(a, b) + i) * a.Hq + h;
   constexpr int D = NV * 32;
   float* dst = a.a_out + row * D;
   const float Ln = lse2 * kLn2;
@@ -255,7 +284,7 @@ __device__ __forceinline__ void write_final_rows(const AttnArgs& a, int b, int h
       int i, h;
       row_of(a, b, hk, r[k], i, h);
       ok[k] = row_selected(a, b, h);
-      row[k] = ((long long)b * a.B + i) * a.Hq + h;
+      row[k] = (q_row0(a, b) + i) * a.Hq + h;
     }
   }
 #pragma unroll
@@ -449,6 +478,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   const int split = blockIdx.x / a.n_row_tiles;
   const int hk = blockIdx.y, b = blockIdx.z;
   if (!cta_selected(a, b, hk)) return;
+  const int Rb = rows_of(a, b);  // stacked rows of this sequence
+  if (rt * a.row_tile >= Rb) return;
 
   const int n_tiles = n_tiles_of(a, b, hk);
   const int tile0 = split * a.tiles_per_split;
@@ -560,10 +591,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
       const int r = row_base + g8 + hr * 8;
-      if (r < a.R) {
+      if (r < Rb) {
         int i, h;
         row_of(a, b, hk, r, i, h);
-        rowp[hr] = qb + (((long long)b * a.B + i) * a.Hq + h) * D;
+        rowp[hr] = qb + ((q_row0(a, b) + i) * a.Hq + h) * D;
       }
     }
 #pragma unroll
@@ -736,7 +767,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     for (int k = 0; k < RB; ++k) {
       const int rl = rl0 + k * kNWC;
       const int r = rt * a.row_tile + rl;
-      rr_[k] = (rl < RG * 16 && r < a.R) ? r : -1;
+      rr_[k] = (rl < RG * 16 && r < Rb) ? r : -1;
       const int rgi = (rl >> 4) < RG ? (rl >> 4) : RG - 1, rr = rl & 15;
       float M = -INFINITY;
 #pragma unroll
@@ -802,6 +833,8 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const __grid_constant__ A
   const int split = blockIdx.x / a.n_row_tiles;
   const int hk = blockIdx.y, b = blockIdx.z;
   if (!cta_selected(a, b, hk)) return;
+  const int Rb = rows_of(a, b);  // stacked rows of this sequence
+  if (rt * a.row_tile >= Rb) return;
   const GroupInfo gi = group_info(a, b, hk);
   const int n_tiles = n_tiles_of(a, gi);
   const int tile0 = split * a.tiles_per_split;
@@ -814,10 +847,10 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const __grid_constant__ A
   for (int idx = tid; idx < kF32Rows * C4; idx += blockDim.x) {
     const int rl = idx / C4, c4 = idx - rl * C4;
     const int r = rt * kF32Rows + rl;
-    if (r < a.R) {
+    if (r < Rb) {
       int i, h;
       row_of(a, b, hk, r, i, h);
-      cp_async16(smem_u32(Qs + rl * D + 4 * c4), qf + (((long long)b * a.B + i) * a.Hq + h) * D + 4 * c4,
+      cp_async16(smem_u32(Qs + rl * D + 4 * c4), qf + ((q_row0(a, b) + i) * a.Hq + h) * D + 4 * c4,
                  16u);
     } else {
       *reinterpret_cast<float4*>(Qs + rl * D + 4 * c4) = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -941,7 +974,7 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const __grid_constant__ A
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int r = rt * kF32Rows + warp * 4 + k;
-    if (r >= a.R) break;
+    if (r >= Rb) break;
     const float inv = l_r[k] > 0.f ? 1.f / l_r[k] : 0.f;
     float val[NV];
 #pragma unroll
@@ -953,8 +986,8 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const __grid_constant__ A
 
 // ---------------------------------------------------------------------------
 // Split-KV combine: one warp per row of (b, hk); same log-space rule as the
-// FlashBlock merge, over n_splits partials. Empty partials (lse = -inf) are
-// skipped, so their (never written) outputs are never read.
+// FlashBlock merge, over n_splits partials (an empty split has weight 0 and
+// is left out of the sum).
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ AttnArgs a) {
@@ -969,6 +1002,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ At
   const int r = warp % a.R;
   const int hk = (warp / a.R) % a.Hkv;
   const int b = warp / (a.R * a.Hkv);
+  if (r >= rows_of(a, b)) return;  // packed rows: past this sequence's count
   int i, h;
   row_of(a, b, hk, r, i, h);
   if (!row_selected(a, b, h)) return;

@@ -89,12 +89,14 @@ __global__ void __launch_bounds__(kT2Threads, 1)
   const int split = blockIdx.x / a.n_row_tiles;
   const int hk = blockIdx.y, b = blockIdx.z;
   if (!cta_selected(a, b, hk)) return;
+  const int Rb = rows_of(a, b);  // stacked rows of this sequence
+  if (rt * kT2Rows >= Rb) return;
   // key range of this split in 64-key sub-tiles (tiles_per_split is even)
   const int n64 = max(0, min(a.tiles_per_split, n_tiles_of(a, b, hk) - split * a.tiles_per_split));
   const int tile0 = split * a.tiles_per_split;
   const int n_it = (n64 + 1) >> 1;  // 128-key tiles
   const int n_chunks = kTK / a.chunk;  // metadata chunks per 64-key sub-tile
-  const bool has_b = a.R - rt * kT2Rows > kT2TileRows;
+  const bool has_b = Rb - rt * kT2Rows > kT2TileRows;
 
   const uint32_t base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
   uint8_t* base_ptr = dyn_smem + (base - smem_u32(dyn_smem));
@@ -285,11 +287,11 @@ __global__ void __launch_bounds__(kT2Threads, 1)
     const int r = rt * kT2Rows + x * kT2TileRows + trow;
     {  // this row of Q into shared memory, 128-byte swizzled, K-major
       const uint4* src = nullptr;
-      if (r < a.R) {
+      if (r < Rb) {
         int i, h;
         row_of(a, b, hk, r, i, h);
         src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
-                                             (((long long)b * a.B + i) * a.Hq + h) * D);
+                                             ((q_row0(a, b) + i) * a.Hq + h) * D);
       }
       uint4 qv[16];
 #pragma unroll
@@ -430,13 +432,13 @@ __global__ void __launch_bounds__(kT2Threads, 1)
     const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
     const float lse2 = l_sum > 0.f ? m_used + log2f(l_sum) : -INFINITY;
     long long row = -1;
-    bool write = r < a.R;
+    bool write = r < Rb;
     float wn = 1.f, wo = 0.f, Lfin = lse2 * kLn2;
     if (write && a.n_splits <= 1) {
       int i, h;
       row_of(a, b, hk, r, i, h);
       write = row_selected(a, b, h);
-      row = ((long long)b * a.B + i) * a.Hq + h;
+      row = (q_row0(a, b) + i) * a.Hq + h;
       if (write && a.mrg_a) {
         const float Lo = a.mrg_l[row];
         const float m = fmaxf(Lo, Lfin);

@@ -27,16 +27,28 @@
 namespace fb {
 
 struct BlockArgs {
-  const __nv_bfloat16* q;  // [batch, B, Hq, D]
-  const __nv_bfloat16* k;  // [batch, B, Hkv, D]
+  const __nv_bfloat16* q;  // [batch, B, Hq, D], or [total, Hq, D] packed (cu)
+  const __nv_bfloat16* k;  // [batch, B, Hkv, D], or [total, Hkv, D] packed
   const __nv_bfloat16* v;
+  const int32_t* cu;       // packed rows: sequence b owns rows cu[b] .. cu[b+1]-1, or NULL
+  int total;               // rows of the packed buffers
   const float* mrg_a;  // [batch, B, Hq, D] cached block-external partial, or NULL (no merge)
   const float* mrg_l;  // [batch, B, Hq]
   float* a_out;        // [batch, B, Hq, D]: A_in, or A_full with the merge
   float* l_out;        // [batch, B, Hq]: natural log
-  int batch, B, Hq, Hkv, G, R;  // R = B * G rows per (sequence, kv head)
+  int batch, B, Hq, Hkv, G, R;  // R = B * G rows per (sequence, kv head); packed: B = most rows
   float scale_log2;
 };
+
+// First row and row count of sequence b (packed or batched layout).
+template <typename Args>
+__device__ __forceinline__ int block_rows(const Args& a, int b, long long& base) {
+  if (!a.cu) {
+    base = (long long)b * a.B;
+    return a.B;
+  }
+  return packed_range(a.cu, b, a.total, a.B, base);
+}
 
 template <int D>
 struct BlockSmem {
@@ -62,6 +74,9 @@ __global__ void __launch_bounds__(128) block_attn_kernel(const __grid_constant__
   const int rt = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int row0 = rt * RT;
   const bool merge = a.mrg_a != nullptr;
+  long long base;
+  const int Bb = block_rows(a, b, base);  // block rows (= keys) of this sequence
+  const int Rb = Bb * a.G;
 
   const uint32_t sQ = smem_u32(smem);
   const uint32_t sK = sQ + RT * S::kRowB;
@@ -76,17 +91,17 @@ __global__ void __launch_bounds__(128) block_attn_kernel(const __grid_constant__
     const int r = row0 + rl;
     const __nv_bfloat16* src = a.q;
     uint32_t nb = 0;
-    if (r < a.R) {
+    if (r < Rb) {
       const int i = r / a.G, h = hk * a.G + (r - i * a.G);
-      src = a.q + (((long long)b * a.B + i) * a.Hq + h) * D + c * 8;
+      src = a.q + ((base + i) * a.Hq + h) * D + c * 8;
       nb = 16;
     }
     cp_async16(sQ + rl * S::kRowB + c * 16, src, nb);
   }
   for (int idx = tid; idx < NK * C8; idx += nthr) {
     const int j = idx / C8, c = idx - j * C8;
-    const long long off = (((long long)b * a.B + j) * a.Hkv + hk) * D + c * 8;
-    const bool ok = j < a.B;  // keys past the block are zero-filled (and masked below)
+    const long long off = ((base + j) * a.Hkv + hk) * D + c * 8;
+    const bool ok = j < Bb;  // keys past the block are zero-filled (and masked below)
     cp_async16(sK + j * S::kRowB + c * 16, ok ? a.k + off : a.k, ok ? 16u : 0u);
     cp_async16(sV + j * S::kRowB + c * 16, ok ? a.v + off : a.v, ok ? 16u : 0u);
   }
@@ -100,9 +115,9 @@ __global__ void __launch_bounds__(128) block_attn_kernel(const __grid_constant__
       const int r = row0 + rl;
       const float* src = a.mrg_a;
       uint32_t nb = 0;
-      if (r < a.R) {
+      if (r < Rb) {
         const int i = r / a.G, h = hk * a.G + (r - i * a.G);
-        src = a.mrg_a + (((long long)b * a.B + i) * a.Hq + h) * D + c * 4;
+        src = a.mrg_a + ((base + i) * a.Hq + h) * D + c * 4;
         nb = 16;
       }
       cp_async16(sM + rl * S::kRowM + c * 16, src, nb);
@@ -118,16 +133,16 @@ __global__ void __launch_bounds__(128) block_attn_kernel(const __grid_constant__
 #pragma unroll
   for (int hr = 0; hr < 2; ++hr) {
     const int r = wrow0 + g8 + hr * 8;
-    if (r < a.R) {
+    if (r < Rb) {
       const int i = r / a.G, h = hk * a.G + (r - i * a.G);
-      grow[hr] = ((long long)b * a.B + i) * a.Hq + h;
+      grow[hr] = (base + i) * a.Hq + h;
       if (merge) Lo[hr] = __ldg(a.mrg_l + grow[hr]);
     }
   }
 
   cp_async_wait<1>();  // Q, K, V of this thread landed
   __syncthreads();     // ... and every other thread's
-  if (wrow0 >= a.R) {
+  if (wrow0 >= Rb) {
     cp_async_wait<0>();  // no copy of this thread outlives it
     return;
   }
@@ -158,7 +173,7 @@ __global__ void __launch_bounds__(128) block_attn_kernel(const __grid_constant__
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int key = n * 8 + 2 * t4 + (e & 1);
-      const float x = key < a.B ? s[n][e] * a.scale_log2 : -INFINITY;
+      const float x = key < Bb ? s[n][e] * a.scale_log2 : -INFINITY;
       s[n][e] = x;
       mx[e >> 1] = fmaxf(mx[e >> 1], x);
     }
@@ -250,9 +265,11 @@ __global__ void __launch_bounds__(128) block_attn_kernel(const __grid_constant__
 // The FlashBlock merge with the cached partial is fused as in the bf16 kernel.
 // ---------------------------------------------------------------------------
 struct BlockArgsF32 {
-  const float* q;  // [batch, B, Hq, D]
+  const float* q;  // [batch, B, Hq, D], or packed as in BlockArgs
   const float* k;  // [batch, B, Hkv, D]
   const float* v;
+  const int32_t* cu;
+  int total;
   const float* mrg_a;
   const float* mrg_l;
   float* a_out;
@@ -274,30 +291,33 @@ __global__ void __launch_bounds__(256) block_attn_f32_kernel(const __grid_consta
   float* kT = qs + a.R * D;    // [D][KP]
   const int hk = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+  long long base;
+  const int Bb = block_rows(a, b, base);  // block rows (= keys) of this sequence
+  const int Rb = Bb * a.G;                // a.R (the most rows) sizes the shared layout
   // V and Q rows by cp.async (16-byte chunks), K through registers into the
   // transposed layout; keys past the block are zero
   constexpr int C4 = D / 4;
   for (int idx = tid; idx < NK * C4; idx += blockDim.x) {
     const int j = idx / C4, c = idx - j * C4;
-    const bool ok = j < a.B;
-    const long long off = (((long long)b * a.B + (ok ? j : 0)) * a.Hkv + hk) * D + c * 4;
+    const bool ok = j < Bb;
+    const long long off = ((base + (ok ? j : 0)) * a.Hkv + hk) * D + c * 4;
     cp_async16(smem_u32(vs + j * D + c * 4), a.v + off, ok ? 16u : 0u);
   }
-  for (int idx = tid; idx < a.R * C4; idx += blockDim.x) {
+  for (int idx = tid; idx < Rb * C4; idx += blockDim.x) {
     const int r = idx / C4, c = idx - r * C4;
     const int i = r / a.G, h = hk * a.G + (r - i * a.G);
-    cp_async16(smem_u32(qs + r * D + c * 4), a.q + (((long long)b * a.B + i) * a.Hq + h) * D + c * 4,
+    cp_async16(smem_u32(qs + r * D + c * 4), a.q + ((base + i) * a.Hq + h) * D + c * 4,
                16u);
   }
   cp_async_commit();
   for (int idx = tid; idx < NK * D; idx += blockDim.x) {
     const int j = idx / D, c = idx - j * D;
-    kT[c * KP + j] = j < a.B ? a.k[(((long long)b * a.B + j) * a.Hkv + hk) * D + c] : 0.f;
+    kT[c * KP + j] = j < Bb ? a.k[((base + j) * a.Hkv + hk) * D + c] : 0.f;
   }
   cp_async_wait<0>();
   __syncthreads();
   constexpr int NV = D / 32;
-  for (int r = warp; r < a.R; r += nw) {
+  for (int r = warp; r < Rb; r += nw) {
     const float* qr = qs + r * D;
     float s0 = 0.f, s1 = 0.f;  // keys lane and lane + 32
 #pragma unroll 8
@@ -306,8 +326,8 @@ __global__ void __launch_bounds__(256) block_attn_f32_kernel(const __grid_consta
       s0 = fmaf(qc, kT[c * KP + lane], s0);
       s1 = fmaf(qc, kT[c * KP + lane + 32], s1);
     }
-    s0 = lane < a.B ? s0 * a.scale : -INFINITY;
-    s1 = lane + 32 < a.B ? s1 * a.scale : -INFINITY;
+    s0 = lane < Bb ? s0 * a.scale : -INFINITY;
+    s1 = lane + 32 < Bb ? s1 * a.scale : -INFINITY;
     float m = fmaxf(s0, s1);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -318,13 +338,13 @@ __global__ void __launch_bounds__(256) block_attn_f32_kernel(const __grid_consta
     float o[NV];
 #pragma unroll
     for (int t = 0; t < NV; ++t) o[t] = 0.f;
-    for (int j = 0; j < a.B; ++j) {
+    for (int j = 0; j < Bb; ++j) {
       const float pj = __shfl_sync(0xffffffffu, j < 32 ? p0 : p1, j & 31);
 #pragma unroll
       for (int t = 0; t < NV; ++t) o[t] = fmaf(pj, vs[j * D + lane + 32 * t], o[t]);
     }
     const int i = r / a.G, h = hk * a.G + (r - i * a.G);
-    const long long row = ((long long)b * a.B + i) * a.Hq + h;
+    const long long row = (base + i) * a.Hq + h;
     const float Ln = m + logf(l);
     float wn = 1.f / l, wo = 0.f, L = Ln;
     if (a.mrg_a) {

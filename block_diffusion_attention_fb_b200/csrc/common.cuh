@@ -14,6 +14,22 @@ __device__ int g_fb_error_word;
 constexpr int kErrTimeout = 1;      // a bounded wait gave up
 constexpr int kErrBadPage = 2;      // block commit: page-table entry outside the pool
 constexpr int kErrBadReadPage = 4;  // a read path met a page-table entry outside the pool
+constexpr int kErrBadRows = 8;      // packed row offsets outside the buffer or decreasing
+
+// Packed (variable-length) rows: rows [r0, r0 + n) of a packed buffer of `total` rows from offsets cu[b],
+// cu[b+1], with n capped at `cap`. Offsets that leave the buffer or decrease
+// give an empty range and set the error word (nothing is read through them).
+__device__ __forceinline__ int packed_range(const int32_t* cu, int b, int total, int cap,
+                                            long long& r0) {
+  const int lo = cu[b], hi = cu[b + 1];
+  r0 = lo;
+  if (lo < 0 || hi < lo || hi > total || hi - lo > cap) {
+    atomicOr(&g_fb_error_word, kErrBadRows);
+    r0 = 0;
+    return 0;
+  }
+  return hi - lo;
+}
 
 // Budget of a bounded wait: about one second at B200 clocks.
 constexpr long long kWaitBudgetCycles = 2000000000LL;

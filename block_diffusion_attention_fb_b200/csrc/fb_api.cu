@@ -303,7 +303,9 @@ int make_tmap(CUtensorMap* m, const void* base, int D, int Hkv, long long n_slot
   return FB_OK;
 }
 
-int validate_kv(const fb_kv* kv) {
+// packed: a varlen block's own keys (rows of each sequence given by offsets,
+// so the per-sequence capacity check of a contiguous cache does not apply)
+int validate_kv(const fb_kv* kv, bool packed = false) {
   if (!kv) return fail(FB_ERR_ARG, "kv is NULL");
   if (!kv->k || !kv->v) return fail(FB_ERR_ARG, "kv->k / kv->v is NULL");
   if (kv->batch <= 0 || kv->batch > 256) return fail(FB_ERR_ARG, "batch must be in [1, 256]");
@@ -317,7 +319,7 @@ int validate_kv(const fb_kv* kv) {
     return fail(FB_ERR_SHAPE, "page_size must be a power of two >= 16");
   if (kv->page_table && kv->max_pages_per_seq * (long long)kv->page_size < kv->max_seq_len)
     return fail(FB_ERR_ARG, "max_pages_per_seq * page_size < max_seq_len");
-  if (!kv->page_table && (long long)kv->batch * kv->max_seq_len > kv->n_slots)
+  if (!packed && !kv->page_table && (long long)kv->batch * kv->max_seq_len > kv->n_slots)
     return fail(FB_ERR_ARG, "contiguous cache needs batch * max_seq_len <= n_slots");
   if (!aligned16(kv->k) || !aligned16(kv->v)) return fail(FB_ERR_ALIGN, "k / v not 16-byte aligned");
   return FB_OK;
@@ -346,6 +348,9 @@ struct PartialCall {
   bool single_split;  // one CTA streams the whole key set (no workspace)
   const float* mrg_a;  // optional: merge every final row with this partial (FlashBlock merge)
   const float* mrg_l;
+  const int32_t* q_cu;   // optional: packed query rows (device [batch + 1] offsets), q_total rows
+  int q_total;
+  const int32_t* kv_cu;  // optional: packed contiguous key set (device [batch + 1] offsets)
 };
 
 // The kernels order keys by raw score when forming the row maximum, which
@@ -389,6 +394,10 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
   a.scale_log2 = c.scale * kLog2e;
   a.mrg_a = c.mrg_a;
   a.mrg_l = c.mrg_l;
+  if (c.q_cu && c.row_list) return fail(FB_ERR_ARG, "packed rows cannot take a row list");
+  a.q_cu = c.q_cu;
+  a.q_total = c.q_total;
+  a.kv_cu = c.kv_cu;
   a.a_out = c.a_out;
   a.l_out = c.l_out;
   a.a_prev = c.a_prev;
@@ -544,9 +553,11 @@ dim3 page_score_grid(const KvView& v, int num_sms, int& cpc) {
 // grid within two CTAs per SM (more CTAs = more of the block's loads in flight).
 int block_attn_short(const void* q, const void* k_in, const void* v_in, int batch, int B, int Hq,
                      int Hkv, int D, float scale, float* a_out, float* l_out, const float* mrg_a,
-                     const float* mrg_l, cudaStream_t stream) {
+                     const float* mrg_l, const int32_t* cu, int total, cudaStream_t stream) {
   if (int rc_ = validate_scale(scale)) return rc_;
   BlockArgs a{};
+  a.cu = cu;
+  a.total = total;
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.k = static_cast<const __nv_bfloat16*>(k_in);
   a.v = static_cast<const __nv_bfloat16*>(v_in);
@@ -601,9 +612,12 @@ int block_attn_short(const void* q, const void* k_in, const void* v_in, int batc
 // Short fp32 blocks (B <= 64): one CTA of up to 8 warps per (sequence, kv head).
 int block_attn_short_f32(const void* q, const void* k_in, const void* v_in, int batch, int B,
                          int Hq, int Hkv, int D, float scale, float* a_out, float* l_out,
-                         const float* mrg_a, const float* mrg_l, cudaStream_t stream) {
+                         const float* mrg_a, const float* mrg_l, const int32_t* cu, int total,
+                         cudaStream_t stream) {
   if (int rc_ = validate_scale(scale)) return rc_;
   BlockArgsF32 a{};
+  a.cu = cu;
+  a.total = total;
   a.q = static_cast<const float*>(q);
   a.k = static_cast<const float*>(k_in);
   a.v = static_cast<const float*>(v_in);
@@ -636,32 +650,36 @@ int block_attn_short_f32(const void* q, const void* k_in, const void* v_in, int 
   return check_launch("fp32 block attention kernel");
 }
 
+// Block-internal partial of every block row (optionally merged with mrg_a /
+// mrg_l). Packed rows (cu != NULL): sequence b's rows and keys are rows
+// cu[b] .. cu[b+1]-1 of the total packed rows, at most B of them.
 int block_attn_impl(const void* q, const void* k_in, const void* v_in, int batch, int B, int Hq,
                     int Hkv, int D, float scale, fb_dtype dt, float* a_in, float* l_in,
                     cudaStream_t stream, const float* mrg_a = nullptr,
-                    const float* mrg_l = nullptr) {
+                    const float* mrg_l = nullptr, const int32_t* cu = nullptr, int total = 0) {
   fb_kv kv{};
   kv.k = k_in;
   kv.v = v_in;
-  kv.n_slots = (long long)batch * B;
+  kv.n_slots = cu ? (long long)(total > 0 ? total : 1) : (long long)batch * B;
   kv.batch = batch;
   kv.n_heads_kv = Hkv;
   kv.head_dim = D;
   kv.page_size = 16;
   kv.max_seq_len = B;
   kv.dtype = dt;
-  int rc = validate_kv(&kv);
+  int rc = validate_kv(&kv, cu != nullptr);
   if (rc) return rc;
   rc = validate_q(q, B, Hq, &kv);
   if (rc) return rc;
   if (!a_in || !l_in) return fail(FB_ERR_ARG, "a_in / l_in is NULL");
   if (mrg_a && !mrg_l) return fail(FB_ERR_ARG, "merge partner without its L");
+  if (cu && total == 0) return FB_OK;  // no rows at all
   if (dt == FB_BF16 && (D == 64 || D == 128) && B <= 64) return block_attn_short(
-      q, k_in, v_in, batch, B, Hq, Hkv, D, scale, a_in, l_in, mrg_a, mrg_l, stream);
+      q, k_in, v_in, batch, B, Hq, Hkv, D, scale, a_in, l_in, mrg_a, mrg_l, cu, total, stream);
   if (dt == FB_F32 && (D == 64 || D == 128) && B <= 64 &&
       block_f32_smem(D, B * (Hq / Hkv)) <= 200 * 1024)
     return block_attn_short_f32(q, k_in, v_in, batch, B, Hq, Hkv, D, scale, a_in, l_in, mrg_a,
-                                mrg_l, stream);
+                                mrg_l, cu, total, stream);
   PartialCall c{};
   c.q = q;
   c.B = B;
@@ -676,6 +694,9 @@ int block_attn_impl(const void* q, const void* k_in, const void* v_in, int batch
   c.num_sms = sm_count();
   c.mrg_a = mrg_a;
   c.mrg_l = mrg_l;
+  c.q_cu = cu;
+  c.q_total = total;
+  c.kv_cu = cu;
   return launch_partial(c, stream);
 }
 
@@ -749,6 +770,9 @@ int fb_device_status(void) {
   if (word & kErrBadReadPage)
     return fail(FB_ERR_ARG, "a page-table entry outside the pool was read (its tokens were "
                             "treated as absent)");
+  if (word & kErrBadRows)
+    return fail(FB_ERR_ARG, "packed row offsets left the buffer, decreased or exceeded the most "
+                            "rows per sequence (that sequence was treated as empty)");
   if (word) return fail(FB_ERR_TIMEOUT, "a device-side wait exceeded its budget");
   return FB_OK;
 }
@@ -1047,11 +1071,16 @@ int losa_gather(const void* q, int32_t B, int32_t n_heads_q, const int32_t* acti
   return launch_partial(c, stream);
 }
 
-int fb_step(const fb_policy* policy, fb_cache* cache, const void* q, const void* k_in,
-            const void* v_in, int32_t B, int32_t n_heads_q, const fb_kv* prefix,
-            const void* page_min, const void* page_max, const int32_t* m_updated, float* a_full,
-            float* l_full, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+// One denoise step (fb_step); with cu != NULL the block rows are packed
+// (fb_step_varlen): B is the most rows any sequence has, total the packed rows.
+static int step_impl(const fb_policy* policy, fb_cache* cache, const void* q, const void* k_in,
+                     const void* v_in, int32_t B, int32_t n_heads_q, const fb_kv* prefix,
+                     const void* page_min, const void* page_max, const int32_t* m_updated,
+                     float* a_full, float* l_full, void* workspace, size_t workspace_bytes,
+                     const int32_t* cu, int32_t total, cudaStream_t stream) {
   if (!policy || !cache) return fail(FB_ERR_ARG, "policy / cache is NULL");
+  if (cu && policy->mode != FB_THRESHOLD)
+    return fail(FB_ERR_ARG, "packed rows support the threshold controller only");
   int rc = validate_kv(prefix);
   if (rc) return rc;
   rc = validate_q(q, B, n_heads_q, prefix);
@@ -1081,6 +1110,8 @@ int fb_step(const fb_policy* policy, fb_cache* cache, const void* q, const void*
   c.ws_bytes = workspace_bytes;
   c.ws_offset = w.part;
   c.num_sms = num_sms;
+  c.q_cu = cu;
+  c.q_total = total;
 
   if (policy->mode == FB_THRESHOLD) {
     unsigned long long bits[4] = {0, 0, 0, 0};
@@ -1190,10 +1221,82 @@ int fb_step(const fb_policy* policy, fb_cache* cache, const void* q, const void*
   // block-external partial in one kernel: A_full directly
   float* lf = l_full ? l_full : reinterpret_cast<float*>(ws + w.l_in);
   rc = block_attn_impl(q, k_in, v_in, batch, B, Hq, Hkv, D, policy->scale, prefix->dtype, a_full,
-                       lf, stream, cache->a_out, cache->l_out);
+                       lf, stream, cache->a_out, cache->l_out, cu, total);
   if (rc) return rc;
   cache->step = s + 1;
   return FB_OK;
+}
+
+int fb_step(const fb_policy* policy, fb_cache* cache, const void* q, const void* k_in,
+            const void* v_in, int32_t B, int32_t n_heads_q, const fb_kv* prefix,
+            const void* page_min, const void* page_max, const int32_t* m_updated, float* a_full,
+            float* l_full, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return step_impl(policy, cache, q, k_in, v_in, B, n_heads_q, prefix, page_min, page_max,
+                   m_updated, a_full, l_full, workspace, workspace_bytes, nullptr, 0, stream);
+}
+
+// Host checks shared by the packed-row entry points.
+static int validate_packed(const int32_t* cu_rows, int32_t max_rows, int32_t total_rows) {
+  if (!cu_rows) return fail(FB_ERR_ARG, "cu_rows is NULL");
+  if (max_rows <= 0) return fail(FB_ERR_ARG, "max_rows must be positive");
+  if (total_rows < 0) return fail(FB_ERR_ARG, "total_rows must be >= 0");
+  return FB_OK;
+}
+
+int fb_prefix_attn_varlen(const void* q, const int32_t* cu_rows, int32_t max_rows,
+                          int32_t total_rows, int32_t n_heads_q, float scale, const fb_kv* kv,
+                          float* a_out, float* l_out, void* workspace, size_t workspace_bytes,
+                          cudaStream_t stream) {
+  int rc = validate_kv(kv);
+  if (rc) return rc;
+  if ((rc = validate_packed(cu_rows, max_rows, total_rows))) return rc;
+  rc = validate_q(q, max_rows, n_heads_q, kv);
+  if (rc) return rc;
+  if (!a_out || !l_out) return fail(FB_ERR_ARG, "a_out / l_out is NULL");
+  if (total_rows == 0) return FB_OK;
+  PartialCall c{};
+  c.q = q;
+  c.B = max_rows;
+  c.Hq = n_heads_q;
+  c.scale = scale;
+  c.kv = kv;
+  c.a_out = a_out;
+  c.l_out = l_out;
+  c.ws = workspace;
+  c.ws_bytes = workspace_bytes;
+  c.num_sms = sm_count();
+  c.q_cu = cu_rows;
+  c.q_total = total_rows;
+  return launch_partial(c, stream);
+}
+
+int fb_block_attn_varlen(const void* q, const void* k_in, const void* v_in,
+                         const int32_t* cu_rows, int32_t batch, int32_t max_rows,
+                         int32_t total_rows, int32_t n_heads_q, int32_t n_heads_kv,
+                         int32_t head_dim, float scale, fb_dtype dtype, float* a_in, float* l_in,
+                         cudaStream_t stream) {
+  int rc = validate_packed(cu_rows, max_rows, total_rows);
+  if (rc) return rc;
+  if (!k_in || !v_in) return fail(FB_ERR_ARG, "k_in / v_in is NULL");
+  if (!aligned16(k_in) || !aligned16(v_in)) return fail(FB_ERR_ALIGN, "k_in / v_in not 16-byte aligned");
+  return block_attn_impl(q, k_in, v_in, batch, max_rows, n_heads_q, n_heads_kv, head_dim, scale,
+                         dtype, a_in, l_in, stream, nullptr, nullptr, cu_rows, total_rows);
+}
+
+int fb_step_varlen(const fb_policy* policy, fb_cache* cache, const void* q, const void* k_in,
+                   const void* v_in, const int32_t* cu_rows, int32_t max_rows,
+                   int32_t total_rows, int32_t n_heads_q, const fb_kv* prefix,
+                   const int32_t* m_updated, float* a_full, float* l_full, void* workspace,
+                   size_t workspace_bytes, cudaStream_t stream) {
+  int rc = validate_packed(cu_rows, max_rows, total_rows);
+  if (rc) return rc;
+  if (total_rows == 0) {
+    if (cache) cache->step += 1;
+    return FB_OK;
+  }
+  return step_impl(policy, cache, q, k_in, v_in, max_rows, n_heads_q, prefix, nullptr, nullptr,
+                   m_updated, a_full, l_full, workspace, workspace_bytes, cu_rows, total_rows,
+                   stream);
 }
 
 // Unique id of the calling thread's current context (false if none is current

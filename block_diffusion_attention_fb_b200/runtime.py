@@ -11,7 +11,7 @@ from typing import Optional, Sequence
 import torch
 
 from . import (FB_LOSA, FB_PER_HEAD, FB_SPARSE_RESIDUAL, FB_THRESHOLD, KV, fb_cache,
-               fb_page_summary, fb_policy, fb_step, fb_workspace_size)
+               fb_page_summary, fb_policy, fb_step, fb_step_varlen, fb_workspace_size)
 
 _MODES = {"threshold": FB_THRESHOLD, "per_head": FB_PER_HEAD, "losa": FB_LOSA,
           "sparse_residual": FB_SPARSE_RESIDUAL}
@@ -87,6 +87,47 @@ class BlockAttention:
     @property
     def step_index(self) -> int:
         return self.cache.step
+
+    @property
+    def recomputed(self) -> int:
+        return self.cache.recomputed
+
+
+class VarlenBlockAttention:
+    """Threshold (tau) reuse over packed block rows: the blocks (branches) of
+    all sequences, of different sizes, in one launch per step.
+
+    cu_rows: int32 [batch + 1] row offsets (host sequence or tensor); sequence
+    b owns packed rows cu_rows[b] .. cu_rows[b+1]-1. Cache buffers are packed
+    [total, Hq, d] like q; the workspace is sized for the longest block.
+    """
+
+    def __init__(self, kv: KV, cu_rows, n_heads_q: int, tau: int = 0, scale: float = 1.0,
+                 device=None):
+        dev = device or kv.k.device
+        cu = [int(x) for x in (cu_rows.tolist() if hasattr(cu_rows, "tolist") else cu_rows)]
+        if len(cu) != kv.batch + 1:
+            raise ValueError("cu_rows needs batch + 1 offsets")
+        self.kv, self.Hq = kv, n_heads_q
+        self.total = cu[-1]
+        self.max_rows = max(1, max(b - a for a, b in zip(cu[:-1], cu[1:])))
+        self.cu = torch.tensor(cu, dtype=torch.int32, device=dev)
+        d = kv.c.head_dim
+        self.policy = fb_policy(FB_THRESHOLD, tau, 2.0, 0, 0, scale)
+        self.a_out = torch.zeros(max(self.total, 1), n_heads_q, d, dtype=torch.float32, device=dev)
+        self.l_out = torch.zeros(max(self.total, 1), n_heads_q, dtype=torch.float32, device=dev)
+        self.workspace = torch.empty(fb_workspace_size(kv, self.max_rows, n_heads_q),
+                                     dtype=torch.uint8, device=dev)
+        self.cache = fb_cache(self.a_out.data_ptr(), self.l_out.data_ptr(), None, None, None, None,
+                              None, None, None, None, None, 0, 0, None, None, None, None)
+
+    def reset(self) -> None:
+        self.cache.step = 0
+
+    def step(self, q, k_in, v_in, a_full, l_full=None,
+             m_updated: Optional[Sequence[int]] = None, stream=None) -> None:
+        fb_step_varlen(self.policy, self.cache, q, k_in, v_in, self.cu, self.max_rows, self.kv,
+                       a_full, l_full, m_updated, self.workspace, stream)
 
     @property
     def recomputed(self) -> int:

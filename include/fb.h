@@ -297,6 +297,53 @@ int fb_step(const fb_policy* policy, fb_cache* cache, const void* q, const void*
             const void* page_min, const void* page_max, const int32_t* m_updated, float* a_full,
             float* l_full, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Packed (variable-length) block rows. Several blocks or branches of different
+ * sizes share one launch: the BlockBatch page (gist.science, es), "Optimizacion
+ * del Sistema", packs the unmasked query positions of all active branches into
+ * one variable-length buffer so that branches of different block sizes run in
+ * a single forward. Here sequence b of the batch (a branch, with its own prefix
+ * through kv; branches of one request may share prefix pages through the page
+ * table) owns block rows cu_rows[b] .. cu_rows[b+1]-1 of every packed buffer:
+ *   q, a_*      [total_rows, n_heads_q, head_dim], l_* [total_rows, n_heads_q]
+ *   k_in, v_in  [total_rows, n_heads_kv, head_dim] (the block's own keys)
+ * cu_rows     DEVICE [batch + 1] int32, cu_rows[0] = 0, non-decreasing,
+ *             cu_rows[batch] = total_rows. A sequence may have 0 rows.
+ * max_rows    HOST: the most rows any sequence has (plans the launch and sizes
+ *             the workspace: fb_workspace_size(kv, max_rows, n_heads_q, 0, 0, 0)).
+ * total_rows  HOST: rows of the packed buffers.
+ * The kernels check every sequence's offsets: a range that leaves
+ * [0, total_rows], decreases or holds more than max_rows rows is treated as
+ * empty (nothing is read or written through it) and the next
+ * fb_device_status() returns FB_ERR_ARG.
+ * ------------------------------------------------------------------------- */
+
+/* fb_prefix_attn over packed rows: (A_out, L_out) of every packed row over its
+ * own sequence's block-external keys ([FB] section 2). No head mask. */
+int fb_prefix_attn_varlen(const void* q, const int32_t* cu_rows, int32_t max_rows,
+                          int32_t total_rows, int32_t n_heads_q, float scale, const fb_kv* kv,
+                          float* a_out, float* l_out, void* workspace, size_t workspace_bytes,
+                          cudaStream_t stream);
+
+/* fb_block_attn over packed rows: every row of sequence b attends the B_b =
+ * cu_rows[b+1] - cu_rows[b] keys of its own block (bidirectional). */
+int fb_block_attn_varlen(const void* q, const void* k_in, const void* v_in,
+                         const int32_t* cu_rows, int32_t batch, int32_t max_rows,
+                         int32_t total_rows, int32_t n_heads_q, int32_t n_heads_kv,
+                         int32_t head_dim, float scale, fb_dtype dtype, float* a_in, float* l_in,
+                         cudaStream_t stream);
+
+/* fb_step over packed rows, THRESHOLD mode only (FB_ERR_ARG otherwise): each
+ * sequence recomputes its A_out when step == 0 or m_updated[b] >= tau, then
+ * the block-internal partial is computed and merged ([FB] section 2). The
+ * cache's a_out / l_out are packed like q ([total_rows, n_heads_q, head_dim]).
+ * total_rows = 0 only advances cache->step. */
+int fb_step_varlen(const fb_policy* policy, fb_cache* cache, const void* q, const void* k_in,
+                   const void* v_in, const int32_t* cu_rows, int32_t max_rows,
+                   int32_t total_rows, int32_t n_heads_q, const fb_kv* prefix,
+                   const int32_t* m_updated, float* a_full, float* l_full, void* workspace,
+                   size_t workspace_bytes, cudaStream_t stream);
+
 /*
  * Block commit: the finished block joins the block-external cache. Block
  * diffusion is causal between blocks ([FB] abstract, section 2), so once a

@@ -13,9 +13,10 @@ Modules:
   controllers  threshold (tau), per-head (gamma) and LoSA step procedures
   cache        block commit: a finished block's K/V appended to the cache
   residual     FlashBlock + sparse attention: cached residual of unselected pages
+  varlen       packed (variable-length) block rows of several sequences
 """
 
-from . import attention, cache, controllers, losa, residual  # noqa: F401
+from . import attention, cache, controllers, losa, residual, varlen  # noqa: F401
 from .attention import (  # noqa: F401
     block_partial,
     dense_attention,

@@ -231,3 +231,36 @@ def test_step_binding_rejects_too_few_update_counts():
     q = torch.zeros(3, 4, 4, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="3 sequences"):
         fb.fb_step(fb.fb_policy(), fb.fb_cache(), q, q, q, kv, q, m_updated=[1, 2])
+
+
+# ------------------------------------------------------ packed-row entry points
+def test_varlen_entry_points_reject_bad_row_arguments(lib):
+    kv = make_kv()
+    # cu_rows NULL, max_rows <= 0, total_rows < 0
+    for cu, mx, tot in ((None, 4, 8), (DEV, 0, 8), (DEV, 4, -1)):
+        rc = lib.fb_prefix_attn_varlen(DEV, cu, mx, tot, 4, 1.0, ctypes.byref(kv), DEV, DEV, DEV,
+                                       1 << 30, None)
+        assert rc == fb.FB_ERR_ARG, err(lib)
+        rc = lib.fb_block_attn_varlen(DEV, DEV, DEV, cu, 1, mx, tot, 4, 2, 128, 1.0, fb.FB_BF16,
+                                      DEV, DEV, None)
+        assert rc == fb.FB_ERR_ARG, err(lib)
+    # misaligned block keys
+    rc = lib.fb_block_attn_varlen(DEV, MISALIGNED, DEV, DEV, 1, 4, 8, 4, 2, 128, 1.0, fb.FB_BF16,
+                                  DEV, DEV, None)
+    assert rc == fb.FB_ERR_ALIGN, err(lib)
+    # a bad cache is still a bad cache
+    rc = lib.fb_prefix_attn_varlen(DEV, DEV, 4, 8, 4, 1.0, ctypes.byref(make_kv(head_dim=96)), DEV,
+                                   DEV, DEV, 1 << 30, None)
+    assert rc == fb.FB_ERR_SHAPE
+
+
+@pytest.mark.parametrize("mode", [fb.FB_PER_HEAD, fb.FB_LOSA, fb.FB_SPARSE_RESIDUAL])
+def test_step_varlen_takes_the_threshold_controller_only(lib, mode):
+    kv = make_kv()
+    pol = fb.fb_policy(mode, 2, 0.9, 2, 4, 1.0)
+    cache = fb.fb_cache()
+    cache.a_out = cache.l_out = DEV
+    rc = lib.fb_step_varlen(ctypes.byref(pol), ctypes.byref(cache), DEV, DEV, DEV, DEV, 4, 8, 4,
+                            ctypes.byref(kv), None, DEV, DEV, DEV, 1 << 30, None)
+    assert rc == fb.FB_ERR_ARG
+    assert "threshold" in err(lib)
