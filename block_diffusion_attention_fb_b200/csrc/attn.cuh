@@ -195,6 +195,17 @@ __device__ __forceinline__ void chunk_slot(const AttnArgs& a, int b, int hk, int
   chunk_slot(a, group_info(a, b, hk), b, hk, tl, c, slot, valid);
 }
 
+// Key tiles per split of (b, hk). Dense key sets use the plan's; page lists,
+// whose lengths the host plan only bounds, spread their actual tiles evenly
+// over the planned splits (no more than the plan's, so every buffer sized by
+// the plan still holds). even: a whole number of 128-key tiles (tcgen05).
+__device__ __forceinline__ int split_tiles(const AttnArgs& a, int n_tiles, bool even) {
+  if (!a.page_list) return a.tiles_per_split;
+  int t = (n_tiles + a.n_splits - 1) / a.n_splits;
+  if (even) t = (t + 1) & ~1;
+  return min(max(t, even ? 2 : 1), a.tiles_per_split);
+}
+
 // Maps row r of (b, hk) to the block row i and q head h.
 __device__ __forceinline__ void row_of(const AttnArgs& a, int b, int hk, int r, int& i, int& h) {
   const int i_idx = r / a.G;
@@ -482,8 +493,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   if (rt * a.row_tile >= Rb) return;
 
   const int n_tiles = n_tiles_of(a, b, hk);
-  const int tile0 = split * a.tiles_per_split;
-  const int n_it = max(0, min(a.tiles_per_split, n_tiles - tile0));
+  const int tps = split_tiles(a, n_tiles, false);
+  const int tile0 = split * tps;
+  const int n_it = max(0, min(tps, n_tiles - tile0));
   const int n_chunks = kTK / a.chunk;
 
   const uint32_t base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
@@ -837,8 +849,9 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const __grid_constant__ A
   if (rt * a.row_tile >= Rb) return;
   const GroupInfo gi = group_info(a, b, hk);
   const int n_tiles = n_tiles_of(a, gi);
-  const int tile0 = split * a.tiles_per_split;
-  const int n_it = max(0, min(a.tiles_per_split, n_tiles - tile0));
+  const int tps = split_tiles(a, n_tiles, false);
+  const int tile0 = split * tps;
+  const int n_it = max(0, min(tps, n_tiles - tile0));
   const int n_chunks = kTK / a.chunk;
   const float* qf = static_cast<const float*>(a.q);
   const float* kg = static_cast<const float*>(a.k);

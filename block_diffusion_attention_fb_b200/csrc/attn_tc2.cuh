@@ -91,9 +91,11 @@ __global__ void __launch_bounds__(kT2Threads, 1)
   if (!cta_selected(a, b, hk)) return;
   const int Rb = rows_of(a, b);  // stacked rows of this sequence
   if (rt * kT2Rows >= Rb) return;
-  // key range of this split in 64-key sub-tiles (tiles_per_split is even)
-  const int n64 = max(0, min(a.tiles_per_split, n_tiles_of(a, b, hk) - split * a.tiles_per_split));
-  const int tile0 = split * a.tiles_per_split;
+  // key range of this split in 64-key sub-tiles (an even number per split)
+  const int n64_all = n_tiles_of(a, b, hk);
+  const int tps = split_tiles(a, n64_all, true);
+  const int n64 = max(0, min(tps, n64_all - split * tps));
+  const int tile0 = split * tps;
   const int n_it = (n64 + 1) >> 1;  // 128-key tiles
   const int n_chunks = kTK / a.chunk;  // metadata chunks per 64-key sub-tile
   const bool has_b = Rb - rt * kT2Rows > kT2TileRows;

@@ -718,7 +718,7 @@ int sr_select(const void* q, int B, int Hq, const void* page_min, const void* pa
   int cpc;
   const dim3 g2 = page_score_grid(v, sm_count(), cpc);
   const int es = (int)elem_size(kv->dtype);
-  const int psm = RQ * D * 4 + 4 * kPsPages * (D + 16 / es) * es;
+  const int psm = page_score_smem(RQ, D, es);
   int rc;
 #define FB_HPS(TT, DD)                                                                       \
   do {                                                                                       \
@@ -1007,8 +1007,7 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
   if (rc) return rc;
   int cpc;
   const dim3 g2 = page_score_grid(v, num_sms, cpc);
-  const int psm = na * G * D * 4 + 4 * kPsPages * (D + 16 / (int)elem_size(kv->dtype)) *
-                                       (int)elem_size(kv->dtype);
+  const int psm = page_score_smem(na * G, D, (int)elem_size(kv->dtype));
   if (kv->dtype == FB_BF16) {
     auto kfn = D == 128 ? page_score_kernel<__nv_bfloat16, 128> : page_score_kernel<__nv_bfloat16, 64>;
     if ((rc = set_smem_once((const void*)kfn, psm))) return rc;

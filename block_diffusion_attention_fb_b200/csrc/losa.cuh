@@ -236,6 +236,9 @@ __global__ void __launch_bounds__(256)
 // handled in chunks of kPsPages.
 // ---------------------------------------------------------------------------
 constexpr int kPsPages = 64;
+// chunk buffers of the page scorers: bf16 three (two load while one is scored),
+// float32 two (its chunks are twice as large)
+__host__ __device__ constexpr int ps_stages(int elem_bytes) { return elem_bytes == 2 ? 3 : 2; }
 
 // Shared-memory row stride (elements) of the staged page summaries: rows stay
 // 16-byte aligned for vector loads, and consecutive pages start 4 banks apart,
@@ -293,6 +296,106 @@ __device__ __forceinline__ float page_bound(const float* qr, const T* mnr, const
   return y[0];
 }
 
+// The same bound for bf16 inputs, evaluated as tree_sum_c q_c * s_c with s_c =
+// kmax_c where q_c >= 0 and kmin_c where q_c < 0. A product of two bf16 values
+// is exact in float32, so max(q_c kmin_c, q_c kmax_c) IS q_c s_c, bit for bit
+// (for q_c = 0 both are zeros); the products and the tree are unchanged, only
+// the selection happens before the multiply. Two channels per 32-bit word: the
+// per-row mask qm (0xFFFF in the half of each channel with q_c < 0) picks the
+// bf16 halves with one bitwise select; products and tree levels with stride >= 2
+// run on packed float pairs (f32x2), each lane single-rounded as in the
+// definition. q row qr (float) and qm are read by every lane of the warp at the
+// same address (broadcast); mnr / mxr are this lane's page.
+template <int D>
+__device__ __forceinline__ float page_bound_sel(const float* qr, const uint32_t* qm,
+                                                const __nv_bfloat16* mnr,
+                                                const __nv_bfloat16* mxr) {
+  // The first three tree levels (channel strides D/2, D/4, D/8) are formed per
+  // output channel n < E = D/8 from the eight channels n + k E, k = 0..7:
+  //   ((a_n + a_n+4E) + (a_n+2E + a_n+6E)) + ((a_n+E + a_n+5E) + (a_n+3E + a_n+7E)),
+  // which is the tree's own pairing and order; only E values stay live.
+  constexpr int E = D / 8;
+  float2 z[E / 2];  // level-3 sums of channels (2i, 2i + 1)
+  // products of the channel pairs c8 + 2j (+1) + k E, j = 0..3
+  auto prod = [&](int c8, int k, float2 (&a)[4]) {
+    const int c = c8 + k * E;
+    const uint4 n = *reinterpret_cast<const uint4*>(mnr + c);
+    const uint4 x = *reinterpret_cast<const uint4*>(mxr + c);
+    const uint4 m = *reinterpret_cast<const uint4*>(qm + c / 2);
+    const float4 qa = *reinterpret_cast<const float4*>(qr + c);
+    const float4 qb = *reinterpret_cast<const float4*>(qr + c + 4);
+    const uint32_t nn[4] = {n.x, n.y, n.z, n.w}, xx[4] = {x.x, x.y, x.z, x.w};
+    const uint32_t mm[4] = {m.x, m.y, m.z, m.w};
+    const float2 qq[4] = {make_float2(qa.x, qa.y), make_float2(qa.z, qa.w),
+                          make_float2(qb.x, qb.y), make_float2(qb.z, qb.w)};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t sel = (xx[j] & ~mm[j]) | (nn[j] & mm[j]);
+      a[j] = fmul2(qq[j], make_float2(__uint_as_float(sel << 16),
+                                      __uint_as_float(sel & 0xFFFF0000u)));
+    }
+  };
+  // level-1 pair (k, k + 4) of the eight offsets
+  auto level1 = [&](int c8, int k, float2 (&b)[4]) {
+    float2 lo[4], hi[4];
+    prod(c8, k, lo);
+    prod(c8, k + 4, hi);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) b[j] = fadd2(lo[j], hi[j]);
+  };
+#pragma unroll
+  for (int c8 = 0; c8 < E; c8 += 8) {
+    // keeps the next group's loads from being hoisted above this one (which
+    // would hold both groups' operands at once and spill)
+    if (c8 > 0) asm volatile("" ::: "memory");
+    float2 b0[4], b2[4], c0[4];
+    level1(c8, 0, b0);
+    level1(c8, 2, b2);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) c0[j] = fadd2(b0[j], b2[j]);
+    float2 b1[4], b3[4];
+    level1(c8, 1, b1);
+    level1(c8, 3, b3);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) z[c8 / 2 + j] = fadd2(c0[j], fadd2(b1[j], b3[j]));
+  }
+#pragma unroll
+  for (int st = E / 4; st >= 1; st >>= 1)  // channel strides 2 st = E/2 ... 2, in pairs
+#pragma unroll
+    for (int i = 0; i < st; ++i) z[i] = fadd2(z[i], z[i + st]);
+  return __fadd_rn(z[0].x, z[0].y);  // the last level: channel 0 + channel 1
+}
+
+// Shared memory of the page scorers for RQ staged q rows: the rows (float),
+// their sign masks (bf16 inputs), and two buffers of a chunk's summaries.
+__host__ __device__ constexpr int page_score_smem(int RQ, int D, int elem_bytes) {
+  return RQ * D * 4 + (elem_bytes == 2 ? RQ * (D / 2) * 4 : 0) +
+         2 * ps_stages(elem_bytes) * kPsPages * (D + 16 / elem_bytes) * elem_bytes;
+}
+
+// Stages the active q rows of (b, hk) as float, and for bf16 the per-channel
+// sign masks of page_bound_sel: qs [RQ][D], qm [RQ][D/2].
+template <typename T, int D>
+__device__ __forceinline__ void stage_q_rows(const T* q, const int32_t* active, int b, int B,
+                                             int Hq, int G, int hk, int n_act, int RQ, float* qs,
+                                             uint32_t* qm) {
+  for (int idx = threadIdx.x; idx < RQ * D; idx += blockDim.x) {
+    const int rq = idx / D, c = idx - (idx / D) * D;
+    const int a_i = rq / G, g = rq - (rq / G) * G;
+    const int i = active ? active[b * n_act + a_i] : a_i;
+    qs[idx] = ld_f32<T>(q + (((long long)b * B + i) * Hq + hk * G + g) * D + c);
+  }
+  if constexpr (sizeof(T) == 2) {
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < RQ * (D / 2); idx += blockDim.x) {
+      const int rq = idx / (D / 2), c2 = idx - rq * (D / 2);
+      const uint32_t lo = __float_as_uint(qs[rq * D + 2 * c2]) >> 31;
+      const uint32_t hi = __float_as_uint(qs[rq * D + 2 * c2 + 1]) >> 31;
+      qm[idx] = (lo ? 0x0000FFFFu : 0u) | (hi ? 0xFFFF0000u : 0u);
+    }
+  }
+}
+
 // Stages the summaries of 64-page chunk `chunk` of (b, hk) into one of two
 // shared buffers with cp.async (zero-filled past the sequence's pages).
 template <typename T, int D>
@@ -309,28 +412,63 @@ __device__ __forceinline__ void stage_page_chunk(const T* pmin, const T* pmax, c
     cp_async16(smem_u32(smn + pg * PS + cv * VE), pmin + so, ok ? 16u : 0u);
     cp_async16(smem_u32(smx + pg * PS + cv * VE), pmax + so, ok ? 16u : 0u);
   }
-  cp_async_commit();
 }
+
+// The chunk ring of the page scorers: chunks c0 .. c1-1 of (b, hk) cycle
+// through kStages buffers of [64][PS] minima then [64][PS] maxima. One
+// cp.async group is committed per chunk (empty past c1), so that waiting for
+// all but the newest kStages - 1 groups means chunk ch has landed.
+template <typename T, int D>
+struct PageRing {
+  T* sbuf;
+  const T* pmin;
+  const T* pmax;
+  const KvView& kv;
+  int b, hk, c0, c1, n_pages;
+  static constexpr int PS = ps_stride<T, D>();
+  static constexpr int kStages = ps_stages((int)sizeof(T));
+  __device__ T* mn(int ch) const { return sbuf + ((ch - c0) % kStages) * 2 * kPsPages * PS; }
+  __device__ T* mx(int ch) const { return mn(ch) + kPsPages * PS; }
+  __device__ void issue(int ch) const {
+    if (ch < c1) stage_page_chunk<T, D>(pmin, pmax, kv, b, hk, ch, n_pages, mn(ch), mx(ch));
+    cp_async_commit();
+  }
+  __device__ void prologue() const {
+#pragma unroll
+    for (int k = 0; k < kStages - 1; ++k) issue(c0 + k);
+  }
+  // before scoring chunk ch: load chunk ch + kStages - 1 into the buffer that
+  // chunk ch - 1 left (the caller's trailing __syncthreads freed it), wait for ch
+  __device__ void advance(int ch) const {
+    issue(ch + kStages - 1);
+    cp_async_wait<kStages - 1>();
+  }
+};
 
 // Step 3a: QUEST-style page scores u_p = tree_sum_c max(q_c kmin_c, q_c kmax_c)
 // for every active row a and q head h of kv head hk. A CTA scores `cpc`
 // consecutive chunks of 64 pages of one (b, hk): the active q rows once into
 // shared memory, the summaries chunk by chunk into two buffers with cp.async,
-// the next chunk loading while the current one is scored by one thread per
-// (page, row) (page_bound: single-rounded products, stride-halving tree).
+// the next chunk loading while the current one is scored. bf16: a warp takes
+// one q row (broadcast reads) and 32 pages (one per lane; warps 2r and 2r+1
+// the two halves of the chunk, rows r, r + 4, ... for the 8 warps), bound by
+// page_bound_sel; float32: one thread per (page, row) by page_bound. Both are
+// single-rounded products and the stride-halving tree.
 // scores: [batch, n_act, Hq, max_pages]. Block (0, hk, b) also clears the
 // union bitmap of (b, hk) for the top-k kernel that follows.
 template <typename T, int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
     page_score_kernel(const T* __restrict__ q, const int32_t* __restrict__ active, int B, int Hq,
                       int G, int n_act, const T* __restrict__ pmin, const T* __restrict__ pmax,
                       const KvView kv, float* __restrict__ scores, uint32_t* __restrict__ bitmap,
                       int words, int cpc) {
   constexpr int PS = ps_stride<T, D>();
+  constexpr bool kSel = sizeof(T) == 2;  // bf16: masked-select bound, warp per row
   extern __shared__ __align__(16) float sm[];
   const int RQ = n_act * G;
-  float* qs = sm;                              // [RQ][D]
-  T* sbuf = reinterpret_cast<T*>(qs + RQ * D);  // 2 x ([kPsPages][PS] min, then max)
+  float* qs = sm;                                            // [RQ][D]
+  uint32_t* qm = reinterpret_cast<uint32_t*>(qs + RQ * D);   // [RQ][D/2] (bf16)
+  T* sbuf = reinterpret_cast<T*>(qm + (kSel ? RQ * (D / 2) : 0));  // 2 x ([64][PS] min, max)
   const int hk = blockIdx.y, b = blockIdx.z;
   if (blockIdx.x == 0)
     for (int w = threadIdx.x; w < words; w += blockDim.x)
@@ -339,34 +477,36 @@ __global__ void __launch_bounds__(256)
   const int c0 = blockIdx.x * cpc;
   const int c1 = min(c0 + cpc, (n_pages + kPsPages - 1) / kPsPages);
   if (c0 >= c1) return;
-  stage_page_chunk<T, D>(pmin, pmax, kv, b, hk, c0, n_pages, sbuf, sbuf + kPsPages * PS);
-  for (int idx = threadIdx.x; idx < RQ * D; idx += blockDim.x) {
-    const int rq = idx / D, c = idx - (idx / D) * D;
-    const int a_i = rq / G, g = rq - (rq / G) * G;
-    const int i = active ? active[b * n_act + a_i] : a_i;
-    qs[idx] = ld_f32<T>(q + (((long long)b * B + i) * Hq + hk * G + g) * D + c);
-  }
+  const PageRing<T, D> ring{sbuf, pmin, pmax, kv, b, hk, c0, c1, n_pages};
+  ring.prologue();
+  stage_q_rows<T, D>(q, active, b, B, Hq, G, hk, n_act, RQ, qs, qm);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, n_warps = blockDim.x >> 5;
   for (int ch = c0; ch < c1; ++ch) {
-    const int buf = (ch - c0) & 1;
-    T* smn = sbuf + buf * 2 * kPsPages * PS;
-    T* smx = smn + kPsPages * PS;
-    if (ch + 1 < c1) {
-      T* nmn = sbuf + (buf ^ 1) * 2 * kPsPages * PS;
-      stage_page_chunk<T, D>(pmin, pmax, kv, b, hk, ch + 1, n_pages, nmn, nmn + kPsPages * PS);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
+    ring.advance(ch);
+    const T* smn = ring.mn(ch);
+    const T* smx = ring.mx(ch);
     __syncthreads();  // chunk ch (and the q rows) visible to every thread
-    for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
-      const int pg = task % kPsPages, rq = task / kPsPages;
+    if constexpr (kSel) {
+      const int pg = (warp & 1) * 32 + lane;
       const int p = ch * kPsPages + pg;
-      if (p >= n_pages) continue;
-      const float yb = page_bound<T, D>(qs + rq * D, smn + pg * PS, smx + pg * PS);
-      const int a_i = rq / G, g = rq - (rq / G) * G;
-      scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = yb;
+      for (int rq = warp >> 1; rq < RQ; rq += n_warps >> 1) {
+        const float yb = page_bound_sel<D>(qs + rq * D, qm + rq * (D / 2), smn + pg * PS,
+                                           smx + pg * PS);
+        const int a_i = rq / G, g = rq - (rq / G) * G;
+        if (p < n_pages)
+          scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = yb;
+      }
+    } else {
+      for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
+        const int pg = task % kPsPages, rq = task / kPsPages;
+        const int p = ch * kPsPages + pg;
+        if (p >= n_pages) continue;
+        const float yb = page_bound<T, D>(qs + rq * D, smn + pg * PS, smx + pg * PS);
+        const int a_i = rq / G, g = rq - (rq / G) * G;
+        scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = yb;
+      }
     }
-    __syncthreads();  // buffer `buf` is refilled two chunks later
+    __syncthreads();  // this chunk's buffer is refilled in the next iteration
   }
 }
 
@@ -417,9 +557,18 @@ __global__ void __launch_bounds__(kTopkThreads)
     for (int d = tid; d < 256; d += blockDim.x) hist[d] = 0;
     __syncthreads();
     const uint32_t prefix = s_prefix;
-    for (int p = tid; p < n; p += blockDim.x) {
-      const uint32_t key = keys[p];
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
+    // Keys still matching the prefix land in their digit's bucket. Scores of
+    // one row are alike, so many keys share a digit (all of them in the first
+    // pass): the lanes of a warp holding the same digit add their count once.
+    for (int p0 = 0; p0 < n; p0 += blockDim.x) {
+      const int p = p0 + tid;
+      uint32_t dg = 256u;  // no bucket
+      if (p < n) {
+        const uint32_t key = keys[p];
+        if ((key & mask) == prefix) dg = (key >> shift) & 0xFFu;
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, dg);
+      if (dg < 256u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[dg], __popc(peers));
     }
     __syncthreads();
     if (tid < 32) {
@@ -548,17 +697,19 @@ __device__ __forceinline__ float order_key_inv(uint32_t k) {
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
     head_page_score_kernel(const T* __restrict__ q, int B, int Hq, int G,
                            const T* __restrict__ pmin, const T* __restrict__ pmax,
                            const KvView kv, float* __restrict__ scores,
                            uint32_t* __restrict__ bitmap, int words, int cpc) {
   constexpr int PS = ps_stride<T, D>();
+  constexpr bool kSel = sizeof(T) == 2;  // bf16: masked-select bound, warp per row
   extern __shared__ __align__(16) float sm[];
   __shared__ uint32_t best[kPsPages];
   const int RQ = B * G;
-  float* qs = sm;                               // [RQ][D], row r = i * G + g
-  T* sbuf = reinterpret_cast<T*>(qs + RQ * D);  // 2 x ([kPsPages][PS] min, then max)
+  float* qs = sm;                                            // [RQ][D], row r = i * G + g
+  uint32_t* qm = reinterpret_cast<uint32_t*>(qs + RQ * D);   // [RQ][D/2] (bf16)
+  T* sbuf = reinterpret_cast<T*>(qm + (kSel ? RQ * (D / 2) : 0));  // 2 x ([64][PS] min, max)
   const int hk = blockIdx.y, b = blockIdx.z;
   if (blockIdx.x == 0)
     for (int w = threadIdx.x; w < words; w += blockDim.x)
@@ -567,31 +718,31 @@ __global__ void __launch_bounds__(256)
   const int c0 = blockIdx.x * cpc;
   const int c1 = min(c0 + cpc, (n_pages + kPsPages - 1) / kPsPages);
   if (c0 >= c1) return;
-  stage_page_chunk<T, D>(pmin, pmax, kv, b, hk, c0, n_pages, sbuf, sbuf + kPsPages * PS);
-  for (int idx = threadIdx.x; idx < RQ * D; idx += blockDim.x) {
-    const int rq = idx / D, c = idx - (idx / D) * D;
-    const int i = rq / G, g = rq - (rq / G) * G;
-    qs[idx] = ld_f32<T>(q + (((long long)b * B + i) * Hq + hk * G + g) * D + c);
-  }
+  const PageRing<T, D> ring{sbuf, pmin, pmax, kv, b, hk, c0, c1, n_pages};
+  ring.prologue();
+  stage_q_rows<T, D>(q, nullptr, b, B, Hq, G, hk, B, RQ, qs, qm);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, n_warps = blockDim.x >> 5;
   for (int ch = c0; ch < c1; ++ch) {
-    const int buf = (ch - c0) & 1;
-    T* smn = sbuf + buf * 2 * kPsPages * PS;
-    T* smx = smn + kPsPages * PS;
     for (int pg = threadIdx.x; pg < kPsPages; pg += blockDim.x) best[pg] = 0u;  // below every key
-    if (ch + 1 < c1) {
-      T* nmn = sbuf + (buf ^ 1) * 2 * kPsPages * PS;
-      stage_page_chunk<T, D>(pmin, pmax, kv, b, hk, ch + 1, n_pages, nmn, nmn + kPsPages * PS);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
+    ring.advance(ch);
+    const T* smn = ring.mn(ch);
+    const T* smx = ring.mx(ch);
     __syncthreads();  // chunk ch, the q rows and the cleared maxima visible to every thread
-    for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
-      const int pg = task % kPsPages, rq = task / kPsPages;
-      const int p = ch * kPsPages + pg;
-      if (p >= n_pages) continue;
-      const float yb = page_bound<T, D>(qs + rq * D, smn + pg * PS, smx + pg * PS);
-      atomicMax(&best[pg], order_key(yb));
+    if constexpr (kSel) {
+      const int pg = (warp & 1) * 32 + lane;
+      uint32_t mx = 0u;  // below every key
+      for (int rq = warp >> 1; rq < RQ; rq += n_warps >> 1)
+        mx = max(mx, order_key(page_bound_sel<D>(qs + rq * D, qm + rq * (D / 2), smn + pg * PS,
+                                                  smx + pg * PS)));
+      if (ch * kPsPages + pg < n_pages) atomicMax(&best[pg], mx);
+    } else {
+      for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
+        const int pg = task % kPsPages, rq = task / kPsPages;
+        const int p = ch * kPsPages + pg;
+        if (p >= n_pages) continue;
+        const float yb = page_bound<T, D>(qs + rq * D, smn + pg * PS, smx + pg * PS);
+        atomicMax(&best[pg], order_key(yb));
+      }
     }
     __syncthreads();
     for (int pg = threadIdx.x; pg < kPsPages; pg += blockDim.x) {
@@ -599,7 +750,7 @@ __global__ void __launch_bounds__(256)
       if (p < n_pages)
         scores[((long long)b * kv.Hkv + hk) * kv.max_pages + p] = order_key_inv(best[pg]);
     }
-    __syncthreads();  // maxima read out, buffer `buf` free for chunk ch + 2
+    __syncthreads();  // maxima read out, this chunk's buffer free for the next iteration
   }
 }
 
