@@ -467,6 +467,8 @@ template <int D, int RG>
 __global__ void __launch_bounds__(kAttnThreads, 2)
     attn_bf16_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV) {
+  grid_dependency_wait();  // launched as a programmatic dependent
+  allow_dependent_launch();
   using S = Bf16Smem<D>;
   constexpr int KS = kNWC / RG;   // key slices
   constexpr int KW = kTK / KS;    // keys per warp per tile
@@ -510,9 +512,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  // Every CTA of this grid is resident from here on: let the split combine
-  // (launched as a programmatic dependent) be scheduled into the spare slots.
-  allow_dependent_launch();
 
   if (warp == kNWC) {
     // ----------------------------- producer -----------------------------
@@ -831,6 +830,8 @@ struct F32Smem {
 
 template <int D>
 __global__ void __launch_bounds__(128) attn_f32_kernel(const __grid_constant__ AttnArgs a) {
+  grid_dependency_wait();  // launched as a programmatic dependent
+  allow_dependent_launch();
   constexpr int NV = D / 32, KP = F32Smem<D>::KP, C4 = D / 4;
   extern __shared__ __align__(16) float fs[];
   float* Qs = fs;                   // [kF32Rows][D]
@@ -1007,6 +1008,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ At
   // Launched as a programmatic dependent of the partial kernel: wait until that
   // grid has completed and its partials are visible (no-op on a plain launch).
   grid_dependency_wait();
+  allow_dependent_launch();
   constexpr int NV = D / 32;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;

@@ -64,6 +64,8 @@ struct Tc2Smem {
 __global__ void __launch_bounds__(kT2Threads, 1)
     attn_tc2_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV) {
+  grid_dependency_wait();  // launched as a programmatic dependent
+  allow_dependent_launch();
   constexpr int D = 128;
   using S = Tc2Smem;
   __shared__ __align__(8) uint64_t full_bar[kT2Slots];

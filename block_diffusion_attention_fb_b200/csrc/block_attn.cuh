@@ -63,6 +63,8 @@ struct BlockSmem {
 // KT: key tiles of 16 (the block's B keys padded to 16 * KT <= 64).
 template <int D, int KT>
 __global__ void __launch_bounds__(128) block_attn_kernel(const __grid_constant__ BlockArgs a) {
+  grid_dependency_wait();  // launched as a programmatic dependent
+  allow_dependent_launch();
   using S = BlockSmem<D>;
   constexpr int NT = 2 * KT;  // n8 tiles of keys
   constexpr int KD = D / 16;  // k16 steps over the head dim
@@ -283,6 +285,8 @@ constexpr int block_f32_smem(int D, int R) { return 4 * D * (64 + R + 65); }
 
 template <int D>
 __global__ void __launch_bounds__(256) block_attn_f32_kernel(const __grid_constant__ BlockArgsF32 a) {
+  grid_dependency_wait();  // launched as a programmatic dependent
+  allow_dependent_launch();
   constexpr int NK = 64;       // keys staged (B <= 64)
   constexpr int KP = NK + 1;   // padded stride of the transposed keys: no bank conflicts
   extern __shared__ __align__(16) float fsm[];

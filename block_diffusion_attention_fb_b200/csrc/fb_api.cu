@@ -47,11 +47,38 @@ int fail(int code, const char* fmt, ...) {
   return code;
 }
 
+thread_local cudaError_t t_launch_error = cudaSuccess;  // of the last launch_pdl
+
 int check_launch(const char* what) {
-  const cudaError_t e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = t_launch_error;
+  t_launch_error = cudaSuccess;
   if (e != cudaSuccess) return fail(FB_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FB_OK;
+}
+
+// Launch as a programmatic dependent of the previous kernel on the stream: the
+// grid may be scheduled while its predecessor finishes (every kernel of this
+// library waits for its predecessor's results with griddepcontrol.wait before
+// touching memory, and lets its own dependents launch right after). Inside a
+// CUDA graph the edge stays programmatic. The error, if any, is reported by
+// the next check_launch.
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e != cudaSuccess) t_launch_error = e;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -438,7 +465,7 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
   do {                                                                            \
     auto kfn = attn_f32_kernel<DD>;                                               \
     if (int rc_ = set_smem_once((const void*)kfn, F32Smem<DD>::bytes)) return rc_; \
-    kfn<<<grid, 128, F32Smem<DD>::bytes, stream>>>(a);                            \
+    launch_pdl(kfn, grid, dim3(128), F32Smem<DD>::bytes, stream, a);              \
   } while (0)
     if (D == 128)
       FB_LAUNCH_F32(128);
@@ -456,11 +483,11 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
     auto kfn = attn_bf16_kernel<DD, RGV>;                                                    \
     const int smem = Bf16Smem<DD>::kBytes;                                                   \
     if (int rc_ = set_smem_once((const void*)kfn, smem)) return rc_;                       \
-    kfn<<<grid, kAttnThreads, smem, stream>>>(a, tk, tv);                                    \
+    launch_pdl(kfn, grid, dim3(kAttnThreads), smem, stream, a, tk, tv);                      \
   } while (0)
     if (use_tc(kv->dtype, D, a.R)) {
       if (int rc_ = set_smem_once((const void*)attn_tc2_kernel, Tc2Smem::kBytes)) return rc_;
-      attn_tc2_kernel<<<grid, kT2Threads, Tc2Smem::kBytes, stream>>>(a, tk, tv);
+      launch_pdl(attn_tc2_kernel, grid, dim3(kT2Threads), Tc2Smem::kBytes, stream, a, tk, tv);
     } else if (D == 128) {
       if (p.rg == 1)
         FB_LAUNCH_BF16(128, 1);
@@ -588,7 +615,7 @@ int block_attn_short(const void* q, const void* k_in, const void* v_in, int batc
   do {                                                                                 \
     auto kfn = block_attn_kernel<DD, KTV>;                                             \
     if (int rc_ = set_smem_once((const void*)kfn, smem_d)) return rc_;                \
-    kfn<<<grid, 32 * warps, smem_d, stream>>>(a);                                      \
+    launch_pdl(kfn, grid, dim3(32 * warps), smem_d, stream, a);                        \
   } while (0)
   if (D == 128) {
     switch (kt) {
@@ -640,7 +667,7 @@ int block_attn_short_f32(const void* q, const void* k_in, const void* v_in, int 
   do {                                                                   \
     auto kfn = block_attn_f32_kernel<DD>;                                \
     if (int rc_ = set_smem_once((const void*)kfn, smem)) return rc_;    \
-    kfn<<<dim3(Hkv, batch), 32 * warps, smem, stream>>>(a);              \
+    launch_pdl(kfn, dim3(Hkv, batch), dim3(32 * warps), smem, stream, a); \
   } while (0)
   if (D == 128)
     FB_BLOCK_F32_LAUNCH(128);
@@ -724,10 +751,9 @@ int sr_select(const void* q, int B, int Hq, const void* page_min, const void* pa
   do {                                                                                       \
     auto kfn = head_page_score_kernel<TT, DD>;                                               \
     if ((rc = set_smem_once((const void*)kfn, psm))) return rc;                            \
-    kfn<<<g2, 256, psm, stream>>>(static_cast<const TT*>(q), B, Hq, G,                       \
-                                  static_cast<const TT*>(page_min),                          \
-                                  static_cast<const TT*>(page_max), v, head_scores, bitmap,  \
-                                  words, cpc);                                               \
+    launch_pdl(kfn, g2, dim3(256), psm, stream, static_cast<const TT*>(q), B, Hq, G,        \
+               static_cast<const TT*>(page_min), static_cast<const TT*>(page_max), v,        \
+               head_scores, bitmap, words, cpc);                                             \
   } while (0)
   if (kv->dtype == FB_BF16) {
     if (D == 128) FB_HPS(__nv_bfloat16, 128); else FB_HPS(__nv_bfloat16, 64);
@@ -739,14 +765,14 @@ int sr_select(const void* q, int B, int Hq, const void* page_min, const void* pa
   const int ksm = v.max_pages * 4;
   if ((rc = set_smem_once((const void*)topk_pages_kernel, ksm))) return rc;
   // one "row" per kv head: scores [batch, 1, Hkv, pages], G = 1
-  topk_pages_kernel<<<dim3(v.Hkv, kv->batch), kTopkThreads, ksm, stream>>>(
-      head_scores, v, v.Hkv, 1, 1, topk, bitmap, words);
+  launch_pdl(topk_pages_kernel, dim3(v.Hkv, kv->batch), dim3(kTopkThreads), ksm, stream,
+             (const float*)head_scores, v, v.Hkv, 1, 1, topk, bitmap, words);
   if ((rc = check_launch("top-k pages kernel"))) return rc;
-  union_compact_kernel<<<dim3(v.Hkv, kv->batch), 256, 0, stream>>>(bitmap, words, v.Hkv,
-                                                                   v.max_pages, list, count);
+  launch_pdl(union_compact_kernel, dim3(v.Hkv, kv->batch), dim3(256), 0, stream,
+             (const uint32_t*)bitmap, words, v.Hkv, v.max_pages, list, count);
   if ((rc = check_launch("selection compaction kernel"))) return rc;
-  complement_compact_kernel<<<dim3(v.Hkv, kv->batch), 256, 0, stream>>>(
-      bitmap, words, v, v.max_pages, comp_list, comp_count);
+  launch_pdl(complement_compact_kernel, dim3(v.Hkv, kv->batch), dim3(256), 0, stream,
+             (const uint32_t*)bitmap, words, v, v.max_pages, comp_list, comp_count);
   return check_launch("complement compaction kernel");
 }
 
@@ -968,9 +994,8 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
   if (N2 >= 256 && N2 <= 256 * 32) {
     // register tree (E elements per thread)
 #define FB_LOC(TT, EE)                                                                         \
-  locality_score_reg_kernel<TT, EE><<<g1, 256, 0, stream>>>(static_cast<const TT*>(q_cur),     \
-                                                             static_cast<const TT*>(q_prev), B, \
-                                                             N, rs)
+  launch_pdl(locality_score_reg_kernel<TT, EE>, g1, dim3(256), 0, stream,                     \
+             static_cast<const TT*>(q_cur), static_cast<const TT*>(q_prev), B, N, rs)
 #define FB_LOC_E(TT)          \
   switch (N2 / 256) {         \
     case 1: FB_LOC(TT, 1); break;   \
@@ -993,16 +1018,18 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
              : set_smem_once((const void*)locality_score_kernel<float>, N2 * 4);
     if (rc) return rc;
     if (kv->dtype == FB_BF16)
-      locality_score_kernel<__nv_bfloat16><<<g1, 256, N2 * 4, stream>>>(
-          static_cast<const __nv_bfloat16*>(q_cur), static_cast<const __nv_bfloat16*>(q_prev), B,
-          N, N2, rs);
+      launch_pdl(locality_score_kernel<__nv_bfloat16>, g1, dim3(256), N2 * 4, stream,
+                 static_cast<const __nv_bfloat16*>(q_cur),
+                 static_cast<const __nv_bfloat16*>(q_prev), B, N, N2, rs);
     else
-      locality_score_kernel<float><<<g1, 256, N2 * 4, stream>>>(
-          static_cast<const float*>(q_cur), static_cast<const float*>(q_prev), B, N, N2, rs);
+      launch_pdl(locality_score_kernel<float>, g1, dim3(256), N2 * 4, stream,
+                 static_cast<const float*>(q_cur), static_cast<const float*>(q_prev), B, N, N2,
+                 rs);
   }
   rc = check_launch("locality score kernel");
   if (rc) return rc;
-  active_rows_kernel<<<kv->batch, 256, B * 4, stream>>>(rs, B, na, active_rows);
+  launch_pdl(active_rows_kernel, dim3(kv->batch), dim3(256), B * 4, stream, (const float*)rs, B,
+             na, active_rows);
   rc = check_launch("active rows kernel");
   if (rc) return rc;
   int cpc;
@@ -1011,29 +1038,28 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
   if (kv->dtype == FB_BF16) {
     auto kfn = D == 128 ? page_score_kernel<__nv_bfloat16, 128> : page_score_kernel<__nv_bfloat16, 64>;
     if ((rc = set_smem_once((const void*)kfn, psm))) return rc;
-    kfn<<<g2, 256, psm, stream>>>(static_cast<const __nv_bfloat16*>(q_cur), active_rows, B, Hq, G,
-                                  na, static_cast<const __nv_bfloat16*>(page_min),
-                                  static_cast<const __nv_bfloat16*>(page_max), v, page_scores,
-                                  union_bitmap, words, cpc);
+    launch_pdl(kfn, g2, dim3(256), psm, stream, static_cast<const __nv_bfloat16*>(q_cur),
+               (const int32_t*)active_rows, B, Hq, G, na,
+               static_cast<const __nv_bfloat16*>(page_min),
+               static_cast<const __nv_bfloat16*>(page_max), v, page_scores, union_bitmap, words,
+               cpc);
   } else {
     auto kfn = D == 128 ? page_score_kernel<float, 128> : page_score_kernel<float, 64>;
     if ((rc = set_smem_once((const void*)kfn, psm))) return rc;
-    kfn<<<g2, 256, psm, stream>>>(static_cast<const float*>(q_cur), active_rows, B, Hq, G, na,
-                                  static_cast<const float*>(page_min),
-                                  static_cast<const float*>(page_max), v, page_scores,
-                                  union_bitmap, words, cpc);
+    launch_pdl(kfn, g2, dim3(256), psm, stream, static_cast<const float*>(q_cur),
+               (const int32_t*)active_rows, B, Hq, G, na, static_cast<const float*>(page_min),
+               static_cast<const float*>(page_max), v, page_scores, union_bitmap, words, cpc);
   }
   rc = check_launch("page score kernel");
   if (rc) return rc;
   const int ksm = v.max_pages * 4;
   if ((rc = set_smem_once((const void*)topk_pages_kernel, ksm))) return rc;
-  topk_pages_kernel<<<dim3(na * Hq, kv->batch), kTopkThreads, ksm, stream>>>(
-      page_scores, v, Hq, G, na, topk_pages, union_bitmap, words);
+  launch_pdl(topk_pages_kernel, dim3(na * Hq, kv->batch), dim3(kTopkThreads), ksm, stream,
+             (const float*)page_scores, v, Hq, G, na, topk_pages, union_bitmap, words);
   rc = check_launch("top-k pages kernel");
   if (rc) return rc;
-  union_compact_kernel<<<dim3(v.Hkv, kv->batch), 256, 0, stream>>>(union_bitmap, words, v.Hkv,
-                                                                   v.max_pages, union_list,
-                                                                   union_count);
+  launch_pdl(union_compact_kernel, dim3(v.Hkv, kv->batch), dim3(256), 0, stream,
+             (const uint32_t*)union_bitmap, words, v.Hkv, v.max_pages, union_list, union_count);
   return check_launch("union compaction kernel");
 }
 

@@ -114,6 +114,8 @@ template <typename T>
 __global__ void __launch_bounds__(256)
     locality_score_kernel(const T* __restrict__ qc, const T* __restrict__ qp, int B, int N,
                           int N2, float* __restrict__ score) {
+  grid_dependency_wait();  // launched as a programmatic dependent
+  allow_dependent_launch();
   extern __shared__ float xs[];  // N2 floats
   const int i = blockIdx.x, b = blockIdx.y;
   const long long off = ((long long)b * B + i) * N;
@@ -141,6 +143,8 @@ template <typename T, int E>
 __global__ void __launch_bounds__(256)
     locality_score_reg_kernel(const T* __restrict__ qc, const T* __restrict__ qp, int B, int N,
                               float* __restrict__ score) {
+  grid_dependency_wait();  // launched as a programmatic dependent
+  allow_dependent_launch();
   __shared__ float red[256];
   const int i = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
   const long long off = ((long long)b * B + i) * N;
@@ -182,6 +186,8 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(256)
     active_rows_kernel(const float* __restrict__ score, int B, int n_act,
                        int32_t* __restrict__ active) {
+  grid_dependency_wait();  // launched as a programmatic dependent
+  allow_dependent_launch();
   extern __shared__ float sc[];
   const int b = blockIdx.x;
   for (int i = threadIdx.x; i < B; i += blockDim.x) sc[i] = score[(long long)b * B + i];
@@ -462,6 +468,8 @@ __global__ void __launch_bounds__(256, 2)
                       int G, int n_act, const T* __restrict__ pmin, const T* __restrict__ pmax,
                       const KvView kv, float* __restrict__ scores, uint32_t* __restrict__ bitmap,
                       int words, int cpc) {
+  grid_dependency_wait();  // launched as a programmatic dependent
+  allow_dependent_launch();
   constexpr int PS = ps_stride<T, D>();
   constexpr bool kSel = sizeof(T) == 2;  // bf16: masked-select bound, warp per row
   extern __shared__ __align__(16) float sm[];
@@ -528,6 +536,8 @@ constexpr int kTopkThreads = 512;
 __global__ void __launch_bounds__(kTopkThreads)
     topk_pages_kernel(const float* __restrict__ scores, const KvView kv, int Hq, int G, int n_act,
                       int topk, uint32_t* __restrict__ bitmap, int words) {
+  grid_dependency_wait();  // launched as a programmatic dependent
+  allow_dependent_launch();
   extern __shared__ uint32_t keys[];  // max_pages
   __shared__ int hist[256];
   __shared__ int seg_cnt[kTopkThreads];
@@ -651,6 +661,8 @@ __global__ void __launch_bounds__(kTopkThreads)
 __global__ void __launch_bounds__(256)
     union_compact_kernel(const uint32_t* __restrict__ bitmap, int words, int Hkv, int stride,
                          int32_t* __restrict__ list, int32_t* __restrict__ count) {
+  grid_dependency_wait();  // launched as a programmatic dependent
+  allow_dependent_launch();
   __shared__ int wsum[256];
   const int hk = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const uint32_t* bm = bitmap + ((long long)b * Hkv + hk) * words;
@@ -702,6 +714,8 @@ __global__ void __launch_bounds__(256, 2)
                            const T* __restrict__ pmin, const T* __restrict__ pmax,
                            const KvView kv, float* __restrict__ scores,
                            uint32_t* __restrict__ bitmap, int words, int cpc) {
+  grid_dependency_wait();  // launched as a programmatic dependent
+  allow_dependent_launch();
   constexpr int PS = ps_stride<T, D>();
   constexpr bool kSel = sizeof(T) == 2;  // bf16: masked-select bound, warp per row
   extern __shared__ __align__(16) float sm[];
@@ -760,6 +774,8 @@ __global__ void __launch_bounds__(256)
     complement_compact_kernel(const uint32_t* __restrict__ bitmap, int words, const KvView kv,
                               int stride, int32_t* __restrict__ list,
                               int32_t* __restrict__ count) {
+  grid_dependency_wait();  // launched as a programmatic dependent
+  allow_dependent_launch();
   __shared__ int wsum[256];
   const int hk = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int n_pages = (kv_tokens(kv, b) + kv.page_size - 1) / kv.page_size;
