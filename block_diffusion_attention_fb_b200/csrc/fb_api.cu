@@ -171,6 +171,19 @@ struct Plan {
 // HBM-bound). fp32 runs on the CUDA-core kernel.
 bool use_tc(fb_dtype dt, int D, int R) { return dt == FB_BF16 && D == 128 && R > 64; }
 
+// Of every 8 key pairs, how many the tcgen05 softmax exponentiates on the FMA
+// pipe by default (FB_TC_POLY overrides).
+constexpr int kTcPolyDefault = 0;
+
+int tc_poly() {
+  const char* e = getenv("FB_TC_POLY");
+  if (e && *e) {
+    const int v = atoi(e);
+    if (v == 0 || v == 2 || v == 3 || v == 4) return v;
+  }
+  return kTcPolyDefault;
+}
+
 int tc_splits(long long units, int slots, int max_tiles, int batch) {
   if (const int forced = env_int("FB_TC_SPLITS", 1, 4096)) return forced;
   // cost in key-tile times: waves x (tiles per CTA + start-up) + combine reads
@@ -486,8 +499,13 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
     launch_pdl(kfn, grid, dim3(kAttnThreads), smem, stream, a, tk, tv);                      \
   } while (0)
     if (use_tc(kv->dtype, D, a.R)) {
-      if (int rc_ = set_smem_once((const void*)attn_tc2_kernel, Tc2Smem::kBytes)) return rc_;
-      launch_pdl(attn_tc2_kernel, grid, dim3(kT2Threads), Tc2Smem::kBytes, stream, a, tk, tv);
+      // exponentials moved to the FMA pipe per 8 key pairs (FB_TC_POLY: 0, 2, 3 or 4)
+      const int poly = tc_poly();
+      auto kfn = poly == 0 ? attn_tc2_kernel<0>
+                           : (poly == 2 ? attn_tc2_kernel<2>
+                                        : (poly == 3 ? attn_tc2_kernel<3> : attn_tc2_kernel<4>));
+      if (int rc_ = set_smem_once((const void*)kfn, Tc2Smem::kBytes)) return rc_;
+      launch_pdl(kfn, grid, dim3(kT2Threads), Tc2Smem::kBytes, stream, a, tk, tv);
     } else if (D == 128) {
       if (p.rg == 1)
         FB_LAUNCH_BF16(128, 1);
@@ -563,15 +581,18 @@ KvView kv_view(const fb_kv* kv) {
 }
 
 // Page scoring grid: chunks of kPsPages pages per (sequence, kv head), `cpc`
-// consecutive chunks per CTA so that about two CTAs per SM cover the chunks
-// (each CTA's next chunk then loads while it scores the current one).
-dim3 page_score_grid(const KvView& v, int num_sms, int& cpc) {
+// consecutive chunks per CTA so that the grid is ONE wave of the CTAs an SM
+// holds at this shared-memory size (up to two): a second, partial wave would
+// double the time of the chunks it runs.
+dim3 page_score_grid(const KvView& v, int num_sms, int smem_bytes, int& cpc) {
   const int chunks = ceil_div(v.max_pages, kPsPages);
   const long long groups = (long long)v.batch * v.Hkv;
-  const long long slots = 2LL * (num_sms > 0 ? num_sms : 148);
+  const int per_sm = smem_bytes + 1024 <= (227 * 1024) / 2 ? 2 : 1;
+  const long long slots = (long long)per_sm * (num_sms > 0 ? num_sms : 148);
   cpc = (int)((groups * chunks + slots - 1) / slots);
   if (cpc < 1) cpc = 1;
   if (cpc > chunks) cpc = chunks;
+  while (cpc < chunks && (long long)ceil_div(chunks, cpc) * groups > slots) ++cpc;
   return dim3(ceil_div(chunks, cpc), v.Hkv, v.batch);
 }
 
@@ -743,9 +764,9 @@ int sr_select(const void* q, int B, int Hq, const void* page_min, const void* pa
   if (!aligned16(page_min) || !aligned16(page_max))
     return fail(FB_ERR_ALIGN, "page summaries not 16-byte aligned");
   int cpc;
-  const dim3 g2 = page_score_grid(v, sm_count(), cpc);
   const int es = (int)elem_size(kv->dtype);
   const int psm = page_score_smem(RQ, D, es);
+  const dim3 g2 = page_score_grid(v, sm_count(), psm, cpc);
   int rc;
 #define FB_HPS(TT, DD)                                                                       \
   do {                                                                                       \
@@ -1033,8 +1054,8 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
   rc = check_launch("active rows kernel");
   if (rc) return rc;
   int cpc;
-  const dim3 g2 = page_score_grid(v, num_sms, cpc);
   const int psm = page_score_smem(na * G, D, (int)elem_size(kv->dtype));
+  const dim3 g2 = page_score_grid(v, num_sms, psm, cpc);
   if (kv->dtype == FB_BF16) {
     auto kfn = D == 128 ? page_score_kernel<__nv_bfloat16, 128> : page_score_kernel<__nv_bfloat16, 64>;
     if ((rc = set_smem_once((const void*)kfn, psm))) return rc;

@@ -567,18 +567,9 @@ __global__ void __launch_bounds__(kTopkThreads)
     for (int d = tid; d < 256; d += blockDim.x) hist[d] = 0;
     __syncthreads();
     const uint32_t prefix = s_prefix;
-    // Keys still matching the prefix land in their digit's bucket. Scores of
-    // one row are alike, so many keys share a digit (all of them in the first
-    // pass): the lanes of a warp holding the same digit add their count once.
-    for (int p0 = 0; p0 < n; p0 += blockDim.x) {
-      const int p = p0 + tid;
-      uint32_t dg = 256u;  // no bucket
-      if (p < n) {
-        const uint32_t key = keys[p];
-        if ((key & mask) == prefix) dg = (key >> shift) & 0xFFu;
-      }
-      const unsigned peers = __match_any_sync(0xffffffffu, dg);
-      if (dg < 256u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[dg], __popc(peers));
+    for (int p = tid; p < n; p += blockDim.x) {
+      const uint32_t key = keys[p];
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
     }
     __syncthreads();
     if (tid < 32) {
