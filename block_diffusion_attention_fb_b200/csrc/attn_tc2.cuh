@@ -61,9 +61,6 @@ struct Tc2Smem {
   static constexpr int kBytes = 1024 + 2 * kQTile + kT2Slots * kKVTile;
 };
 
-// kPoly: of every 8 key pairs of a row, how many take their exponentials on
-// the FMA pipe (exp2_poly2) instead of the exponential unit.
-template <int kPoly>
 __global__ void __launch_bounds__(kT2Threads, 1)
     attn_tc2_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV) {
@@ -414,12 +411,8 @@ __global__ void __launch_bounds__(kT2Threads, 1)
         for (int k = 0; k < 16; ++k) {
           const float2 xx = ffma2(make_float2(sv[c * 32 + 2 * k], sv[c * 32 + 2 * k + 1]), sc2, nb2);
           float2 pp;
-          if ((k & 7) < kPoly) {
-            pp = exp2_poly2(xx);
-          } else {
-            pp.x = fast_exp2(xx.x);
-            pp.y = fast_exp2(xx.y);
-          }
+          pp.x = fast_exp2(xx.x);
+          pp.y = fast_exp2(xx.y);
           lc = fadd2(lc, pp);
           pk[k] = pack_bf16(pp.x, pp.y);
         }

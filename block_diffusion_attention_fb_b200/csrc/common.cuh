@@ -178,36 +178,6 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
 }
-// 2^x for a pair on the FMA pipe (packed f32x2), for softmax loops whose
-// exponential unit is the busiest pipe. Range reduction: n = floor(x) by a
-// round-toward-minus-infinity add of 1.5 * 2^23 (n then sits in the low
-// mantissa bits of the sum), f = x - n in [0, 1); 2^f by a cubic, and 2^n
-// joined by adding n to the exponent field. The cubic was fitted in this
-// repository to 2^f on [0, 1) by weighted least squares on Chebyshev nodes,
-// iterated toward equal relative error (Lawson); its largest relative error is
-// 7.5e-5 (the bf16 rounding P goes through afterwards is 2^-9 = 2.0e-3).
-// x is clamped to >= -126 first, so -inf (a masked key) gives 2^-126 * p(0),
-// about 1.2e-38, instead of a NaN.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kC0 = 0.99992522f, kC1 = 0.69583354f, kC2 = 0.22606716f, kC3 = 0.07802452f;
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  float2 j;
-  asm("{.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\t"
-      "add.rm.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(j.x), "=f"(j.y)
-      : "f"(x.x), "f"(x.y), "f"(12582912.f));
-  const float2 n = fadd2(j, make_float2(-12582912.f, -12582912.f));  // floor(x), exact
-  const float2 f = fadd2(x, make_float2(-n.x, -n.y));
-  float2 p = ffma2(f, make_float2(kC3, kC3), make_float2(kC2, kC2));
-  p = ffma2(p, f, make_float2(kC1, kC1));
-  p = ffma2(p, f, make_float2(kC0, kC0));
-  // the low mantissa bits of j hold n; 1.5 * 2^23 shifted left by 23 is 0 mod 2^32
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(j.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(j.y) << 23)));
-}
-
 // max(a, b, c) in one instruction (sm_100 three-input max)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;

@@ -171,19 +171,6 @@ struct Plan {
 // HBM-bound). fp32 runs on the CUDA-core kernel.
 bool use_tc(fb_dtype dt, int D, int R) { return dt == FB_BF16 && D == 128 && R > 64; }
 
-// Of every 8 key pairs, how many the tcgen05 softmax exponentiates on the FMA
-// pipe by default (FB_TC_POLY overrides).
-constexpr int kTcPolyDefault = 0;
-
-int tc_poly() {
-  const char* e = getenv("FB_TC_POLY");
-  if (e && *e) {
-    const int v = atoi(e);
-    if (v == 0 || v == 2 || v == 3 || v == 4) return v;
-  }
-  return kTcPolyDefault;
-}
-
 int tc_splits(long long units, int slots, int max_tiles, int batch) {
   if (const int forced = env_int("FB_TC_SPLITS", 1, 4096)) return forced;
   // cost in key-tile times: waves x (tiles per CTA + start-up) + combine reads
@@ -270,7 +257,7 @@ size_t partial_ws_bytes(fb_dtype dt, int batch, int Hkv, int R, int D, int max_t
 
 // Workspace regions shared by every entry point (offsets in bytes).
 struct WsLayout {
-  size_t part, scores, cos, a_in, l_in, total;
+  size_t part, scores, tickets, cos, a_in, l_in, total;
 };
 
 int logical_pages(const fb_kv* kv) {
@@ -289,7 +276,7 @@ WsLayout ws_layout(const fb_kv* kv, int B, int Hq, int n_active, int topk, int n
   const int R = B * G;
   size_t part = partial_ws_bytes(kv->dtype, kv->batch, kv->n_heads_kv, R, D,
                                  ceil_div(kv->max_seq_len, kTK), num_sms);
-  size_t scores = 0;
+  size_t scores = 0, tickets = 0;
   if (n_active > 0 && topk > 0) {
     const int na = n_active < B ? n_active : B;
     const int per_tile = kTK / (kv->page_size < kTK ? kv->page_size : kTK);
@@ -299,13 +286,15 @@ WsLayout ws_layout(const fb_kv* kv, int B, int Hq, int n_active, int topk, int n
     part = part > pgb ? part : pgb;
     scores = round_up((size_t)kv->batch * na * Hq * logical_pages(kv) * 4, 256) +
              round_up((size_t)kv->batch * B * 4, 256);
+    tickets = round_up((size_t)kv->batch * kv->n_heads_kv * 4, 256);  // top-k group tickets
   }
   const int P = next_pow2(B * D);
   const int T1 = P < kCosT1Max ? P : kCosT1Max;
   const size_t cosb = round_up((size_t)kv->batch * Hq * 3 * T1 * 8, 256);
   w.part = 0;
   w.scores = w.part + part;
-  w.cos = w.scores + scores;
+  w.tickets = w.scores + scores;
+  w.cos = w.tickets + tickets;
   w.a_in = w.cos + cosb;
   w.l_in = w.a_in + round_up((size_t)kv->batch * B * Hq * D * 4, 256);
   w.total = w.l_in + round_up((size_t)kv->batch * B * Hq * 4, 256);
@@ -499,13 +488,8 @@ int launch_partial(const PartialCall& c, cudaStream_t stream) {
     launch_pdl(kfn, grid, dim3(kAttnThreads), smem, stream, a, tk, tv);                      \
   } while (0)
     if (use_tc(kv->dtype, D, a.R)) {
-      // exponentials moved to the FMA pipe per 8 key pairs (FB_TC_POLY: 0, 2, 3 or 4)
-      const int poly = tc_poly();
-      auto kfn = poly == 0 ? attn_tc2_kernel<0>
-                           : (poly == 2 ? attn_tc2_kernel<2>
-                                        : (poly == 3 ? attn_tc2_kernel<3> : attn_tc2_kernel<4>));
-      if (int rc_ = set_smem_once((const void*)kfn, Tc2Smem::kBytes)) return rc_;
-      launch_pdl(kfn, grid, dim3(kT2Threads), Tc2Smem::kBytes, stream, a, tk, tv);
+      if (int rc_ = set_smem_once((const void*)attn_tc2_kernel, Tc2Smem::kBytes)) return rc_;
+      launch_pdl(attn_tc2_kernel, grid, dim3(kT2Threads), Tc2Smem::kBytes, stream, a, tk, tv);
     } else if (D == 128) {
       if (p.rg == 1)
         FB_LAUNCH_BF16(128, 1);
@@ -754,7 +738,7 @@ int block_attn_impl(const void* q, const void* k_in, const void* v_in, int batch
 // sequence into comp_list / comp_count.
 int sr_select(const void* q, int B, int Hq, const void* page_min, const void* page_max,
               const fb_kv* kv, int topk, uint32_t* bitmap, int32_t* list, int32_t* count,
-              int32_t* comp_list, int32_t* comp_count, float* head_scores,
+              int32_t* comp_list, int32_t* comp_count, float* head_scores, int* tickets,
               cudaStream_t stream) {
   const KvView v = kv_view(kv);
   const int D = v.D, G = Hq / v.Hkv, RQ = B * G;
@@ -774,7 +758,7 @@ int sr_select(const void* q, int B, int Hq, const void* page_min, const void* pa
     if ((rc = set_smem_once((const void*)kfn, psm))) return rc;                            \
     launch_pdl(kfn, g2, dim3(256), psm, stream, static_cast<const TT*>(q), B, Hq, G,        \
                static_cast<const TT*>(page_min), static_cast<const TT*>(page_max), v,        \
-               head_scores, bitmap, words, cpc);                                             \
+               head_scores, bitmap, words, tickets, cpc);                                    \
   } while (0)
   if (kv->dtype == FB_BF16) {
     if (D == 128) FB_HPS(__nv_bfloat16, 128); else FB_HPS(__nv_bfloat16, 64);
@@ -783,15 +767,14 @@ int sr_select(const void* q, int B, int Hq, const void* page_min, const void* pa
   }
 #undef FB_HPS
   if ((rc = check_launch("head page score kernel"))) return rc;
-  const int ksm = v.max_pages * 4;
+  const int ksm = (v.max_pages + words) * 4;
   if ((rc = set_smem_once((const void*)topk_pages_kernel, ksm))) return rc;
-  // one "row" per kv head: scores [batch, 1, Hkv, pages], G = 1
+  // one "row" per kv head: scores [batch, 1, Hkv, pages], G = 1; each CTA is its
+  // own group and compacts its selection
   launch_pdl(topk_pages_kernel, dim3(v.Hkv, kv->batch), dim3(kTopkThreads), ksm, stream,
-             (const float*)head_scores, v, v.Hkv, 1, 1, topk, bitmap, words);
+             (const float*)head_scores, v, v.Hkv, 1, 1, topk, bitmap, words, list, count,
+             v.max_pages, tickets);
   if ((rc = check_launch("top-k pages kernel"))) return rc;
-  launch_pdl(union_compact_kernel, dim3(v.Hkv, kv->batch), dim3(256), 0, stream,
-             (const uint32_t*)bitmap, words, v.Hkv, v.max_pages, list, count);
-  if ((rc = check_launch("selection compaction kernel"))) return rc;
   launch_pdl(complement_compact_kernel, dim3(v.Hkv, kv->batch), dim3(256), 0, stream,
              (const uint32_t*)bitmap, words, v, v.max_pages, comp_list, comp_count);
   return check_launch("complement compaction kernel");
@@ -998,6 +981,7 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
                 workspace_bytes);
   char* ws = static_cast<char*>(workspace);
   float* page_scores = reinterpret_cast<float*>(ws + w.scores);
+  int* tickets = reinterpret_cast<int*>(ws + w.tickets);
   float* rs = row_scores
                   ? row_scores
                   : reinterpret_cast<float*>(ws + w.scores +
@@ -1049,39 +1033,44 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
   }
   rc = check_launch("locality score kernel");
   if (rc) return rc;
-  launch_pdl(active_rows_kernel, dim3(kv->batch), dim3(256), B * 4, stream, (const float*)rs, B,
-             na, active_rows);
-  rc = check_launch("active rows kernel");
-  if (rc) return rc;
+  // Up to 32 active rows are picked inside the page scorer (every CTA of a
+  // sequence from the same locality scores); more take the rank kernel.
+  const bool pick_in_scorer = na <= 32;
+  if (!pick_in_scorer) {
+    launch_pdl(active_rows_kernel, dim3(kv->batch), dim3(256), B * 4, stream, (const float*)rs,
+               B, na, active_rows);
+    rc = check_launch("active rows kernel");
+    if (rc) return rc;
+  }
+  const int32_t* act_in = pick_in_scorer ? nullptr : active_rows;
+  const float* rs_in = pick_in_scorer ? rs : nullptr;
   int cpc;
-  const int psm = page_score_smem(na * G, D, (int)elem_size(kv->dtype));
+  const int psm = page_score_smem(na * G, D, (int)elem_size(kv->dtype)) + (pick_in_scorer ? B * 4 : 0);
   const dim3 g2 = page_score_grid(v, num_sms, psm, cpc);
   if (kv->dtype == FB_BF16) {
     auto kfn = D == 128 ? page_score_kernel<__nv_bfloat16, 128> : page_score_kernel<__nv_bfloat16, 64>;
     if ((rc = set_smem_once((const void*)kfn, psm))) return rc;
-    launch_pdl(kfn, g2, dim3(256), psm, stream, static_cast<const __nv_bfloat16*>(q_cur),
-               (const int32_t*)active_rows, B, Hq, G, na,
-               static_cast<const __nv_bfloat16*>(page_min),
+    launch_pdl(kfn, g2, dim3(256), psm, stream, static_cast<const __nv_bfloat16*>(q_cur), act_in,
+               rs_in, active_rows, B, Hq, G, na, static_cast<const __nv_bfloat16*>(page_min),
                static_cast<const __nv_bfloat16*>(page_max), v, page_scores, union_bitmap, words,
-               cpc);
+               tickets, cpc);
   } else {
     auto kfn = D == 128 ? page_score_kernel<float, 128> : page_score_kernel<float, 64>;
     if ((rc = set_smem_once((const void*)kfn, psm))) return rc;
-    launch_pdl(kfn, g2, dim3(256), psm, stream, static_cast<const float*>(q_cur),
-               (const int32_t*)active_rows, B, Hq, G, na, static_cast<const float*>(page_min),
-               static_cast<const float*>(page_max), v, page_scores, union_bitmap, words, cpc);
+    launch_pdl(kfn, g2, dim3(256), psm, stream, static_cast<const float*>(q_cur), act_in, rs_in,
+               active_rows, B, Hq, G, na, static_cast<const float*>(page_min),
+               static_cast<const float*>(page_max), v, page_scores, union_bitmap, words, tickets,
+               cpc);
   }
   rc = check_launch("page score kernel");
   if (rc) return rc;
-  const int ksm = v.max_pages * 4;
+  // top-k per (active row, q head); the last CTA of each kv head compacts the union
+  const int ksm = (v.max_pages + words) * 4;
   if ((rc = set_smem_once((const void*)topk_pages_kernel, ksm))) return rc;
   launch_pdl(topk_pages_kernel, dim3(na * Hq, kv->batch), dim3(kTopkThreads), ksm, stream,
-             (const float*)page_scores, v, Hq, G, na, topk_pages, union_bitmap, words);
-  rc = check_launch("top-k pages kernel");
-  if (rc) return rc;
-  launch_pdl(union_compact_kernel, dim3(v.Hkv, kv->batch), dim3(256), 0, stream,
-             (const uint32_t*)union_bitmap, words, v.Hkv, v.max_pages, union_list, union_count);
-  return check_launch("union compaction kernel");
+             (const float*)page_scores, v, Hq, G, na, topk_pages, union_bitmap, words, union_list,
+             union_count, v.max_pages, tickets);
+  return check_launch("top-k pages kernel");
 }
 
 int losa_gather(const void* q, int32_t B, int32_t n_heads_q, const int32_t* active_rows,
@@ -1215,7 +1204,8 @@ static int step_impl(const fb_policy* policy, fb_cache* cache, const void* q, co
     if (refresh) {
       rc = sr_select(q, B, Hq, page_min, page_max, prefix, policy->topk_pages,
                      cache->union_bitmap, cache->union_list, cache->union_count, cache->comp_list,
-                     cache->comp_count, reinterpret_cast<float*>(ws + w.scores), stream);
+                     cache->comp_count, reinterpret_cast<float*>(ws + w.scores),
+                     reinterpret_cast<int*>(ws + w.tickets), stream);
       if (rc) return rc;
       PartialCall cr = c;  // residual: every row over the unselected pages
       cr.page_list = cache->comp_list;

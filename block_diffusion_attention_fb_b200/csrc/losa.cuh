@@ -183,6 +183,45 @@ __global__ void __launch_bounds__(256)
 // of a block-wide maximum over the key (order-preserving score bits, ~row), so
 // a higher score wins and equal scores go to the lower row; more active rows:
 // O(B^2) ranks. Scores are sums of squares, never NaN.
+//
+// The rounds, for one sequence, by the whole CTA (blockDim a multiple of 32,
+// at most 1024): score_b [B] from global, sc [B] shared scratch, taken [32]
+// receives the rows in rank order (shared). Every thread returns after the
+// last round's barrier, so taken[] is visible to all.
+__device__ __forceinline__ void pick_active_rows(const float* score_b, int B, int n_act,
+                                                 float* sc, int* taken) {
+  __shared__ unsigned long long wbest[32];
+  for (int i = threadIdx.x; i < B; i += blockDim.x) sc[i] = score_b[i];
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int r = 0; r < n_act; ++r) {
+    unsigned long long best = 0ull;
+    for (int i = threadIdx.x; i < B; i += blockDim.x) {
+      bool used = false;
+      for (int t = 0; t < r; ++t) used |= (taken[t] == i);
+      if (used) continue;
+      const float f = sc[i] == 0.f ? 0.f : sc[i];  // -0 and +0 rank equal
+      const uint32_t u = __float_as_uint(f);
+      const uint32_t key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+      const unsigned long long k = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)i);
+      best = k > best ? k : best;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+      best = other > best ? other : best;
+    }
+    if (lane == 0) wbest[wid] = best;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      unsigned long long m = 0ull;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = wbest[w] > m ? wbest[w] : m;
+      taken[r] = (int)(0xFFFFFFFFu - (uint32_t)(m & 0xFFFFFFFFull));
+    }
+    __syncthreads();
+  }
+}
+
 __global__ void __launch_bounds__(256)
     active_rows_kernel(const float* __restrict__ score, int B, int n_act,
                        int32_t* __restrict__ active) {
@@ -190,42 +229,14 @@ __global__ void __launch_bounds__(256)
   allow_dependent_launch();
   extern __shared__ float sc[];
   const int b = blockIdx.x;
-  for (int i = threadIdx.x; i < B; i += blockDim.x) sc[i] = score[(long long)b * B + i];
-  __syncthreads();
   if (n_act <= 32) {
-    __shared__ unsigned long long wbest[8];
     __shared__ int taken[32];
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    for (int r = 0; r < n_act; ++r) {
-      unsigned long long best = 0ull;
-      for (int i = threadIdx.x; i < B; i += blockDim.x) {
-        bool used = false;
-        for (int t = 0; t < r; ++t) used |= (taken[t] == i);
-        if (used) continue;
-        const float f = sc[i] == 0.f ? 0.f : sc[i];  // -0 and +0 rank equal
-        const uint32_t u = __float_as_uint(f);
-        const uint32_t key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-        const unsigned long long k = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)i);
-        best = k > best ? k : best;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
-        best = other > best ? other : best;
-      }
-      if (lane == 0) wbest[wid] = best;
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        unsigned long long m = 0ull;
-        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = wbest[w] > m ? wbest[w] : m;
-        const int row = (int)(0xFFFFFFFFu - (uint32_t)(m & 0xFFFFFFFFull));
-        taken[r] = row;
-        active[b * n_act + r] = row;
-      }
-      __syncthreads();
-    }
+    pick_active_rows(score + (long long)b * B, B, n_act, sc, taken);
+    for (int r = threadIdx.x; r < n_act; r += blockDim.x) active[b * n_act + r] = taken[r];
     return;
   }
+  for (int i = threadIdx.x; i < B; i += blockDim.x) sc[i] = score[(long long)b * B + i];
+  __syncthreads();
   for (int i = threadIdx.x; i < B; i += blockDim.x) {
     const float si = sc[i];
     int rank = 0;
@@ -381,14 +392,16 @@ __host__ __device__ constexpr int page_score_smem(int RQ, int D, int elem_bytes)
 
 // Stages the active q rows of (b, hk) as float, and for bf16 the per-channel
 // sign masks of page_bound_sel: qs [RQ][D], qm [RQ][D/2].
+// act: the n_act active rows of sequence b (global or shared), or NULL for
+// rows 0 .. n_act-1.
 template <typename T, int D>
-__device__ __forceinline__ void stage_q_rows(const T* q, const int32_t* active, int b, int B,
+__device__ __forceinline__ void stage_q_rows(const T* q, const int* act, int b, int B,
                                              int Hq, int G, int hk, int n_act, int RQ, float* qs,
                                              uint32_t* qm) {
   for (int idx = threadIdx.x; idx < RQ * D; idx += blockDim.x) {
     const int rq = idx / D, c = idx - (idx / D) * D;
     const int a_i = rq / G, g = rq - (rq / G) * G;
-    const int i = active ? active[b * n_act + a_i] : a_i;
+    const int i = act ? act[a_i] : a_i;
     qs[idx] = ld_f32<T>(q + (((long long)b * B + i) * Hq + hk * G + g) * D + c);
   }
   if constexpr (sizeof(T) == 2) {
@@ -461,33 +474,51 @@ struct PageRing {
 // page_bound_sel; float32: one thread per (page, row) by page_bound. Both are
 // single-rounded products and the stride-halving tree.
 // scores: [batch, n_act, Hq, max_pages]. Block (0, hk, b) also clears the
-// union bitmap of (b, hk) for the top-k kernel that follows.
+// union bitmap of (b, hk) and its ticket for the top-k kernel that follows.
+// Active rows: given (active), or picked here from the locality scores
+// row_scores [batch, B] (n_act <= 32; every CTA of a sequence picks the same
+// rows, block (0, 0, b) writes them to active_out).
 template <typename T, int D>
 __global__ void __launch_bounds__(256, 2)
-    page_score_kernel(const T* __restrict__ q, const int32_t* __restrict__ active, int B, int Hq,
-                      int G, int n_act, const T* __restrict__ pmin, const T* __restrict__ pmax,
-                      const KvView kv, float* __restrict__ scores, uint32_t* __restrict__ bitmap,
-                      int words, int cpc) {
+    page_score_kernel(const T* __restrict__ q, const int32_t* __restrict__ active,
+                      const float* __restrict__ row_scores, int32_t* __restrict__ active_out,
+                      int B, int Hq, int G, int n_act, const T* __restrict__ pmin,
+                      const T* __restrict__ pmax, const KvView kv, float* __restrict__ scores,
+                      uint32_t* __restrict__ bitmap, int words, int* __restrict__ tickets,
+                      int cpc) {
   grid_dependency_wait();  // launched as a programmatic dependent
   allow_dependent_launch();
   constexpr int PS = ps_stride<T, D>();
   constexpr bool kSel = sizeof(T) == 2;  // bf16: masked-select bound, warp per row
   extern __shared__ __align__(16) float sm[];
+  __shared__ int s_active[32];
   const int RQ = n_act * G;
   float* qs = sm;                                            // [RQ][D]
   uint32_t* qm = reinterpret_cast<uint32_t*>(qs + RQ * D);   // [RQ][D/2] (bf16)
-  T* sbuf = reinterpret_cast<T*>(qm + (kSel ? RQ * (D / 2) : 0));  // 2 x ([64][PS] min, max)
+  T* sbuf = reinterpret_cast<T*>(qm + (kSel ? RQ * (D / 2) : 0));  // stages of [64][PS] min, max
+  float* sc = reinterpret_cast<float*>(sbuf + 2 * ps_stages((int)sizeof(T)) * kPsPages * PS);
   const int hk = blockIdx.y, b = blockIdx.z;
-  if (blockIdx.x == 0)
+  if (blockIdx.x == 0) {
     for (int w = threadIdx.x; w < words; w += blockDim.x)
       bitmap[((long long)b * kv.Hkv + hk) * words + w] = 0u;
+    if (tickets && threadIdx.x == 0) tickets[b * kv.Hkv + hk] = 0;
+  }
   const int n_pages = (kv_tokens(kv, b) + kv.page_size - 1) / kv.page_size;
   const int c0 = blockIdx.x * cpc;
   const int c1 = min(c0 + cpc, (n_pages + kPsPages - 1) / kPsPages);
-  if (c0 >= c1) return;
+  const bool pick = row_scores != nullptr;
+  if (c0 >= c1 && !(pick && blockIdx.x == 0 && hk == 0)) return;
+  const int* act = active ? active + b * n_act : nullptr;
+  if (pick) {
+    pick_active_rows(row_scores + (long long)b * B, B, n_act, sc, s_active);
+    if (blockIdx.x == 0 && hk == 0)
+      for (int r = threadIdx.x; r < n_act; r += blockDim.x) active_out[b * n_act + r] = s_active[r];
+    if (c0 >= c1) return;
+    act = s_active;
+  }
   const PageRing<T, D> ring{sbuf, pmin, pmax, kv, b, hk, c0, c1, n_pages};
   ring.prologue();
-  stage_q_rows<T, D>(q, active, b, B, Hq, G, hk, n_act, RQ, qs, qm);
+  stage_q_rows<T, D>(q, act, b, B, Hq, G, hk, n_act, RQ, qs, qm);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, n_warps = blockDim.x >> 5;
   for (int ch = c0; ch < c1; ++ch) {
     ring.advance(ch);
@@ -528,161 +559,186 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 // ---------------------------------------------------------------------------
 // Step 3b: top-k pages of one (active row, q head): exact radix select of the
 // k-th largest key (4 passes of 8 bits), then every key above it plus the
-// lowest-index keys equal to it. The picks are OR-ed into the union bitmap of
-// the kv head. One CTA of kTopkThreads per (b, a, h).
+// lowest-index keys equal to it. The picks are gathered in a shared bitmap and
+// OR-ed into the union bitmap of the kv head one word at a time. One CTA of
+// kTopkThreads per (b, a, h).
+// Step 3c: the last of the n_act * G CTAs of a (b, hk) to finish (a ticket
+// that the page scorer zeroed) turns the union bitmap into the ascending page
+// list and count.
 // ---------------------------------------------------------------------------
 constexpr int kTopkThreads = 512;
 
-__global__ void __launch_bounds__(kTopkThreads)
-    topk_pages_kernel(const float* __restrict__ scores, const KvView kv, int Hq, int G, int n_act,
-                      int topk, uint32_t* __restrict__ bitmap, int words) {
-  grid_dependency_wait();  // launched as a programmatic dependent
-  allow_dependent_launch();
-  extern __shared__ uint32_t keys[];  // max_pages
-  __shared__ int hist[256];
-  __shared__ int seg_cnt[kTopkThreads];
-  __shared__ uint32_t s_prefix;
-  __shared__ int s_need;
-  const int ah = blockIdx.x, b = blockIdx.y;
-  const int h = ah % Hq;
-  const int hk = h / G;
-  const int tid = threadIdx.x;
-  const int n = (kv_tokens(kv, b) + kv.page_size - 1) / kv.page_size;
-  const int k = min(topk, n);
-  uint32_t* bm = bitmap + ((long long)b * kv.Hkv + hk) * words;
-  const float* sc = scores + ((long long)b * n_act * Hq + ah) * kv.max_pages;
-  if (k <= 0) return;
-  if (k == n) {
-    for (int p = tid; p < n; p += blockDim.x) atomicOr(&bm[p >> 5], 1u << (p & 31));
-    return;
-  }
-  for (int p = tid; p < n; p += blockDim.x) keys[p] = order_key(sc[p]);
-  if (tid == 0) {
-    s_prefix = 0u;
-    s_need = k;
-  }
-  uint32_t mask = 0u;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int d = tid; d < 256; d += blockDim.x) hist[d] = 0;
-    __syncthreads();
-    const uint32_t prefix = s_prefix;
-    for (int p = tid; p < n; p += blockDim.x) {
-      const uint32_t key = keys[p];
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
-    }
-    __syncthreads();
-    if (tid < 32) {
-      // buckets in descending order: lane l owns digits 255-8l ... 248-8l
-      int cnt[8], tot = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        cnt[j] = hist[255 - 8 * tid - j];
-        tot += cnt[j];
-      }
-      int incl = tot;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (tid >= o) incl += v;
-      }
-      const int need = s_need;
-      const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
-      const int owner = __ffs(hit) - 1;  // first lane whose running count reaches need
-      if (tid == owner) {
-        int cum = incl - tot, sel = 0, rem = need;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (cum + cnt[j] >= need) {
-            sel = 255 - 8 * tid - j;
-            rem = need - cum;
-            break;
-          }
-          cum += cnt[j];
-        }
-        s_prefix = prefix | ((uint32_t)sel << shift);
-        s_need = rem;
-      }
-    }
-    mask |= 0xFFu << shift;
-    __syncthreads();
-  }
-  const uint32_t T = s_prefix;  // key of the k-th largest score
-  const int need = s_need;      // how many keys equal to T are taken
-  // keys equal to T: take the lowest indices, via a scan of per-thread segments
-  const int seg = (n + kTopkThreads - 1) / kTopkThreads;
-  const int p0 = tid * seg, p1 = min(n, p0 + seg);
-  int cnt = 0;
-  for (int p = p0; p < p1; ++p) cnt += (keys[p] == T);
-  // exclusive scan of the per-thread counts (thread order = index order)
-  const int lane = tid & 31, wid = tid >> 5;
-  int incl = cnt;
+// Exclusive prefix sum over the CTA (blockDim a multiple of 32, at most 1024)
+// of one value per thread; total receives the sum. Ends with a barrier.
+__device__ __forceinline__ int block_exclusive_scan(int x, int* warp_sums, int& total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int incl = x;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int v = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += v;
   }
-  if (lane == 31) seg_cnt[wid] = incl;
+  if (lane == 31) warp_sums[wid] = incl;
   __syncthreads();
   if (wid == 0) {
-    const int nw = kTopkThreads / 32;
-    int x = lane < nw ? seg_cnt[lane] : 0;
-    int wi = x;
+    const int w = lane < nw ? warp_sums[lane] : 0;
+    int wi = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, wi, o);
       if (lane >= o) wi += v;
     }
-    if (lane < nw) seg_cnt[lane] = wi - x;  // exclusive warp offsets
+    if (lane < nw) warp_sums[lane] = wi - w;
+    if (lane == 31) warp_sums[32] = wi;
   }
   __syncthreads();
-  int eq_before = seg_cnt[wid] + incl - cnt;
-  for (int p = p0; p < p1; ++p) {
-    const uint32_t key = keys[p];
-    bool take = key > T;
-    if (key == T) {
-      take = eq_before < need;
-      ++eq_before;
-    }
-    if (take) atomicOr(&bm[p >> 5], 1u << (p & 31));
-  }
+  total = warp_sums[32];
+  const int res = warp_sums[wid] + incl - x;
+  __syncthreads();  // warp_sums may be reused by the caller
+  return res;
 }
 
-// Step 3c: union bitmap -> ascending page list and count per (b, hk).
-__global__ void __launch_bounds__(256)
-    union_compact_kernel(const uint32_t* __restrict__ bitmap, int words, int Hkv, int stride,
-                         int32_t* __restrict__ list, int32_t* __restrict__ count) {
-  grid_dependency_wait();  // launched as a programmatic dependent
-  allow_dependent_launch();
-  __shared__ int wsum[256];
-  const int hk = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const uint32_t* bm = bitmap + ((long long)b * Hkv + hk) * words;
-  int32_t* out = list + ((long long)b * Hkv + hk) * stride;
-  const int per = (words + 255) / 256;
-  const int w0 = tid * per, w1 = min(words, w0 + per);
+// Bitmap (words, read through L2) -> ascending list of set bits and their count.
+__device__ __forceinline__ void compact_bitmap(const uint32_t* bm, int words, int32_t* out,
+                                               int32_t* count, int* warp_sums) {
+  const int per = (words + blockDim.x - 1) / blockDim.x;
+  const int w0 = threadIdx.x * per, w1 = min(words, w0 + per);
   int c = 0;
-  for (int w = w0; w < w1; ++w) c += __popc(bm[w]);
-  wsum[tid] = c;
-  __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int t = 0; t < 256; ++t) {
-      const int x = wsum[t];
-      wsum[t] = run;
-      run += x;
-    }
-    count[b * Hkv + hk] = run;
-  }
-  __syncthreads();
-  int pos = wsum[tid];
+  for (int w = w0; w < w1; ++w) c += __popc(__ldcg(bm + w));
+  int total;
+  int pos = block_exclusive_scan(c, warp_sums, total);
+  if (threadIdx.x == 0) *count = total;
   for (int w = w0; w < w1; ++w) {
-    uint32_t bits = bm[w];
+    uint32_t bits = __ldcg(bm + w);
     while (bits) {
       const int bit = __ffs(bits) - 1;
       bits &= bits - 1;
       out[pos++] = w * 32 + bit;
     }
   }
+}
+
+__global__ void __launch_bounds__(kTopkThreads)
+    topk_pages_kernel(const float* __restrict__ scores, const KvView kv, int Hq, int G, int n_act,
+                      int topk, uint32_t* __restrict__ bitmap, int words,
+                      int32_t* __restrict__ list, int32_t* __restrict__ count, int list_stride,
+                      int* __restrict__ tickets) {
+  grid_dependency_wait();  // launched as a programmatic dependent
+  allow_dependent_launch();
+  extern __shared__ uint32_t keys[];  // max_pages keys, then a words-long bitmap
+  __shared__ int hist[256];
+  __shared__ int warp_sums[33];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_need, s_last;
+  const int ah = blockIdx.x, b = blockIdx.y;
+  const int h = ah % Hq;
+  const int hk = h / G;
+  const int tid = threadIdx.x;
+  const int n = (kv_tokens(kv, b) + kv.page_size - 1) / kv.page_size;
+  const int k = min(topk, n);
+  uint32_t* sbm = keys + kv.max_pages;
+  uint32_t* bm = bitmap + ((long long)b * kv.Hkv + hk) * words;
+  const float* sc = scores + ((long long)b * n_act * Hq + ah) * kv.max_pages;
+  for (int w = tid; w < words; w += blockDim.x) sbm[w] = 0u;
+  auto take = [&](int p) { atomicOr(&sbm[p >> 5], 1u << (p & 31)); };
+  if (k == n) {
+    __syncthreads();
+    for (int p = tid; p < n; p += blockDim.x) take(p);
+  } else if (k > 0) {
+    for (int p = tid; p < n; p += blockDim.x) keys[p] = order_key(sc[p]);
+    if (tid == 0) {
+      s_prefix = 0u;
+      s_need = k;
+    }
+    uint32_t mask = 0u;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      for (int d = tid; d < 256; d += blockDim.x) hist[d] = 0;
+      __syncthreads();
+      const uint32_t prefix = s_prefix;
+      for (int p = tid; p < n; p += blockDim.x) {
+        const uint32_t key = keys[p];
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
+      }
+      __syncthreads();
+      if (tid < 32) {
+        // buckets in descending order: lane l owns digits 255-8l ... 248-8l
+        int cnt[8], tot = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          cnt[j] = hist[255 - 8 * tid - j];
+          tot += cnt[j];
+        }
+        int incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (tid >= o) incl += v;
+        }
+        const int need = s_need;
+        const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
+        const int owner = __ffs(hit) - 1;  // first lane whose running count reaches need
+        if (tid == owner) {
+          int cum = incl - tot, sel = 0, rem = need;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (cum + cnt[j] >= need) {
+              sel = 255 - 8 * tid - j;
+              rem = need - cum;
+              break;
+            }
+            cum += cnt[j];
+          }
+          s_prefix = prefix | ((uint32_t)sel << shift);
+          s_need = rem;
+        }
+      }
+      mask |= 0xFFu << shift;
+      __syncthreads();
+    }
+    const uint32_t T = s_prefix;  // key of the k-th largest score
+    const int need = s_need;      // how many keys equal to T are taken
+    // every key above T; count the keys equal to it
+    int eq = 0;
+    for (int p = tid; p < n; p += blockDim.x) {
+      const uint32_t key = keys[p];
+      if (key > T) take(p);
+      eq += key == T;
+    }
+    int n_eq;
+    block_exclusive_scan(eq, warp_sums, n_eq);
+    if (n_eq == need) {
+      for (int p = tid; p < n; p += blockDim.x)
+        if (keys[p] == T) take(p);
+    } else {
+      // more keys equal the k-th largest than are taken: the lowest indices,
+      // from a scan over per-thread index segments (thread order = index order)
+      const int seg = (n + blockDim.x - 1) / blockDim.x;
+      const int p0 = tid * seg, p1 = min(n, p0 + seg);
+      int cnt = 0;
+      for (int p = p0; p < p1; ++p) cnt += (keys[p] == T);
+      int tot;
+      int eq_before = block_exclusive_scan(cnt, warp_sums, tot);
+      for (int p = p0; p < p1; ++p) {
+        if (keys[p] == T) {
+          if (eq_before < need) take(p);
+          ++eq_before;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  for (int w = tid; w < words; w += blockDim.x)
+    if (sbm[w]) atomicOr(&bm[w], sbm[w]);
+  // the last CTA of the (b, hk) group compacts the union
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(&tickets[b * kv.Hkv + hk], 1) == n_act * G - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  compact_bitmap(bm, words, list + ((long long)b * kv.Hkv + hk) * list_stride,
+                 count + b * kv.Hkv + hk, warp_sums);
 }
 
 // ---------------------------------------------------------------------------
@@ -704,7 +760,8 @@ __global__ void __launch_bounds__(256, 2)
     head_page_score_kernel(const T* __restrict__ q, int B, int Hq, int G,
                            const T* __restrict__ pmin, const T* __restrict__ pmax,
                            const KvView kv, float* __restrict__ scores,
-                           uint32_t* __restrict__ bitmap, int words, int cpc) {
+                           uint32_t* __restrict__ bitmap, int words, int* __restrict__ tickets,
+                           int cpc) {
   grid_dependency_wait();  // launched as a programmatic dependent
   allow_dependent_launch();
   constexpr int PS = ps_stride<T, D>();
@@ -716,9 +773,11 @@ __global__ void __launch_bounds__(256, 2)
   uint32_t* qm = reinterpret_cast<uint32_t*>(qs + RQ * D);   // [RQ][D/2] (bf16)
   T* sbuf = reinterpret_cast<T*>(qm + (kSel ? RQ * (D / 2) : 0));  // 2 x ([64][PS] min, max)
   const int hk = blockIdx.y, b = blockIdx.z;
-  if (blockIdx.x == 0)
+  if (blockIdx.x == 0) {
     for (int w = threadIdx.x; w < words; w += blockDim.x)
       bitmap[((long long)b * kv.Hkv + hk) * words + w] = 0u;
+    if (tickets && threadIdx.x == 0) tickets[b * kv.Hkv + hk] = 0;
+  }
   const int n_pages = (kv_tokens(kv, b) + kv.page_size - 1) / kv.page_size;
   const int c0 = blockIdx.x * cpc;
   const int c1 = min(c0 + cpc, (n_pages + kPsPages - 1) / kPsPages);
