@@ -752,20 +752,13 @@ int sr_select(const void* q, int B, int Hq, const void* page_min, const void* pa
   const int psm = page_score_smem(RQ, D, es);
   const dim3 g2 = page_score_grid(v, sm_count(), psm, cpc);
   int rc;
-  CUtensorMap tmn{}, tmx{};  // bf16: the summaries staged by TMA in 64-page boxes
-  if (kv->dtype == FB_BF16) {
-    if ((rc = make_tmap(&tmn, page_min, D, v.Hkv, (long long)kv->batch * v.max_pages, kPsPages)))
-      return rc;
-    if ((rc = make_tmap(&tmx, page_max, D, v.Hkv, (long long)kv->batch * v.max_pages, kPsPages)))
-      return rc;
-  }
 #define FB_HPS(TT, DD)                                                                       \
   do {                                                                                       \
     auto kfn = head_page_score_kernel<TT, DD>;                                               \
     if ((rc = set_smem_once((const void*)kfn, psm))) return rc;                            \
     launch_pdl(kfn, g2, dim3(256), psm, stream, static_cast<const TT*>(q), B, Hq, G,        \
                static_cast<const TT*>(page_min), static_cast<const TT*>(page_max), v,        \
-               head_scores, bitmap, words, tickets, cpc, tmn, tmx);                          \
+               head_scores, bitmap, words, tickets, cpc);                                    \
   } while (0)
   if (kv->dtype == FB_BF16) {
     if (D == 128) FB_HPS(__nv_bfloat16, 128); else FB_HPS(__nv_bfloat16, 64);
@@ -1056,27 +1049,20 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
   const dim3 g2 = page_score_grid(v, num_sms, psm, cpc);
   // bf16: a warp scores two q rows over 32 pages, so 64 threads per row pair
   const int ps_threads = min(256, 64 * ceil_div(na * G, 2));
-  CUtensorMap tmn{}, tmx{};  // bf16: the summaries staged by TMA in 64-page boxes
-  if (kv->dtype == FB_BF16) {
-    if ((rc = make_tmap(&tmn, page_min, D, v.Hkv, (long long)kv->batch * v.max_pages, kPsPages)))
-      return rc;
-    if ((rc = make_tmap(&tmx, page_max, D, v.Hkv, (long long)kv->batch * v.max_pages, kPsPages)))
-      return rc;
-  }
   if (kv->dtype == FB_BF16) {
     auto kfn = D == 128 ? page_score_kernel<__nv_bfloat16, 128> : page_score_kernel<__nv_bfloat16, 64>;
     if ((rc = set_smem_once((const void*)kfn, psm))) return rc;
     launch_pdl(kfn, g2, dim3(ps_threads), psm, stream, static_cast<const __nv_bfloat16*>(q_cur), act_in,
                rs_in, active_rows, B, Hq, G, na, static_cast<const __nv_bfloat16*>(page_min),
                static_cast<const __nv_bfloat16*>(page_max), v, page_scores, union_bitmap, words,
-               tickets, cpc, tmn, tmx);
+               tickets, cpc);
   } else {
     auto kfn = D == 128 ? page_score_kernel<float, 128> : page_score_kernel<float, 64>;
     if ((rc = set_smem_once((const void*)kfn, psm))) return rc;
     launch_pdl(kfn, g2, dim3(256), psm, stream, static_cast<const float*>(q_cur), act_in, rs_in,
                active_rows, B, Hq, G, na, static_cast<const float*>(page_min),
                static_cast<const float*>(page_max), v, page_scores, union_bitmap, words, tickets,
-               cpc, tmn, tmx);
+               cpc);
   }
   rc = check_launch("page score kernel");
   if (rc) return rc;

@@ -324,13 +324,10 @@ __device__ __forceinline__ float page_bound(const float* qr, const T* mnr, const
 // definition. q rows qr (float) and qm are read by every lane of the warp at the
 // same address (broadcast); mnr / mxr are this lane's page.
 template <int D>
-__device__ __forceinline__ uint4 ld_page16(const uint8_t* buf, int p, int ch0);
-
-template <int D>
 __device__ __forceinline__ void page_bound_sel2(const float* qr0, const uint32_t* qm0,
                                                 const float* qr1, const uint32_t* qm1,
-                                                const uint8_t* mn, const uint8_t* mx, int p,
-                                                float (&out)[2]) {
+                                                const __nv_bfloat16* mnr,
+                                                const __nv_bfloat16* mxr, float (&out)[2]) {
   // Two q rows against one page: the page's minima and maxima of a group of
   // channels are read from shared memory once and serve both rows (the
   // shared-memory pipe, not the arithmetic, limits this loop).
@@ -350,8 +347,8 @@ __device__ __forceinline__ void page_bound_sel2(const float* qr0, const uint32_t
     uint32_t nn[8][4], xx[8][4];  // this lane's page: channels c8 + k E .. + 7, as bf16 pairs
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const uint4 n = ld_page16<D>(mn, p, c8 + k * E);
-      const uint4 x = ld_page16<D>(mx, p, c8 + k * E);
+      const uint4 n = *reinterpret_cast<const uint4*>(mnr + c8 + k * E);
+      const uint4 x = *reinterpret_cast<const uint4*>(mxr + c8 + k * E);
       nn[k][0] = n.x; nn[k][1] = n.y; nn[k][2] = n.z; nn[k][3] = n.w;
       xx[k][0] = x.x; xx[k][1] = x.y; xx[k][2] = x.z; xx[k][3] = x.w;
     }
@@ -405,14 +402,9 @@ __device__ __forceinline__ void page_bound_sel2(const float* qr0, const uint32_t
 
 // Shared memory of the page scorers for RQ staged q rows: the rows (float),
 // their sign masks (bf16 inputs), and two buffers of a chunk's summaries.
-// bf16: 1024 bytes of alignment slack, three TMA stages of 2 x (D / 64) boxes of
-// 64 pages x 128 bytes, the q rows and their sign masks; float32: the q rows
-// and the cp.async chunk ring.
 __host__ __device__ constexpr int page_score_smem(int RQ, int D, int elem_bytes) {
-  return elem_bytes == 2
-             ? 1024 + 3 * 2 * (D / 64) * kPsPages * 128 + RQ * D * 4 + RQ * (D / 2) * 4
-             : RQ * D * 4 + 2 * ps_stages(elem_bytes) * kPsPages * (D + 16 / elem_bytes) *
-                                elem_bytes;
+  return RQ * D * 4 + (elem_bytes == 2 ? RQ * (D / 2) * 4 : 0) +
+         2 * ps_stages(elem_bytes) * kPsPages * (D + 16 / elem_bytes) * elem_bytes;
 }
 
 // Stages the active q rows of (b, hk) as float, and for bf16 the per-channel
@@ -489,71 +481,6 @@ struct PageRing {
   }
 };
 
-// bf16 summaries reach shared memory by TMA: per chunk, one box of 64 pages x
-// 64 channels (128-byte swizzled rows, 8 KB) per half of the channels, for the
-// minima and the maxima, completing on the stage's mbarrier. A 16-byte load of
-// channels [8c, 8c+8) of page p (within its half) sits at p * 128 + ((c ^ (p & 7))
-// << 4): the 8 lanes of a quarter warp (consecutive pages) hit distinct banks.
-// Thread 0 issues; every thread waits (bounded). Chunk ch goes to stage
-// (ch - c0) % kStages, refilled only after the loop's trailing barrier.
-template <int D>
-struct TmaPageRing {
-  static constexpr int kStages = 3;
-  static constexpr int kHalf = kPsPages * 128;            // one 64-channel box
-  static constexpr int kStageBytes = 2 * (D / 64) * kHalf;  // minima, then maxima
-  uint8_t* base;  // 1024-byte aligned
-  uint64_t* bar;  // [kStages]
-  const CUtensorMap* tmn;
-  const CUtensorMap* tmx;
-  int* abort_flag;
-  int b, hk, c0, c1, max_pages;
-  __device__ uint8_t* mn(int ch) const { return base + ((ch - c0) % kStages) * kStageBytes; }
-  __device__ uint8_t* mx(int ch) const { return mn(ch) + (D / 64) * kHalf; }
-  __device__ void issue(int ch) const {  // thread 0
-    if (ch >= c1) return;
-    uint64_t* fb = &bar[(ch - c0) % kStages];
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // earlier reads of the buffer
-    mbar_arrive_expect_tx(fb, kStageBytes);
-    const int z = b * max_pages + ch * kPsPages;
-#pragma unroll
-    for (int h = 0; h < D / 64; ++h) {
-      tma_load_3d(mn(ch) + h * kHalf, tmn, h * 64, hk, z, fb);
-      tma_load_3d(mx(ch) + h * kHalf, tmx, h * 64, hk, z, fb);
-    }
-  }
-  __device__ void init() const {  // thread 0, before the first barrier of the CTA
-    for (int i = 0; i < kStages; ++i) mbar_init(&bar[i], 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __device__ void prologue() const {  // thread 0
-    for (int k = 0; k < kStages - 1; ++k) issue(c0 + k);
-  }
-  __device__ void advance(int ch) const {
-    if (threadIdx.x == 0) issue(ch + kStages - 1);
-    const int i = ch - c0;
-    mbar_wait(&bar[i % kStages], (i / kStages) & 1, abort_flag);
-  }
-  // after an abandoned wait: no copy may still be landing when the CTA exits
-  __device__ void drain(int ch_next) const {  // thread 0
-    const long long t0 = clock64();
-    for (int ch = ch_next; ch < c1 && ch < ch_next + kStages - 1; ++ch) {
-      const int i = ch - c0;
-      while (!mbar_try_wait(&bar[i % kStages], (i / kStages) & 1) &&
-             clock64() - t0 < kWaitBudgetCycles) {
-      }
-    }
-  }
-};
-
-// 16 bytes (8 bf16 channels from channel ch0, a multiple of 8) of page p of a
-// TMA-staged half-split buffer
-template <int D>
-__device__ __forceinline__ uint4 ld_page16(const uint8_t* buf, int p, int ch0) {
-  const int h = ch0 >> 6, c = (ch0 & 63) >> 3;
-  return *reinterpret_cast<const uint4*>(buf + h * TmaPageRing<D>::kHalf + p * 128 +
-                                         ((c ^ (p & 7)) << 4));
-}
-
 // Step 3a: QUEST-style page scores u_p = tree_sum_c max(q_c kmin_c, q_c kmax_c)
 // for every active row a and q head h of kv head hk. A CTA scores `cpc`
 // consecutive chunks of 64 pages of one (b, hk): the active q rows once into
@@ -575,25 +502,18 @@ __global__ void __launch_bounds__(256, 2)
                       int B, int Hq, int G, int n_act, const T* __restrict__ pmin,
                       const T* __restrict__ pmax, const KvView kv, float* __restrict__ scores,
                       uint32_t* __restrict__ bitmap, int words, int* __restrict__ tickets,
-                      int cpc, const __grid_constant__ CUtensorMap tmMin,
-                      const __grid_constant__ CUtensorMap tmMax) {
+                      int cpc) {
   grid_dependency_wait();  // launched as a programmatic dependent
   allow_dependent_launch();
   constexpr int PS = ps_stride<T, D>();
-  constexpr bool kSel = sizeof(T) == 2;  // bf16: TMA-staged summaries, masked-select bound
-  extern __shared__ uint8_t dsm[];
+  constexpr bool kSel = sizeof(T) == 2;  // bf16: masked-select bound, warp per row
+  extern __shared__ __align__(16) float sm[];
   __shared__ int s_active[32];
-  __shared__ __align__(8) uint64_t tma_bar[TmaPageRing<D>::kStages];
-  __shared__ int abort_flag;
   const int RQ = n_act * G;
-  uint8_t* tbase = dsm + ((1024u - (smem_u32(dsm) & 1023u)) & 1023u);  // TMA stages (bf16)
-  float* qs = kSel ? reinterpret_cast<float*>(tbase + TmaPageRing<D>::kStages *
-                                                          TmaPageRing<D>::kStageBytes)
-                   : reinterpret_cast<float*>(dsm);           // [RQ][D]
+  float* qs = sm;                                            // [RQ][D]
   uint32_t* qm = reinterpret_cast<uint32_t*>(qs + RQ * D);   // [RQ][D/2] (bf16)
-  T* sbuf = reinterpret_cast<T*>(qm + (kSel ? RQ * (D / 2) : 0));  // f32: stages of [64][PS]
-  float* sc = kSel ? reinterpret_cast<float*>(qm + RQ * (D / 2))
-                   : reinterpret_cast<float*>(sbuf + 2 * ps_stages((int)sizeof(T)) * kPsPages * PS);
+  T* sbuf = reinterpret_cast<T*>(qm + (kSel ? RQ * (D / 2) : 0));  // stages of [64][PS] min, max
+  float* sc = reinterpret_cast<float*>(sbuf + 2 * ps_stages((int)sizeof(T)) * kPsPages * PS);
   const int hk = blockIdx.y, b = blockIdx.z;
   if (blockIdx.x == 0) {
     for (int w = threadIdx.x; w < words; w += blockDim.x)
@@ -614,24 +534,11 @@ __global__ void __launch_bounds__(256, 2)
     act = s_active;
   }
   const PageRing<T, D> ring{sbuf, pmin, pmax, kv, b, hk, c0, c1, n_pages};
-  const TmaPageRing<D> tring{tbase, tma_bar, &tmMin, &tmMax, &abort_flag, b, hk, c0, c1,
-                             kv.max_pages};
-  if constexpr (kSel) {
-    if (threadIdx.x == 0) {
-      abort_flag = 0;
-      tring.init();
-      prefetch_tmap(&tmMin);
-      prefetch_tmap(&tmMax);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) tring.prologue();
-  } else {
-    ring.prologue();
-  }
+  ring.prologue();
   stage_q_rows<T, D>(q, act, b, B, Hq, G, hk, n_act, RQ, qs, qm);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, n_warps = blockDim.x >> 5;
   for (int ch = c0; ch < c1; ++ch) {
-    if constexpr (kSel) tring.advance(ch); else ring.advance(ch);
+    ring.advance(ch);
     const T* smn = ring.mn(ch);
     const T* smx = ring.mx(ch);
     __syncthreads();  // chunk ch (and the q rows) visible to every thread
@@ -643,7 +550,7 @@ __global__ void __launch_bounds__(256, 2)
         const int rq1 = rq + 1 < RQ ? rq + 1 : rq;
         float yb[2];
         page_bound_sel2<D>(qs + rq * D, qm + rq * (D / 2), qs + rq1 * D, qm + rq1 * (D / 2),
-                           tring.mn(ch), tring.mx(ch), pg, yb);
+                           smn + pg * PS, smx + pg * PS, yb);
         if (p < n_pages) {
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
@@ -665,10 +572,6 @@ __global__ void __launch_bounds__(256, 2)
       }
     }
     __syncthreads();  // this chunk's buffer is refilled in the next iteration
-  }
-  if constexpr (kSel) {
-    // a wait that gave up may have left copies in flight: let them land
-    if (threadIdx.x == 0 && abort_flag) tring.drain(max(c0, c1 - (TmaPageRing<D>::kStages - 1)));
   }
 }
 
@@ -884,23 +787,17 @@ __global__ void __launch_bounds__(256, 2)
                            const T* __restrict__ pmin, const T* __restrict__ pmax,
                            const KvView kv, float* __restrict__ scores,
                            uint32_t* __restrict__ bitmap, int words, int* __restrict__ tickets,
-                           int cpc, const __grid_constant__ CUtensorMap tmMin,
-                           const __grid_constant__ CUtensorMap tmMax) {
+                           int cpc) {
   grid_dependency_wait();  // launched as a programmatic dependent
   allow_dependent_launch();
   constexpr int PS = ps_stride<T, D>();
-  constexpr bool kSel = sizeof(T) == 2;  // bf16: TMA-staged summaries, masked-select bound
-  extern __shared__ uint8_t dsm[];
+  constexpr bool kSel = sizeof(T) == 2;  // bf16: masked-select bound, warp per row
+  extern __shared__ __align__(16) float sm[];
   __shared__ uint32_t best[kPsPages];
-  __shared__ __align__(8) uint64_t tma_bar[TmaPageRing<D>::kStages];
-  __shared__ int abort_flag;
   const int RQ = B * G;
-  uint8_t* tbase = dsm + ((1024u - (smem_u32(dsm) & 1023u)) & 1023u);  // TMA stages (bf16)
-  float* qs = kSel ? reinterpret_cast<float*>(tbase + TmaPageRing<D>::kStages *
-                                                          TmaPageRing<D>::kStageBytes)
-                   : reinterpret_cast<float*>(dsm);           // [RQ][D], row r = i * G + g
+  float* qs = sm;                                            // [RQ][D], row r = i * G + g
   uint32_t* qm = reinterpret_cast<uint32_t*>(qs + RQ * D);   // [RQ][D/2] (bf16)
-  T* sbuf = reinterpret_cast<T*>(qm + (kSel ? RQ * (D / 2) : 0));  // f32: stages of [64][PS]
+  T* sbuf = reinterpret_cast<T*>(qm + (kSel ? RQ * (D / 2) : 0));  // 2 x ([64][PS] min, max)
   const int hk = blockIdx.y, b = blockIdx.z;
   if (blockIdx.x == 0) {
     for (int w = threadIdx.x; w < words; w += blockDim.x)
@@ -912,25 +809,12 @@ __global__ void __launch_bounds__(256, 2)
   const int c1 = min(c0 + cpc, (n_pages + kPsPages - 1) / kPsPages);
   if (c0 >= c1) return;
   const PageRing<T, D> ring{sbuf, pmin, pmax, kv, b, hk, c0, c1, n_pages};
-  const TmaPageRing<D> tring{tbase, tma_bar, &tmMin, &tmMax, &abort_flag, b, hk, c0, c1,
-                             kv.max_pages};
-  if constexpr (kSel) {
-    if (threadIdx.x == 0) {
-      abort_flag = 0;
-      tring.init();
-      prefetch_tmap(&tmMin);
-      prefetch_tmap(&tmMax);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) tring.prologue();
-  } else {
-    ring.prologue();
-  }
+  ring.prologue();
   stage_q_rows<T, D>(q, nullptr, b, B, Hq, G, hk, B, RQ, qs, qm);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, n_warps = blockDim.x >> 5;
   for (int ch = c0; ch < c1; ++ch) {
     for (int pg = threadIdx.x; pg < kPsPages; pg += blockDim.x) best[pg] = 0u;  // below every key
-    if constexpr (kSel) tring.advance(ch); else ring.advance(ch);
+    ring.advance(ch);
     const T* smn = ring.mn(ch);
     const T* smx = ring.mx(ch);
     __syncthreads();  // chunk ch, the q rows and the cleared maxima visible to every thread
@@ -942,7 +826,7 @@ __global__ void __launch_bounds__(256, 2)
         const int rq1 = rq + 1 < RQ ? rq + 1 : rq;
         float yb[2];
         page_bound_sel2<D>(qs + rq * D, qm + rq * (D / 2), qs + rq1 * D, qm + rq1 * (D / 2),
-                           tring.mn(ch), tring.mx(ch), pg, yb);
+                           smn + pg * PS, smx + pg * PS, yb);
         mx = max(mx, max(order_key(yb[0]), order_key(yb[1])));
       }
       if (ch * kPsPages + pg < n_pages) atomicMax(&best[pg], mx);
@@ -962,10 +846,6 @@ __global__ void __launch_bounds__(256, 2)
         scores[((long long)b * kv.Hkv + hk) * kv.max_pages + p] = order_key_inv(best[pg]);
     }
     __syncthreads();  // maxima read out, this chunk's buffer free for the next iteration
-  }
-  if constexpr (kSel) {
-    // a wait that gave up may have left copies in flight: let them land
-    if (threadIdx.x == 0 && abort_flag) tring.drain(max(c0, c1 - (TmaPageRing<D>::kStages - 1)));
   }
 }
 
