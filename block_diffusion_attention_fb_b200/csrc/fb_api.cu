@@ -1047,12 +1047,10 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
   int cpc;
   const int psm = page_score_smem(na * G, D, (int)elem_size(kv->dtype)) + (pick_in_scorer ? B * 4 : 0);
   const dim3 g2 = page_score_grid(v, num_sms, psm, cpc);
-  // bf16: a warp scores two q rows over 32 pages, so 64 threads per row pair
-  const int ps_threads = min(256, 64 * ceil_div(na * G, 2));
   if (kv->dtype == FB_BF16) {
     auto kfn = D == 128 ? page_score_kernel<__nv_bfloat16, 128> : page_score_kernel<__nv_bfloat16, 64>;
     if ((rc = set_smem_once((const void*)kfn, psm))) return rc;
-    launch_pdl(kfn, g2, dim3(ps_threads), psm, stream, static_cast<const __nv_bfloat16*>(q_cur), act_in,
+    launch_pdl(kfn, g2, dim3(256), psm, stream, static_cast<const __nv_bfloat16*>(q_cur), act_in,
                rs_in, active_rows, B, Hq, G, na, static_cast<const __nv_bfloat16*>(page_min),
                static_cast<const __nv_bfloat16*>(page_max), v, page_scores, union_bitmap, words,
                tickets, cpc);

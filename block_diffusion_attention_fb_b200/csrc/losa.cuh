@@ -321,83 +321,66 @@ __device__ __forceinline__ float page_bound(const float* qr, const T* mnr, const
 // per-row mask qm (0xFFFF in the half of each channel with q_c < 0) picks the
 // bf16 halves with one bitwise select; products and tree levels with stride >= 2
 // run on packed float pairs (f32x2), each lane single-rounded as in the
-// definition. q rows qr (float) and qm are read by every lane of the warp at the
+// definition. q row qr (float) and qm are read by every lane of the warp at the
 // same address (broadcast); mnr / mxr are this lane's page.
 template <int D>
-__device__ __forceinline__ void page_bound_sel2(const float* qr0, const uint32_t* qm0,
-                                                const float* qr1, const uint32_t* qm1,
+__device__ __forceinline__ float page_bound_sel(const float* qr, const uint32_t* qm,
                                                 const __nv_bfloat16* mnr,
-                                                const __nv_bfloat16* mxr, float (&out)[2]) {
-  // Two q rows against one page: the page's minima and maxima of a group of
-  // channels are read from shared memory once and serve both rows (the
-  // shared-memory pipe, not the arithmetic, limits this loop).
+                                                const __nv_bfloat16* mxr) {
   // The first three tree levels (channel strides D/2, D/4, D/8) are formed per
   // output channel n < E = D/8 from the eight channels n + k E, k = 0..7:
   //   ((a_n + a_n+4E) + (a_n+2E + a_n+6E)) + ((a_n+E + a_n+5E) + (a_n+3E + a_n+7E)),
-  // which is the tree's own pairing and order; only E values per row stay live.
+  // which is the tree's own pairing and order; only E values stay live.
   constexpr int E = D / 8;
-  float2 z[2][E / 2];  // level-3 sums of channels (2i, 2i + 1), per row
-  const float* qr[2] = {qr0, qr1};
-  const uint32_t* qm[2] = {qm0, qm1};
+  float2 z[E / 2];  // level-3 sums of channels (2i, 2i + 1)
+  // products of the channel pairs c8 + 2j (+1) + k E, j = 0..3
+  auto prod = [&](int c8, int k, float2 (&a)[4]) {
+    const int c = c8 + k * E;
+    const uint4 n = *reinterpret_cast<const uint4*>(mnr + c);
+    const uint4 x = *reinterpret_cast<const uint4*>(mxr + c);
+    const uint4 m = *reinterpret_cast<const uint4*>(qm + c / 2);
+    const float4 qa = *reinterpret_cast<const float4*>(qr + c);
+    const float4 qb = *reinterpret_cast<const float4*>(qr + c + 4);
+    const uint32_t nn[4] = {n.x, n.y, n.z, n.w}, xx[4] = {x.x, x.y, x.z, x.w};
+    const uint32_t mm[4] = {m.x, m.y, m.z, m.w};
+    const float2 qq[4] = {make_float2(qa.x, qa.y), make_float2(qa.z, qa.w),
+                          make_float2(qb.x, qb.y), make_float2(qb.z, qb.w)};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t sel = (xx[j] & ~mm[j]) | (nn[j] & mm[j]);
+      a[j] = fmul2(qq[j], make_float2(__uint_as_float(sel << 16),
+                                      __uint_as_float(sel & 0xFFFF0000u)));
+    }
+  };
+  // level-1 pair (k, k + 4) of the eight offsets
+  auto level1 = [&](int c8, int k, float2 (&b)[4]) {
+    float2 lo[4], hi[4];
+    prod(c8, k, lo);
+    prod(c8, k + 4, hi);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) b[j] = fadd2(lo[j], hi[j]);
+  };
 #pragma unroll
   for (int c8 = 0; c8 < E; c8 += 8) {
     // keeps the next group's loads from being hoisted above this one (which
     // would hold both groups' operands at once and spill)
     if (c8 > 0) asm volatile("" ::: "memory");
-    uint32_t nn[8][4], xx[8][4];  // this lane's page: channels c8 + k E .. + 7, as bf16 pairs
+    float2 b0[4], b2[4], c0[4];
+    level1(c8, 0, b0);
+    level1(c8, 2, b2);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint4 n = *reinterpret_cast<const uint4*>(mnr + c8 + k * E);
-      const uint4 x = *reinterpret_cast<const uint4*>(mxr + c8 + k * E);
-      nn[k][0] = n.x; nn[k][1] = n.y; nn[k][2] = n.z; nn[k][3] = n.w;
-      xx[k][0] = x.x; xx[k][1] = x.y; xx[k][2] = x.z; xx[k][3] = x.w;
-    }
+    for (int j = 0; j < 4; ++j) c0[j] = fadd2(b0[j], b2[j]);
+    float2 b1[4], b3[4];
+    level1(c8, 1, b1);
+    level1(c8, 3, b3);
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      // products of the channel pairs c8 + 2j (+1) + k E, j = 0..3, for row r
-      auto prod = [&](int k, float2 (&a)[4]) {
-        const int c = c8 + k * E;
-        const uint4 m = *reinterpret_cast<const uint4*>(qm[r] + c / 2);
-        const float4 qa = *reinterpret_cast<const float4*>(qr[r] + c);
-        const float4 qb = *reinterpret_cast<const float4*>(qr[r] + c + 4);
-        const uint32_t mm[4] = {m.x, m.y, m.z, m.w};
-        const float2 qq[4] = {make_float2(qa.x, qa.y), make_float2(qa.z, qa.w),
-                              make_float2(qb.x, qb.y), make_float2(qb.z, qb.w)};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t sel = (xx[k][j] & ~mm[j]) | (nn[k][j] & mm[j]);
-          a[j] = fmul2(qq[j], make_float2(__uint_as_float(sel << 16),
-                                          __uint_as_float(sel & 0xFFFF0000u)));
-        }
-      };
-      // level-1 pair (k, k + 4) of the eight offsets
-      auto level1 = [&](int k, float2 (&b)[4]) {
-        float2 lo[4], hi[4];
-        prod(k, lo);
-        prod(k + 4, hi);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) b[j] = fadd2(lo[j], hi[j]);
-      };
-      float2 b0[4], b2[4], c0[4];
-      level1(0, b0);
-      level1(2, b2);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) c0[j] = fadd2(b0[j], b2[j]);
-      float2 b1[4], b3[4];
-      level1(1, b1);
-      level1(3, b3);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) z[r][c8 / 2 + j] = fadd2(c0[j], fadd2(b1[j], b3[j]));
-    }
+    for (int j = 0; j < 4; ++j) z[c8 / 2 + j] = fadd2(c0[j], fadd2(b1[j], b3[j]));
   }
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
+  for (int st = E / 4; st >= 1; st >>= 1)  // channel strides 2 st = E/2 ... 2, in pairs
 #pragma unroll
-    for (int st = E / 4; st >= 1; st >>= 1)  // channel strides 2 st = E/2 ... 2, in pairs
-#pragma unroll
-      for (int i = 0; i < st; ++i) z[r][i] = fadd2(z[r][i], z[r][i + st]);
-    out[r] = __fadd_rn(z[r][0].x, z[r][0].y);  // the last level: channel 0 + channel 1
-  }
+    for (int i = 0; i < st; ++i) z[i] = fadd2(z[i], z[i + st]);
+  return __fadd_rn(z[0].x, z[0].y);  // the last level: channel 0 + channel 1
 }
 
 // Shared memory of the page scorers for RQ staged q rows: the rows (float),
@@ -543,23 +526,14 @@ __global__ void __launch_bounds__(256, 2)
     const T* smx = ring.mx(ch);
     __syncthreads();  // chunk ch (and the q rows) visible to every thread
     if constexpr (kSel) {
-      // warp: one half of the chunk's pages (lane = page) and rows r, r + 1
       const int pg = (warp & 1) * 32 + lane;
       const int p = ch * kPsPages + pg;
-      for (int rq = 2 * (warp >> 1); rq < RQ; rq += n_warps) {
-        const int rq1 = rq + 1 < RQ ? rq + 1 : rq;
-        float yb[2];
-        page_bound_sel2<D>(qs + rq * D, qm + rq * (D / 2), qs + rq1 * D, qm + rq1 * (D / 2),
-                           smn + pg * PS, smx + pg * PS, yb);
-        if (p < n_pages) {
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const int rr = r == 0 ? rq : rq1;
-            if (r == 1 && rq1 == rq) break;
-            const int a_i = rr / G, g = rr - (rr / G) * G;
-            scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = yb[r];
-          }
-        }
+      for (int rq = warp >> 1; rq < RQ; rq += n_warps >> 1) {
+        const float yb = page_bound_sel<D>(qs + rq * D, qm + rq * (D / 2), smn + pg * PS,
+                                           smx + pg * PS);
+        const int a_i = rq / G, g = rq - (rq / G) * G;
+        if (p < n_pages)
+          scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = yb;
       }
     } else {
       for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
@@ -819,16 +793,11 @@ __global__ void __launch_bounds__(256, 2)
     const T* smx = ring.mx(ch);
     __syncthreads();  // chunk ch, the q rows and the cleared maxima visible to every thread
     if constexpr (kSel) {
-      // warp: one half of the chunk's pages (lane = page) and rows r, r + 1
       const int pg = (warp & 1) * 32 + lane;
       uint32_t mx = 0u;  // below every key
-      for (int rq = 2 * (warp >> 1); rq < RQ; rq += n_warps) {
-        const int rq1 = rq + 1 < RQ ? rq + 1 : rq;
-        float yb[2];
-        page_bound_sel2<D>(qs + rq * D, qm + rq * (D / 2), qs + rq1 * D, qm + rq1 * (D / 2),
-                           smn + pg * PS, smx + pg * PS, yb);
-        mx = max(mx, max(order_key(yb[0]), order_key(yb[1])));
-      }
+      for (int rq = warp >> 1; rq < RQ; rq += n_warps >> 1)
+        mx = max(mx, order_key(page_bound_sel<D>(qs + rq * D, qm + rq * (D / 2), smn + pg * PS,
+                                                  smx + pg * PS)));
       if (ch * kPsPages + pg < n_pages) atomicMax(&best[pg], mx);
     } else {
       for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
