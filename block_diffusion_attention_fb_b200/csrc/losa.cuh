@@ -627,6 +627,7 @@ __global__ void __launch_bounds__(kTopkThreads)
   allow_dependent_launch();
   extern __shared__ uint32_t keys[];  // max_pages keys, then a words-long bitmap
   __shared__ int hist[256];
+  __shared__ int whist[kTopkThreads / 32][256];  // per-warp digit counts
   __shared__ int warp_sums[33];
   __shared__ uint32_t s_prefix;
   __shared__ int s_need, s_last;
@@ -651,14 +652,25 @@ __global__ void __launch_bounds__(kTopkThreads)
       s_need = k;
     }
     uint32_t mask = 0u;
+    const int wid = tid >> 5;
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
-      for (int d = tid; d < 256; d += blockDim.x) hist[d] = 0;
+      for (int d = tid; d < (kTopkThreads / 32) * 256; d += blockDim.x) (&whist[0][0])[d] = 0;
       __syncthreads();
       const uint32_t prefix = s_prefix;
+      // Scores of one row are alike, so a few digits take most keys (all of
+      // them share one in the first pass): each warp counts into its own
+      // histogram, so only a warp's own lanes contend for a counter.
       for (int p = tid; p < n; p += blockDim.x) {
         const uint32_t key = keys[p];
-        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1);
+        if ((key & mask) == prefix) atomicAdd(&whist[wid][(key >> shift) & 0xFFu], 1);
+      }
+      __syncthreads();
+      for (int d = tid; d < 256; d += blockDim.x) {
+        int c = 0;
+#pragma unroll
+        for (int w = 0; w < kTopkThreads / 32; ++w) c += whist[w][d];
+        hist[d] = c;
       }
       __syncthreads();
       if (tid < 32) {
