@@ -307,12 +307,11 @@ class Rig:
         self.topk = sp.topk_pages or LOSA_TOPK
         self.losa = BlockAttention(kv, B, Hq, "losa", n_active=self.n_act, topk_pages=self.topk)
         # FlashBlock + sparse residual: 20% page density (the pages pair FlashBlock
-        # with SparseD at 20-40%); supported up to 64 stacked rows per kv head
+        # with SparseD at 20-40%)
         self.sr_topk = max(1, -(-kv.n_pages * SR_DENSITY_PCT // 100))
         self.sr_tau = sp.tau if sp.tau is not None else 4
-        self.sres = (BlockAttention(kv, B, Hq, "sparse_residual", tau=self.sr_tau,
-                                    topk_pages=self.sr_topk)
-                     if B * (Hq // sp.n_heads_kv) <= 64 else None)
+        self.sres = BlockAttention(kv, B, Hq, "sparse_residual", tau=self.sr_tau,
+                                   topk_pages=self.sr_topk)
         # block commit: a separate contiguous cache with room for every timed
         # commit (the commit reads only the block rows, so its content is not needed)
         self.commit = None
@@ -784,9 +783,6 @@ def run_profile_mode(args, rank):
     name = args.workload or HEADLINE
     rig = Rig(name, args, with_commit=False)
     flush = _Flush()
-    if args.mode == "sr_step" and rig.sres is None:
-        raise SystemExit("sr_step: the sparse-residual mode takes at most 64 stacked rows "
-                         "per kv head")
     fn = {"prefix": rig.prefix_call, "block": rig.block_call, "losa_step": rig.losa_step,
           "sr_step": lambda s: rig.sres_step(s)}[args.mode]
     for _ in range(args.warmup + args.steps):

@@ -743,13 +743,13 @@ int sr_select(const void* q, int B, int Hq, const void* page_min, const void* pa
   const KvView v = kv_view(kv);
   const int D = v.D, G = Hq / v.Hkv, RQ = B * G;
   const int words = ceil_div(v.max_pages, 32);
-  if (RQ > 64) return fail(FB_ERR_SHAPE, "sparse residual supports <= 64 rows per kv head");
+
   if (v.max_pages > 32768) return fail(FB_ERR_SHAPE, "sparse residual supports <= 32768 pages");
   if (!aligned16(page_min) || !aligned16(page_max))
     return fail(FB_ERR_ALIGN, "page summaries not 16-byte aligned");
   int cpc;
   const int es = (int)elem_size(kv->dtype);
-  const int psm = page_score_smem(RQ, D, es);
+  const int psm = page_score_smem(RQ < kHsRows ? RQ : kHsRows, D, es);
   const dim3 g2 = page_score_grid(v, sm_count(), psm, cpc);
   int rc;
 #define FB_HPS(TT, DD)                                                                       \

@@ -393,14 +393,14 @@ __host__ __device__ constexpr int page_score_smem(int RQ, int D, int elem_bytes)
 // Stages the active q rows of (b, hk) as float, and for bf16 the per-channel
 // sign masks of page_bound_sel: qs [RQ][D], qm [RQ][D/2].
 // act: the n_act active rows of sequence b (global or shared), or NULL for
-// rows 0 .. n_act-1.
+// rows 0 .. n_act-1. Stacked rows row0 .. row0 + RQ - 1 are staged.
 template <typename T, int D>
 __device__ __forceinline__ void stage_q_rows(const T* q, const int* act, int b, int B,
                                              int Hq, int G, int hk, int n_act, int RQ, float* qs,
-                                             uint32_t* qm) {
+                                             uint32_t* qm, int row0 = 0) {
   for (int idx = threadIdx.x; idx < RQ * D; idx += blockDim.x) {
     const int rq = idx / D, c = idx - (idx / D) * D;
-    const int a_i = rq / G, g = rq - (rq / G) * G;
+    const int a_i = (row0 + rq) / G, g = (row0 + rq) - a_i * G;
     const int i = act ? act[a_i] : a_i;
     qs[idx] = ld_f32<T>(q + (((long long)b * B + i) * Hq + hk * G + g) * D + c);
   }
@@ -762,7 +762,12 @@ __global__ void __launch_bounds__(kTopkThreads)
 // page_score_kernel (single-rounded products, stride-halving tree); the maximum
 // is order-free, taken on order-preserving keys with shared-memory atomics.
 // scores: [batch, Hkv, max_pages]. Block (0, hk, b) clears the (b, hk) bitmap.
+// Rows are taken kHsRows at a time (q staged per group, every page chunk
+// streamed again per group, from L2 where it fits): the maximum is order-free,
+// and later groups fold theirs into the scores the earlier groups wrote.
 // ---------------------------------------------------------------------------
+constexpr int kHsRows = 64;
+
 __device__ __forceinline__ float order_key_inv(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
@@ -780,10 +785,11 @@ __global__ void __launch_bounds__(256, 2)
   constexpr bool kSel = sizeof(T) == 2;  // bf16: masked-select bound, warp per row
   extern __shared__ __align__(16) float sm[];
   __shared__ uint32_t best[kPsPages];
-  const int RQ = B * G;
-  float* qs = sm;                                            // [RQ][D], row r = i * G + g
-  uint32_t* qm = reinterpret_cast<uint32_t*>(qs + RQ * D);   // [RQ][D/2] (bf16)
-  T* sbuf = reinterpret_cast<T*>(qm + (kSel ? RQ * (D / 2) : 0));  // 2 x ([64][PS] min, max)
+  const int RQ_all = B * G;
+  const int RQmax = RQ_all < kHsRows ? RQ_all : kHsRows;
+  float* qs = sm;                                              // [RQmax][D], row r = i * G + g
+  uint32_t* qm = reinterpret_cast<uint32_t*>(qs + RQmax * D);  // [RQmax][D/2] (bf16)
+  T* sbuf = reinterpret_cast<T*>(qm + (kSel ? RQmax * (D / 2) : 0));  // stages of [64][PS]
   const int hk = blockIdx.y, b = blockIdx.z;
   if (blockIdx.x == 0) {
     for (int w = threadIdx.x; w < words; w += blockDim.x)
@@ -795,9 +801,11 @@ __global__ void __launch_bounds__(256, 2)
   const int c1 = min(c0 + cpc, (n_pages + kPsPages - 1) / kPsPages);
   if (c0 >= c1) return;
   const PageRing<T, D> ring{sbuf, pmin, pmax, kv, b, hk, c0, c1, n_pages};
-  ring.prologue();
-  stage_q_rows<T, D>(q, nullptr, b, B, Hq, G, hk, B, RQ, qs, qm);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, n_warps = blockDim.x >> 5;
+  for (int row0 = 0; row0 < RQ_all; row0 += kHsRows) {
+  const int RQ = RQ_all - row0 < kHsRows ? RQ_all - row0 : kHsRows;
+  ring.prologue();
+  stage_q_rows<T, D>(q, nullptr, b, B, Hq, G, hk, B, RQ, qs, qm, row0);
   for (int ch = c0; ch < c1; ++ch) {
     for (int pg = threadIdx.x; pg < kPsPages; pg += blockDim.x) best[pg] = 0u;  // below every key
     ring.advance(ch);
@@ -823,10 +831,14 @@ __global__ void __launch_bounds__(256, 2)
     __syncthreads();
     for (int pg = threadIdx.x; pg < kPsPages; pg += blockDim.x) {
       const int p = ch * kPsPages + pg;
-      if (p < n_pages)
-        scores[((long long)b * kv.Hkv + hk) * kv.max_pages + p] = order_key_inv(best[pg]);
+      if (p < n_pages) {
+        float* dst = scores + ((long long)b * kv.Hkv + hk) * kv.max_pages + p;
+        // this CTA alone writes these pages: fold into an earlier group's maximum
+        *dst = order_key_inv(row0 == 0 ? best[pg] : max(best[pg], order_key(*dst)));
+      }
     }
     __syncthreads();  // maxima read out, this chunk's buffer free for the next iteration
+  }
   }
 }
 

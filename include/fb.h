@@ -281,8 +281,9 @@ typedef struct fb_cache {
  *              the other pages into comp_list / comp_count, and the partial
  *              over the unselected pages is stored in a_res / l_res. Every step
  *              computes the partial over the selected pages with the current q
- *              and merges it with the cached residual into a_out / l_out. At
- *              most 64 stacked rows (B * Hq / Hkv) per kv head (FB_ERR_SHAPE).
+ *              and merges it with the cached residual into a_out / l_out. The
+ *              head score takes every stacked row (B * Hq / Hkv per kv head), 64
+ *              at a time.
  *              Workspace: fb_workspace_size with n_active = B and topk_pages =
  *              the logical page count.
  * Then the block-internal partial is computed and merged:
