@@ -104,11 +104,10 @@ int sm_count() {
 // The dynamic shared-memory limit is a per-device function attribute: raise it
 // for each (device, kernel) pair when a launch needs more than was set so far.
 int set_smem_once(const void* fn, int bytes) {
-  if (bytes <= 48 * 1024) return FB_OK;
   struct Entry {
     int dev;
     const void* fn;
-    int bytes;
+    int bytes;  // dynamic bytes the kernel may take on this device
   };
   static std::mutex mu;
   static std::vector<Entry> done;
@@ -119,13 +118,22 @@ int set_smem_once(const void* fn, int bytes) {
   for (auto& d : done)
     if (d.dev == dev && d.fn == fn) hit = &d;
   if (hit && hit->bytes >= bytes) return FB_OK;
-  const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e != cudaSuccess)
-    return fail(FB_ERR_CUDA, "cudaFuncSetAttribute(%d bytes): %s", bytes, cudaGetErrorString(e));
+  // the 48 KB default covers static plus dynamic shared memory
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess)
+    return fail(FB_ERR_CUDA, "cudaFuncGetAttributes failed");
+  const int deflt = 48 * 1024 - (int)fa.sharedSizeBytes;
+  if (bytes > deflt) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess)
+      return fail(FB_ERR_CUDA, "cudaFuncSetAttribute(%d bytes): %s", bytes, cudaGetErrorString(e));
+  }
+  const int allowed = bytes > deflt ? bytes : deflt;
   if (hit)
-    hit->bytes = bytes;
+    hit->bytes = allowed;
   else
-    done.push_back(Entry{dev, fn, bytes});
+    done.push_back(Entry{dev, fn, allowed});
   return FB_OK;
 }
 
