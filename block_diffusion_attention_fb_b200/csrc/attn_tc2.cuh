@@ -313,6 +313,11 @@ __global__ void __launch_bounds__(kT2Threads, 1)
     }
     float m_used = -INFINITY, l_sum = 0.f;
     for (int j = 0; j < n_it; ++j) {
+      // Tile j's metadata first: the producer published it before loading K_j,
+      // so this wait overlaps the wait for S_j instead of following it.
+      const int st = j % kT2Meta;
+      mbar_wait(&meta_bar[st], (j / kT2Meta) & 1, &abort_flag);
+      const bool tile_full = meta_full[st] != 0;
       if (!mbar_wait(&s_full[x], j & 1, &abort_flag)) break;
       // lanes leave their waits at different times; the TMEM loads below are
       // warp-collective (.sync.aligned) and need the warp converged
@@ -327,9 +332,6 @@ __global__ void __launch_bounds__(kT2Threads, 1)
         for (int k = 0; k < 32; ++k) sv[c * 32 + k] = t[k];
       }
       tmem_wait_ld();
-      const int st = j % kT2Meta;
-      mbar_wait(&meta_bar[st], (j / kT2Meta) & 1, &abort_flag);  // acquire tile j's metadata
-      const bool tile_full = meta_full[st] != 0;
       const int chunk = a.chunk;
       if (!tile_full) {  // keys outside the key set: raw score -inf
 #pragma unroll
