@@ -191,7 +191,19 @@ __global__ void __launch_bounds__(256)
 __device__ __forceinline__ void pick_active_rows(const float* score_b, int B, int n_act,
                                                  float* sc, int* taken) {
   __shared__ unsigned long long wbest[32];
-  for (int i = threadIdx.x; i < B; i += blockDim.x) sc[i] = score_b[i];
+  for (int i0 = threadIdx.x; i0 < B; i0 += 8 * blockDim.x) {  // 8 loads in flight
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      v[u] = i < B ? __ldcg(score_b + i) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < B) sc[i] = v[u];
+    }
+  }
   __syncthreads();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   for (int r = 0; r < n_act; ++r) {
@@ -646,7 +658,21 @@ __global__ void __launch_bounds__(kTopkThreads)
     __syncthreads();
     for (int p = tid; p < n; p += blockDim.x) take(p);
   } else if (k > 0) {
-    for (int p = tid; p < n; p += blockDim.x) keys[p] = order_key(sc[p]);
+    // the scores, 8 loads in flight per thread (a loop of single loads would
+    // pay the memory latency once per key it reads)
+    for (int p0 = tid; p0 < n; p0 += 8 * blockDim.x) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int p = p0 + u * blockDim.x;
+        v[u] = p < n ? __ldcg(sc + p) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int p = p0 + u * blockDim.x;
+        if (p < n) keys[p] = order_key(v[u]);
+      }
+    }
     if (tid == 0) {
       s_prefix = 0u;
       s_need = k;
