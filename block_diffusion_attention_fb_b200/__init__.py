@@ -36,7 +36,7 @@ EXPORTS = ("fb_workspace_size", "fb_prefix_attn", "fb_block_attn", "fb_merge", "
            "losa_select", "losa_gather", "fb_step", "fb_device_status", "fb_last_error",
            "fb_kernel_launches", "fb_prefix_attn_noalloc", "fb_block_commit",
            "fb_selftest_timeout", "fb_prefix_attn_varlen", "fb_block_attn_varlen",
-           "fb_step_varlen")
+           "fb_step_varlen", "fb_workspace_page_scores")
 
 
 class FbError(RuntimeError):
@@ -88,6 +88,7 @@ def load_library() -> ctypes.CDLL:
     KV = ctypes.POINTER(fb_kv)
     sig = {
         "fb_workspace_size": (SZ, [KV, I32, I32, I32, I32, I32]),
+        "fb_workspace_page_scores": (SZ, [KV, I32, I32, I32, I32, I32]),
         "fb_prefix_attn": (ctypes.c_int, [P, I32, I32, F32, KV, P, P, P, P, SZ, P]),
         "fb_block_attn": (ctypes.c_int, [P, P, P, I32, I32, I32, I32, I32, F32, ctypes.c_int, P, P, P]),
         "fb_merge": (ctypes.c_int, [P, P, P, P, I64, I32, P, P, P]),
@@ -185,6 +186,16 @@ def fb_workspace_size(kv: KV, block: int, n_heads_q: int, n_active: int = 0, top
                                          num_sms)
     if n == 0:
         raise FbError(FB_ERR_ARG, "fb_workspace_size: invalid arguments")
+    return int(n)
+
+
+def fb_workspace_page_scores(kv: KV, block: int, n_heads_q: int, n_active: int, topk_pages: int,
+                             num_sms: int = 0) -> int:
+    """Byte offset of the LoSA page scores inside the workspace."""
+    n = load_library().fb_workspace_page_scores(ctypes.byref(kv.c), block, n_heads_q, n_active,
+                                                topk_pages, num_sms)
+    if n == 0:
+        raise FbError(FB_ERR_ARG, "fb_workspace_page_scores: invalid arguments")
     return int(n)
 
 

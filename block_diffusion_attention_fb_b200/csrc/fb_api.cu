@@ -588,6 +588,21 @@ dim3 page_score_grid(const KvView& v, int num_sms, int smem_bytes, int& cpc) {
   return dim3(ceil_div(chunks, cpc), v.Hkv, v.batch);
 }
 
+// Grid of the bf16 page scorer: tiles of kPcPages pages per (sequence, kv
+// head), `tpc` consecutive tiles per CTA (a multiple of its warps, which take
+// them in turn), as few as keep the grid within one wave.
+dim3 page_cols_grid(const KvView& v, int num_sms, int smem_bytes, int& tpc) {
+  constexpr int nw = kPcThreads / 32;
+  const int tiles = ceil_div(v.max_pages, kPcPages);
+  const long long groups = (long long)v.batch * v.Hkv;
+  const int per_sm = smem_bytes + 1024 <= (227 * 1024) / 2 ? 2 : 1;
+  const long long slots = (long long)per_sm * (num_sms > 0 ? num_sms : 148);
+  tpc = (int)((groups * tiles + slots - 1) / slots);
+  tpc = ceil_div(tpc < 1 ? 1 : tpc, nw) * nw;
+  while (tpc < tiles && (long long)ceil_div(tiles, tpc) * groups > slots) tpc += nw;
+  return dim3(ceil_div(tiles, tpc), v.Hkv, v.batch);
+}
+
 // Short blocks (bf16, B <= 64): the latency-built kernel of block_attn.cuh.
 // Rows per CTA: 16 per warp, 1 to 4 warps, fewer warps while that keeps the
 // grid within two CTAs per SM (more CTAs = more of the block's loads in flight).
@@ -755,25 +770,29 @@ int sr_select(const void* q, int B, int Hq, const void* page_min, const void* pa
   if (v.max_pages > 32768) return fail(FB_ERR_SHAPE, "sparse residual supports <= 32768 pages");
   if (!aligned16(page_min) || !aligned16(page_max))
     return fail(FB_ERR_ALIGN, "page summaries not 16-byte aligned");
-  int cpc;
-  const int es = (int)elem_size(kv->dtype);
-  const int psm = page_score_smem(RQ < kHsRows ? RQ : kHsRows, D, es);
-  const dim3 g2 = page_score_grid(v, sm_count(), psm, cpc);
   int rc;
-#define FB_HPS(TT, DD)                                                                       \
-  do {                                                                                       \
-    auto kfn = head_page_score_kernel<TT, DD>;                                               \
-    if ((rc = set_smem_once((const void*)kfn, psm))) return rc;                            \
-    launch_pdl(kfn, g2, dim3(256), psm, stream, static_cast<const TT*>(q), B, Hq, G,        \
-               static_cast<const TT*>(page_min), static_cast<const TT*>(page_max), v,        \
-               head_scores, bitmap, words, tickets, cpc);                                    \
-  } while (0)
   if (kv->dtype == FB_BF16) {
-    if (D == 128) FB_HPS(__nv_bfloat16, 128); else FB_HPS(__nv_bfloat16, 64);
+    int tpc;
+    const int psm = page_score_cols_smem(RQ, D, true);
+    const dim3 g2 = page_cols_grid(v, sm_count(), psm, tpc);
+    auto kfn = D == 128 ? page_score_cols_kernel<128, kPcHeadMax>
+                        : page_score_cols_kernel<64, kPcHeadMax>;
+    if ((rc = set_smem_once((const void*)kfn, psm))) return rc;
+    launch_pdl(kfn, g2, dim3(kPcThreads), psm, stream, static_cast<const __nv_bfloat16*>(q),
+               (const int32_t*)nullptr, (const float*)nullptr, (int32_t*)nullptr, B, Hq, G, B,
+               static_cast<const __nv_bfloat16*>(page_min),
+               static_cast<const __nv_bfloat16*>(page_max), v, head_scores, bitmap, words,
+               tickets, tpc);
   } else {
-    if (D == 128) FB_HPS(float, 128); else FB_HPS(float, 64);
+    int cpc;
+    const int psm = page_score_smem(RQ < kHsRows ? RQ : kHsRows, D);
+    const dim3 g2 = page_score_grid(v, sm_count(), psm, cpc);
+    auto kfn = D == 128 ? head_page_score_kernel<float, 128> : head_page_score_kernel<float, 64>;
+    if ((rc = set_smem_once((const void*)kfn, psm))) return rc;
+    launch_pdl(kfn, g2, dim3(256), psm, stream, static_cast<const float*>(q), B, Hq, G,
+               static_cast<const float*>(page_min), static_cast<const float*>(page_max), v,
+               head_scores, bitmap, words, tickets, cpc);
   }
-#undef FB_HPS
   if ((rc = check_launch("head page score kernel"))) return rc;
   const int ksm = (v.max_pages + words) * 4;
   if ((rc = set_smem_once((const void*)topk_pages_kernel, ksm))) return rc;
@@ -895,6 +914,14 @@ size_t fb_workspace_size(const fb_kv* kv, int32_t block, int32_t n_heads_q, int3
   if (num_sms <= 0) num_sms = sm_count();
   if (num_sms <= 0) return 0;
   return ws_layout(kv, block, n_heads_q, n_active, topk_pages, num_sms).total;
+}
+
+size_t fb_workspace_page_scores(const fb_kv* kv, int32_t block, int32_t n_heads_q,
+                                int32_t n_active, int32_t topk_pages, int32_t num_sms) {
+  if (n_active <= 0 || topk_pages <= 0) return 0;
+  if (fb_workspace_size(kv, block, n_heads_q, n_active, topk_pages, num_sms) == 0) return 0;
+  if (num_sms <= 0) num_sms = sm_count();
+  return ws_layout(kv, block, n_heads_q, n_active, topk_pages, num_sms).scores;
 }
 
 int fb_prefix_attn(const void* q, int32_t B, int32_t n_heads_q, float scale, const fb_kv* kv,
@@ -1052,17 +1079,25 @@ int losa_select(const void* q_cur, const void* q_prev, int32_t B, int32_t n_head
   }
   const int32_t* act_in = pick_in_scorer ? nullptr : active_rows;
   const float* rs_in = pick_in_scorer ? rs : nullptr;
-  int cpc;
-  const int psm = page_score_smem(na * G, D, (int)elem_size(kv->dtype)) + (pick_in_scorer ? B * 4 : 0);
-  const dim3 g2 = page_score_grid(v, num_sms, psm, cpc);
   if (kv->dtype == FB_BF16) {
-    auto kfn = D == 128 ? page_score_kernel<__nv_bfloat16, 128> : page_score_kernel<__nv_bfloat16, 64>;
+    int tpc;
+    const int psm = page_score_cols_smem(na * G, D, false) + (pick_in_scorer ? B * 4 : 0);
+    const dim3 g2 = page_cols_grid(v, num_sms, psm, tpc);
+    const bool one = na * G <= kPcRows;
+    auto kfn = D == 128 ? (one ? page_score_cols_kernel<128, kPcRowsOnePass>
+                               : page_score_cols_kernel<128, kPcRowsMulti>)
+                        : (one ? page_score_cols_kernel<64, kPcRowsOnePass>
+                               : page_score_cols_kernel<64, kPcRowsMulti>);
     if ((rc = set_smem_once((const void*)kfn, psm))) return rc;
-    launch_pdl(kfn, g2, dim3(256), psm, stream, static_cast<const __nv_bfloat16*>(q_cur), act_in,
-               rs_in, active_rows, B, Hq, G, na, static_cast<const __nv_bfloat16*>(page_min),
+    launch_pdl(kfn, g2, dim3(kPcThreads), psm, stream, static_cast<const __nv_bfloat16*>(q_cur),
+               act_in, rs_in, active_rows, B, Hq, G, na,
+               static_cast<const __nv_bfloat16*>(page_min),
                static_cast<const __nv_bfloat16*>(page_max), v, page_scores, union_bitmap, words,
-               tickets, cpc);
+               tickets, tpc);
   } else {
+    int cpc;
+    const int psm = page_score_smem(na * G, D) + (pick_in_scorer ? B * 4 : 0);
+    const dim3 g2 = page_score_grid(v, num_sms, psm, cpc);
     auto kfn = D == 128 ? page_score_kernel<float, 128> : page_score_kernel<float, 64>;
     if ((rc = set_smem_once((const void*)kfn, psm))) return rc;
     launch_pdl(kfn, g2, dim3(256), psm, stream, static_cast<const float*>(q_cur), act_in, rs_in,

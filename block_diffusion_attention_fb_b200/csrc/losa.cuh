@@ -8,6 +8,8 @@
 // x[n] += x[n + stride] for n < stride). Ties go to the lower index.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace fb {
@@ -261,13 +263,12 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------------------
-// Page scoring (steps 3a of LoSA and the sparse-residual selector): pages are
-// handled in chunks of kPsPages.
+// Page scoring (steps 3a of LoSA and the sparse-residual selector), float32
+// summaries: pages are handled in chunks of kPsPages, staged in shared memory.
+// (bf16 summaries: page_score_cols_kernel below.)
 // ---------------------------------------------------------------------------
 constexpr int kPsPages = 64;
-// chunk buffers of the page scorers: bf16 three (two load while one is scored),
-// float32 two (its chunks are twice as large)
-__host__ __device__ constexpr int ps_stages(int elem_bytes) { return elem_bytes == 2 ? 3 : 2; }
+constexpr int kPsStages = 2;  // chunk buffers: one loads while the other is scored
 
 // Shared-memory row stride (elements) of the staged page summaries: rows stay
 // 16-byte aligned for vector loads, and consecutive pages start 4 banks apart,
@@ -277,16 +278,7 @@ __host__ __device__ constexpr int ps_stride() {
   return D + 16 / (int)sizeof(T);
 }
 
-// 8 consecutive elements as float (exact for bf16 and f32) from shared memory.
-__device__ __forceinline__ void load8_f32(const __nv_bfloat16* p, float (&o)[8]) {
-  const uint4 v = *reinterpret_cast<const uint4*>(p);
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    o[2 * j] = __uint_as_float(w[j] << 16);
-    o[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-  }
-}
+// 8 consecutive floats from shared memory.
 __device__ __forceinline__ void load8_f32(const float* p, float (&o)[8]) {
   const float4 a = *reinterpret_cast<const float4*>(p);
   const float4 b = *reinterpret_cast<const float4*>(p + 4);
@@ -325,105 +317,24 @@ __device__ __forceinline__ float page_bound(const float* qr, const T* mnr, const
   return y[0];
 }
 
-// The same bound for bf16 inputs, evaluated as tree_sum_c q_c * s_c with s_c =
-// kmax_c where q_c >= 0 and kmin_c where q_c < 0. A product of two bf16 values
-// is exact in float32, so max(q_c kmin_c, q_c kmax_c) IS q_c s_c, bit for bit
-// (for q_c = 0 both are zeros); the products and the tree are unchanged, only
-// the selection happens before the multiply. Two channels per 32-bit word: the
-// per-row mask qm (0xFFFF in the half of each channel with q_c < 0) picks the
-// bf16 halves with one bitwise select; products and tree levels with stride >= 2
-// run on packed float pairs (f32x2), each lane single-rounded as in the
-// definition. q row qr (float) and qm are read by every lane of the warp at the
-// same address (broadcast); mnr / mxr are this lane's page.
-template <int D>
-__device__ __forceinline__ float page_bound_sel(const float* qr, const uint32_t* qm,
-                                                const __nv_bfloat16* mnr,
-                                                const __nv_bfloat16* mxr) {
-  // The first three tree levels (channel strides D/2, D/4, D/8) are formed per
-  // output channel n < E = D/8 from the eight channels n + k E, k = 0..7:
-  //   ((a_n + a_n+4E) + (a_n+2E + a_n+6E)) + ((a_n+E + a_n+5E) + (a_n+3E + a_n+7E)),
-  // which is the tree's own pairing and order; only E values stay live.
-  constexpr int E = D / 8;
-  float2 z[E / 2];  // level-3 sums of channels (2i, 2i + 1)
-  // products of the channel pairs c8 + 2j (+1) + k E, j = 0..3
-  auto prod = [&](int c8, int k, float2 (&a)[4]) {
-    const int c = c8 + k * E;
-    const uint4 n = *reinterpret_cast<const uint4*>(mnr + c);
-    const uint4 x = *reinterpret_cast<const uint4*>(mxr + c);
-    const uint4 m = *reinterpret_cast<const uint4*>(qm + c / 2);
-    const float4 qa = *reinterpret_cast<const float4*>(qr + c);
-    const float4 qb = *reinterpret_cast<const float4*>(qr + c + 4);
-    const uint32_t nn[4] = {n.x, n.y, n.z, n.w}, xx[4] = {x.x, x.y, x.z, x.w};
-    const uint32_t mm[4] = {m.x, m.y, m.z, m.w};
-    const float2 qq[4] = {make_float2(qa.x, qa.y), make_float2(qa.z, qa.w),
-                          make_float2(qb.x, qb.y), make_float2(qb.z, qb.w)};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t sel = (xx[j] & ~mm[j]) | (nn[j] & mm[j]);
-      a[j] = fmul2(qq[j], make_float2(__uint_as_float(sel << 16),
-                                      __uint_as_float(sel & 0xFFFF0000u)));
-    }
-  };
-  // level-1 pair (k, k + 4) of the eight offsets
-  auto level1 = [&](int c8, int k, float2 (&b)[4]) {
-    float2 lo[4], hi[4];
-    prod(c8, k, lo);
-    prod(c8, k + 4, hi);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) b[j] = fadd2(lo[j], hi[j]);
-  };
-#pragma unroll
-  for (int c8 = 0; c8 < E; c8 += 8) {
-    // keeps the next group's loads from being hoisted above this one (which
-    // would hold both groups' operands at once and spill)
-    if (c8 > 0) asm volatile("" ::: "memory");
-    float2 b0[4], b2[4], c0[4];
-    level1(c8, 0, b0);
-    level1(c8, 2, b2);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) c0[j] = fadd2(b0[j], b2[j]);
-    float2 b1[4], b3[4];
-    level1(c8, 1, b1);
-    level1(c8, 3, b3);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) z[c8 / 2 + j] = fadd2(c0[j], fadd2(b1[j], b3[j]));
-  }
-#pragma unroll
-  for (int st = E / 4; st >= 1; st >>= 1)  // channel strides 2 st = E/2 ... 2, in pairs
-#pragma unroll
-    for (int i = 0; i < st; ++i) z[i] = fadd2(z[i], z[i + st]);
-  return __fadd_rn(z[0].x, z[0].y);  // the last level: channel 0 + channel 1
+// Shared memory of the page scorers for RQ staged q rows: the rows, and the
+// chunk buffers of minima and maxima.
+__host__ __device__ constexpr int page_score_smem(int RQ, int D) {
+  return RQ * D * 4 + 2 * kPsStages * kPsPages * (D + 4) * 4;
 }
 
-// Shared memory of the page scorers for RQ staged q rows: the rows (float),
-// their sign masks (bf16 inputs), and two buffers of a chunk's summaries.
-__host__ __device__ constexpr int page_score_smem(int RQ, int D, int elem_bytes) {
-  return RQ * D * 4 + (elem_bytes == 2 ? RQ * (D / 2) * 4 : 0) +
-         2 * ps_stages(elem_bytes) * kPsPages * (D + 16 / elem_bytes) * elem_bytes;
-}
-
-// Stages the active q rows of (b, hk) as float, and for bf16 the per-channel
-// sign masks of page_bound_sel: qs [RQ][D], qm [RQ][D/2].
+// Stages the active q rows of (b, hk): qs [RQ][D].
 // act: the n_act active rows of sequence b (global or shared), or NULL for
 // rows 0 .. n_act-1. Stacked rows row0 .. row0 + RQ - 1 are staged.
 template <typename T, int D>
 __device__ __forceinline__ void stage_q_rows(const T* q, const int* act, int b, int B,
                                              int Hq, int G, int hk, int n_act, int RQ, float* qs,
-                                             uint32_t* qm, int row0 = 0) {
+                                             int row0 = 0) {
   for (int idx = threadIdx.x; idx < RQ * D; idx += blockDim.x) {
     const int rq = idx / D, c = idx - (idx / D) * D;
     const int a_i = (row0 + rq) / G, g = (row0 + rq) - a_i * G;
     const int i = act ? act[a_i] : a_i;
     qs[idx] = ld_f32<T>(q + (((long long)b * B + i) * Hq + hk * G + g) * D + c);
-  }
-  if constexpr (sizeof(T) == 2) {
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < RQ * (D / 2); idx += blockDim.x) {
-      const int rq = idx / (D / 2), c2 = idx - rq * (D / 2);
-      const uint32_t lo = __float_as_uint(qs[rq * D + 2 * c2]) >> 31;
-      const uint32_t hi = __float_as_uint(qs[rq * D + 2 * c2 + 1]) >> 31;
-      qm[idx] = (lo ? 0x0000FFFFu : 0u) | (hi ? 0xFFFF0000u : 0u);
-    }
   }
 }
 
@@ -457,7 +368,7 @@ struct PageRing {
   const KvView& kv;
   int b, hk, c0, c1, n_pages;
   static constexpr int PS = ps_stride<T, D>();
-  static constexpr int kStages = ps_stages((int)sizeof(T));
+  static constexpr int kStages = kPsStages;
   __device__ T* mn(int ch) const { return sbuf + ((ch - c0) % kStages) * 2 * kPsPages * PS; }
   __device__ T* mx(int ch) const { return mn(ch) + kPsPages * PS; }
   __device__ void issue(int ch) const {
@@ -480,11 +391,8 @@ struct PageRing {
 // for every active row a and q head h of kv head hk. A CTA scores `cpc`
 // consecutive chunks of 64 pages of one (b, hk): the active q rows once into
 // shared memory, the summaries chunk by chunk into two buffers with cp.async,
-// the next chunk loading while the current one is scored. bf16: a warp takes
-// one q row (broadcast reads) and 32 pages (one per lane; warps 2r and 2r+1
-// the two halves of the chunk, rows r, r + 4, ... for the 8 warps), bound by
-// page_bound_sel; float32: one thread per (page, row) by page_bound. Both are
-// single-rounded products and the stride-halving tree.
+// the next chunk loading while the current one is scored; one thread per
+// (page, row) by page_bound (single-rounded products, stride-halving tree).
 // scores: [batch, n_act, Hq, max_pages]. Block (0, hk, b) also clears the
 // union bitmap of (b, hk) and its ticket for the top-k kernel that follows.
 // Active rows: given (active), or picked here from the locality scores
@@ -500,15 +408,14 @@ __global__ void __launch_bounds__(256, 2)
                       int cpc) {
   grid_dependency_wait();  // launched as a programmatic dependent
   allow_dependent_launch();
+  static_assert(sizeof(T) == 4, "float32 summaries (bf16: page_score_cols_kernel)");
   constexpr int PS = ps_stride<T, D>();
-  constexpr bool kSel = sizeof(T) == 2;  // bf16: masked-select bound, warp per row
   extern __shared__ __align__(16) float sm[];
   __shared__ int s_active[32];
   const int RQ = n_act * G;
-  float* qs = sm;                                            // [RQ][D]
-  uint32_t* qm = reinterpret_cast<uint32_t*>(qs + RQ * D);   // [RQ][D/2] (bf16)
-  T* sbuf = reinterpret_cast<T*>(qm + (kSel ? RQ * (D / 2) : 0));  // stages of [64][PS] min, max
-  float* sc = reinterpret_cast<float*>(sbuf + 2 * ps_stages((int)sizeof(T)) * kPsPages * PS);
+  float* qs = sm;                                    // [RQ][D]
+  T* sbuf = reinterpret_cast<T*>(qs + RQ * D);       // stages of [64][PS] min, max
+  float* sc = reinterpret_cast<float*>(sbuf + 2 * kPsStages * kPsPages * PS);
   const int hk = blockIdx.y, b = blockIdx.z;
   if (blockIdx.x == 0) {
     for (int w = threadIdx.x; w < words; w += blockDim.x)
@@ -530,32 +437,19 @@ __global__ void __launch_bounds__(256, 2)
   }
   const PageRing<T, D> ring{sbuf, pmin, pmax, kv, b, hk, c0, c1, n_pages};
   ring.prologue();
-  stage_q_rows<T, D>(q, act, b, B, Hq, G, hk, n_act, RQ, qs, qm);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, n_warps = blockDim.x >> 5;
+  stage_q_rows<T, D>(q, act, b, B, Hq, G, hk, n_act, RQ, qs);
   for (int ch = c0; ch < c1; ++ch) {
     ring.advance(ch);
     const T* smn = ring.mn(ch);
     const T* smx = ring.mx(ch);
     __syncthreads();  // chunk ch (and the q rows) visible to every thread
-    if constexpr (kSel) {
-      const int pg = (warp & 1) * 32 + lane;
+    for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
+      const int pg = task % kPsPages, rq = task / kPsPages;
       const int p = ch * kPsPages + pg;
-      for (int rq = warp >> 1; rq < RQ; rq += n_warps >> 1) {
-        const float yb = page_bound_sel<D>(qs + rq * D, qm + rq * (D / 2), smn + pg * PS,
-                                           smx + pg * PS);
-        const int a_i = rq / G, g = rq - (rq / G) * G;
-        if (p < n_pages)
-          scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = yb;
-      }
-    } else {
-      for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
-        const int pg = task % kPsPages, rq = task / kPsPages;
-        const int p = ch * kPsPages + pg;
-        if (p >= n_pages) continue;
-        const float yb = page_bound<T, D>(qs + rq * D, smn + pg * PS, smx + pg * PS);
-        const int a_i = rq / G, g = rq - (rq / G) * G;
-        scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = yb;
-      }
+      if (p >= n_pages) continue;
+      const float yb = page_bound<T, D>(qs + rq * D, smn + pg * PS, smx + pg * PS);
+      const int a_i = rq / G, g = rq - (rq / G) * G;
+      scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = yb;
     }
     __syncthreads();  // this chunk's buffer is refilled in the next iteration
   }
@@ -568,6 +462,249 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+__device__ __forceinline__ float order_key_inv(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// ---------------------------------------------------------------------------
+// Step 3a, bf16 summaries: the same bounds with the lanes on channels. A warp
+// scores a tile of kPcPages pages for kPcRows q rows at a time (32 bounds):
+// lane l holds the channel pairs l + 32 k (channels 2l, 2l + 1, 2l + 64, ...),
+// reads them for each page straight from global memory (a warp reads 128
+// contiguous bytes per load), and forms each channel's bound as
+//   fma(q-_c, kmin_c, q+_c * kmax_c),  q+ = max(q, 0), q- = min(q, 0),
+// which is max(q_c kmin_c, q_c kmax_c) exactly: one of the two products is
+// zero and the other is exact in fp32 (bf16 times bf16). The tree levels with
+// channel stride >= 64 are lane-local; the lane's pair (2l, 2l + 1) of each of
+// the 32 bounds then goes through a per-warp shared-memory transpose, and lane
+// o finishes bound o: levels of stride 32 .. 2 pair v[i] with v[i + s/2], the
+// last adds the pair's two channels. Every addition pairs the same channels in
+// the same order as the stride-halving tree, so each bound is that tree's sum.
+// Modes: per-row bounds of the active rows (one pass over a tile for up to
+// kPcRows rows, else several), or the sparse-residual head score: per page the
+// maximum of the bounds over every stacked row of the kv head (the four lanes
+// of a page fold their rows with two shuffles; the running maximum of a page
+// stays with one lane, which also folds it into the value stored by earlier
+// blocks of staged rows).
+// q rows are staged QR at a time as (q+ pair, q- pair) float4s; more rows
+// repeat the page loop. Grid (tile ranges, Hkv, batch), one wave.
+// ---------------------------------------------------------------------------
+constexpr int kPcPages = 8;     // pages per warp tile
+constexpr int kPcRows = 4;      // q rows per pass over a tile (kPcPages * kPcRows = 32)
+constexpr int kPcStride = 34;   // float2 per transpose row: 272 bytes, conflict-free float4 reads
+constexpr int kPcQRows = 64;      // q rows staged at a time (per-row bounds)
+constexpr int kPcQRowsHead = 32;  // the same for the head score (two CTAs per SM)
+constexpr int kPcThreads = 256;
+constexpr int kPcRowsOnePass = 0;  // modes: per-row bounds, at most kPcRows rows
+constexpr int kPcRowsMulti = 1;    //        per-row bounds, more rows
+constexpr int kPcHeadMax = 2;      //        per-page maximum over every stacked row
+
+__host__ __device__ constexpr int page_score_cols_smem(int RQ, int D, bool head_max) {
+  return ((RQ < (head_max ? kPcQRowsHead : kPcQRows) ? (RQ + kPcRows - 1) / kPcRows * kPcRows
+                                                     : (head_max ? kPcQRowsHead : kPcQRows)) *
+          (D / 2) * 16) +
+         (kPcThreads / 32) * 32 * kPcStride * 8;
+}
+
+template <int D, int kMode>
+__global__ void __launch_bounds__(kPcThreads, 2)
+    page_score_cols_kernel(const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ active,
+                           const float* __restrict__ row_scores, int32_t* __restrict__ active_out,
+                           int B, int Hq, int G, int n_act, const __nv_bfloat16* __restrict__ pmin,
+                           const __nv_bfloat16* __restrict__ pmax, const KvView kv,
+                           float* __restrict__ scores, uint32_t* __restrict__ bitmap, int words,
+                           int* __restrict__ tickets, int tpc) {
+  grid_dependency_wait();  // launched as a programmatic dependent
+  allow_dependent_launch();
+  static_assert(D % 64 == 0, "lanes hold D / 64 channel pairs");
+  constexpr int NPL = D / 64;  // channel pairs per lane
+  constexpr bool kOnePass = kMode == kPcRowsOnePass;
+  constexpr bool kHeadMax = kMode == kPcHeadMax;
+  constexpr int QR = kHeadMax ? kPcQRowsHead : kPcQRows;
+  extern __shared__ __align__(16) float sm[];
+  __shared__ int s_active[32];
+  const int RQ = n_act * G;
+  const int RQs = min((RQ + kPcRows - 1) / kPcRows * kPcRows, QR);  // staged rows
+  float4* qpn = reinterpret_cast<float4*>(sm);                            // [RQs][D/2]
+  float2* tr = reinterpret_cast<float2*>(qpn + RQs * (D / 2));            // [warps][32][stride]
+  float* sc = reinterpret_cast<float*>(tr + (kPcThreads / 32) * 32 * kPcStride);  // [B] (pick)
+  const int hk = blockIdx.y, b = blockIdx.z;
+  if (blockIdx.x == 0) {
+    for (int w = threadIdx.x; w < words; w += blockDim.x)
+      bitmap[((long long)b * kv.Hkv + hk) * words + w] = 0u;
+    if (tickets && threadIdx.x == 0) tickets[b * kv.Hkv + hk] = 0;
+  }
+  const int n_pages = (kv_tokens(kv, b) + kv.page_size - 1) / kv.page_size;
+  const int n_tiles = (n_pages + kPcPages - 1) / kPcPages;
+  const int t0 = blockIdx.x * tpc, t1 = min(t0 + tpc, n_tiles);
+  const bool pick = row_scores != nullptr;
+  if (t0 >= t1 && !(pick && blockIdx.x == 0 && hk == 0)) return;
+  const int* act = active ? active + b * n_act : nullptr;
+  if (pick) {
+    pick_active_rows(row_scores + (long long)b * B, B, n_act, sc, s_active);
+    if (blockIdx.x == 0 && hk == 0)
+      for (int r = threadIdx.x; r < n_act; r += blockDim.x) active_out[b * n_act + r] = s_active[r];
+    if (t0 >= t1) return;
+    act = s_active;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int nw = kPcThreads / 32;
+  float2* wtr = tr + warp * 32 * kPcStride;
+  const __nv_bfloat16* mn0 = pmin + ((long long)b * kv.max_pages * kv.Hkv + hk) * D;
+  const __nv_bfloat16* mx0 = pmax + ((long long)b * kv.max_pages * kv.Hkv + hk) * D;
+  uint32_t dmn[kPcPages][NPL], dmx[kPcPages][NPL];
+  // page pi of tile t: the clamped page is read for pages past the sequence
+  // (their bounds are never stored), so every load is unconditional
+  const int ps32 = kv.Hkv * (D / 2);  // 32-bit words from one page's row to the next
+  const uint32_t* mn32 = reinterpret_cast<const uint32_t*>(mn0) + lane;
+  const uint32_t* mx32 = reinterpret_cast<const uint32_t*>(mx0) + lane;
+  auto load_page = [&](int pi, int t) {
+    const int pc = min(t * kPcPages + pi, n_pages - 1);
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) {
+      dmn[pi][k] = __ldg(mn32 + pc * ps32 + 32 * k);
+      dmx[pi][k] = __ldg(mx32 + pc * ps32 + 32 * k);
+    }
+  };
+  float4 qv[kPcRows][NPL];
+  auto load_q = [&](int r0) {
+#pragma unroll
+    for (int r = 0; r < kPcRows; ++r)
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) qv[r][k] = qpn[(r0 + r) * (D / 2) + lane + 32 * k];
+  };
+  // one pass over a tile: the 32 bounds (kPcRows rows from staged row r0, the
+  // tile's pages) up to the lane-local levels, into the transpose buffer. With
+  // `reload`, each page's registers take page pi of tile tl as soon as they
+  // are unpacked, so the next tile's loads overlap almost the whole pass.
+  auto pass_bounds = [&](auto reload, int tl) {
+#pragma unroll
+    for (int pi = 0; pi < kPcPages; ++pi) {
+      float2 n[NPL], x[NPL];
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) {
+        n[k] = make_float2(__uint_as_float(dmn[pi][k] << 16),
+                           __uint_as_float(dmn[pi][k] & 0xFFFF0000u));
+        x[k] = make_float2(__uint_as_float(dmx[pi][k] << 16),
+                           __uint_as_float(dmx[pi][k] & 0xFFFF0000u));
+      }
+      if constexpr (decltype(reload)::value) load_page(pi, tl);
+#pragma unroll
+      for (int r = 0; r < kPcRows; ++r) {
+        float2 s[NPL];
+#pragma unroll
+        for (int k = 0; k < NPL; ++k)
+          s[k] = ffma2(make_float2(qv[r][k].z, qv[r][k].w), n[k],
+                       fmul2(make_float2(qv[r][k].x, qv[r][k].y), x[k]));
+#pragma unroll
+        for (int st = NPL / 2; st >= 1; st >>= 1)  // channel strides D/2 .. 64
+#pragma unroll
+          for (int k = 0; k < st; ++k) s[k] = fadd2(s[k], s[k + st]);
+        wtr[(r * kPcPages + pi) * kPcStride + lane] = s[0];
+      }
+    }
+    __syncwarp();
+  };
+  // one pass: lane o's bound row (row o / kPcPages of rows 0..3), or NULL past RQ
+  float* out_row = nullptr;
+  if (kOnePass && lane / kPcPages < RQ) {
+    const int rq = lane / kPcPages, a_i = rq / G, g = rq - (rq / G) * G;
+    out_row = scores + (((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages;
+  }
+  uint32_t hmax = 0u;  // head score: running maximum key of page (lane % kPcPages)
+  // ... then lane o finishes bound o and stores it (head score: folds it)
+  auto pass_finish = [&](int t, int r0, int row_base) {
+    // float4 j of the row holds pairs 2j and 2j + 1 (channels 4j .. 4j + 3)
+    const float4* row = reinterpret_cast<const float4*>(wtr + lane * kPcStride);
+    float2 v[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      // channel strides 32 then 16: ((i + (i+16)) + ((i+8) + (i+24))) for pairs i = 2j, 2j + 1
+      const float4 a = row[j], b8 = row[j + 4], c = row[j + 8], d = row[j + 12];
+      v[2 * j] = fadd2(fadd2(make_float2(a.x, a.y), make_float2(c.x, c.y)),
+                       fadd2(make_float2(b8.x, b8.y), make_float2(d.x, d.y)));
+      v[2 * j + 1] = fadd2(fadd2(make_float2(a.z, a.w), make_float2(c.z, c.w)),
+                           fadd2(make_float2(b8.z, b8.w), make_float2(d.z, d.w)));
+    }
+#pragma unroll
+    for (int st = 4; st >= 1; st >>= 1)  // channel strides 8 .. 2
+#pragma unroll
+      for (int i = 0; i < st; ++i) v[i] = fadd2(v[i], v[i + st]);
+    const float y = __fadd_rn(v[0].x, v[0].y);  // channel 0 + channel 1
+    __syncwarp();  // the buffer is rewritten by the next pass
+    const int p = t * kPcPages + (lane & (kPcPages - 1));
+    if constexpr (kHeadMax) {
+      const int rq = row_base + r0 + lane / kPcPages;
+      uint32_t key = (p < n_pages && rq < RQ) ? order_key(y) : 0u;  // 0: below every key
+      key = max(key, __shfl_xor_sync(0xffffffffu, key, kPcPages));
+      key = max(key, __shfl_xor_sync(0xffffffffu, key, 2 * kPcPages));
+      hmax = max(hmax, key);
+    } else if (p < n_pages) {
+      if constexpr (kOnePass) {
+        if (out_row) out_row[p] = y;
+      } else {
+        const int rq = row_base + r0 + lane / kPcPages;
+        if (rq < RQ) {
+          const int a_i = rq / G, g = rq - (rq / G) * G;
+          scores[(((long long)b * n_act + a_i) * Hq + hk * G + g) * kv.max_pages + p] = y;
+        }
+      }
+    }
+  };
+  for (int row_base = 0; row_base < RQ; row_base += QR) {
+    if (row_base > 0) __syncthreads();  // every warp is done with the previous rows
+    for (int idx = threadIdx.x; idx < RQs * (D / 2); idx += blockDim.x) {
+      const int rr = idx / (D / 2), c2 = idx - rr * (D / 2);
+      const int rq = row_base + rr;
+      float2 v = make_float2(0.f, 0.f);
+      if (rq < RQ) {
+        const int a_i = rq / G, g = rq - a_i * G;
+        const int i = act ? act[a_i] : a_i;
+        const uint32_t u = *reinterpret_cast<const uint32_t*>(
+            q + (((long long)b * B + i) * Hq + hk * G + g) * D + 2 * c2);
+        v = make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+      }
+      qpn[idx] = make_float4(v.x >= 0.f ? v.x : 0.f, v.y >= 0.f ? v.y : 0.f,
+                             v.x < 0.f ? v.x : 0.f, v.y < 0.f ? v.y : 0.f);
+    }
+    __syncthreads();
+    const int rows_here = min(RQ - row_base, QR);
+    int t = t0 + warp;
+    if (t < t1)
+#pragma unroll
+      for (int pi = 0; pi < kPcPages; ++pi) load_page(pi, t);
+    if constexpr (kOnePass) load_q(0);
+    for (; t < t1; t += nw) {
+      // the last pass over a tile reloads the page registers with the next
+      // tile (the warp's last tile reloads itself: the loads stay unconditional)
+      const int tl = t + nw < t1 ? t + nw : t;
+      if constexpr (kOnePass) {
+        pass_bounds(std::true_type{}, tl);
+        pass_finish(t, 0, row_base);
+      } else {
+        hmax = 0u;
+        for (int r0 = 0; r0 < rows_here; r0 += kPcRows) {
+          load_q(r0);
+          if (r0 + kPcRows >= rows_here)
+            pass_bounds(std::true_type{}, tl);
+          else
+            pass_bounds(std::false_type{}, tl);
+          pass_finish(t, r0, row_base);
+        }
+        if constexpr (kHeadMax) {
+          const int p = t * kPcPages + lane;
+          if (lane < kPcPages && p < n_pages) {
+            // the same lane holds this page in every block of staged rows
+            float* dst = scores + ((long long)b * kv.Hkv + hk) * kv.max_pages + p;
+            *dst = order_key_inv(row_base == 0 ? hmax : max(hmax, order_key(*dst)));
+          }
+        }
+      }
+    }
+  }
+}
+
+
 // ---------------------------------------------------------------------------
 // Step 3b: top-k pages of one (active row, q head): exact radix select of the
 // k-th largest key (4 passes of 8 bits), then every key above it plus the
@@ -579,6 +716,9 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 // list and count.
 // ---------------------------------------------------------------------------
 constexpr int kTopkThreads = 512;
+constexpr int kTopkDigitBits = 12;  // radix digit width of the top-k select
+constexpr int kTopkBinsPerThread = (1 << kTopkDigitBits) / kTopkThreads;
+constexpr int kTopkLoads = 16;      // score loads in flight per thread
 
 // Exclusive prefix sum over the CTA (blockDim a multiple of 32, at most 1024)
 // of one value per thread; total receives the sum. Ends with a barrier.
@@ -638,11 +778,10 @@ __global__ void __launch_bounds__(kTopkThreads)
   grid_dependency_wait();  // launched as a programmatic dependent
   allow_dependent_launch();
   extern __shared__ uint32_t keys[];  // max_pages keys, then a words-long bitmap
-  __shared__ int hist[256];
-  __shared__ int whist[kTopkThreads / 32][256];  // per-warp digit counts
+  __shared__ int hist[1 << kTopkDigitBits];
   __shared__ int warp_sums[33];
-  __shared__ uint32_t s_prefix;
-  __shared__ int s_need, s_last;
+  __shared__ uint32_t s_prefix, s_kmin[kTopkThreads / 32], s_kmax[kTopkThreads / 32];
+  __shared__ int s_need, s_neq, s_last;
   const int ah = blockIdx.x, b = blockIdx.y;
   const int h = ah % Hq;
   const int hk = h / G;
@@ -652,115 +791,142 @@ __global__ void __launch_bounds__(kTopkThreads)
   uint32_t* sbm = keys + kv.max_pages;
   uint32_t* bm = bitmap + ((long long)b * kv.Hkv + hk) * words;
   const float* sc = scores + ((long long)b * n_act * Hq + ah) * kv.max_pages;
-  for (int w = tid; w < words; w += blockDim.x) sbm[w] = 0u;
-  auto take = [&](int p) { atomicOr(&sbm[p >> 5], 1u << (p & 31)); };
-  if (k == n) {
-    __syncthreads();
-    for (int p = tid; p < n; p += blockDim.x) take(p);
-  } else if (k > 0) {
-    // the scores, 8 loads in flight per thread (a loop of single loads would
-    // pay the memory latency once per key it reads)
-    for (int p0 = tid; p0 < n; p0 += 8 * blockDim.x) {
-      float v[8];
+  const int lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  if (k <= 0) {
+    for (int w = tid; w < words; w += blockDim.x) sbm[w] = 0u;
+  } else if (k >= n) {  // every page of the sequence
+    for (int w = tid; w < words; w += blockDim.x) {
+      const int p0 = 32 * w;
+      sbm[w] = p0 + 32 <= n ? 0xFFFFFFFFu : (p0 < n ? (1u << (n - p0)) - 1u : 0u);
+    }
+  } else {
+    // The scores as order-preserving keys (a thread's loads all in flight at
+    // once), with the smallest and largest key on the way.
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    for (int p0 = tid; p0 < n; p0 += kTopkLoads * blockDim.x) {
+      float v[kTopkLoads];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < kTopkLoads; ++u) {
         const int p = p0 + u * blockDim.x;
         v[u] = p < n ? __ldcg(sc + p) : 0.f;
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < kTopkLoads; ++u) {
         const int p = p0 + u * blockDim.x;
-        if (p < n) keys[p] = order_key(v[u]);
+        if (p < n) {
+          const uint32_t key = order_key(v[u]);
+          keys[p] = key;
+          lo = min(lo, key);
+          hi = max(hi, key);
+        }
       }
     }
-    if (tid == 0) {
-      s_prefix = 0u;
-      s_need = k;
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    if (lane == 0) {
+      s_kmin[warp] = lo;
+      s_kmax[warp] = hi;
     }
-    uint32_t mask = 0u;
-    const int wid = tid >> 5;
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      for (int d = tid; d < (kTopkThreads / 32) * 256; d += blockDim.x) (&whist[0][0])[d] = 0;
+    __syncthreads();
+    lo = 0xFFFFFFFFu;
+    hi = 0u;
+    for (int w = 0; w < nw; ++w) {
+      lo = min(lo, s_kmin[w]);
+      hi = max(hi, s_kmax[w]);
+    }
+    // Radix select of the k-th largest key T. The bits every key shares (the
+    // common prefix of the smallest and largest key) are fixed at once; the
+    // rest are resolved kTopkDigitBits at a time, most significant first, each
+    // pass counting only the keys that match the bits fixed so far.
+    int free_bits = (lo ^ hi) ? 32 - __clz(lo ^ hi) : 0;  // bits below the common prefix
+    uint32_t mask = free_bits == 32 ? 0u : ~((1u << free_bits) - 1u);
+    uint32_t prefix = hi & mask;
+    int need = k;   // keys equal to the prefix still to take
+    int n_eq = n;   // keys equal to the prefix
+    while (free_bits > 0) {
+      const int w = free_bits < kTopkDigitBits ? free_bits : kTopkDigitBits;
+      const int shift = free_bits - w;
+      const int nb = 1 << w;
+      for (int d = tid; d < nb; d += blockDim.x) hist[d] = 0;
       __syncthreads();
-      const uint32_t prefix = s_prefix;
-      // Scores of one row are alike, so a few digits take most keys (all of
-      // them share one in the first pass): each warp counts into its own
-      // histogram, so only a warp's own lanes contend for a counter.
       for (int p = tid; p < n; p += blockDim.x) {
         const uint32_t key = keys[p];
-        if ((key & mask) == prefix) atomicAdd(&whist[wid][(key >> shift) & 0xFFu], 1);
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1);
       }
       __syncthreads();
-      for (int d = tid; d < 256; d += blockDim.x) {
-        int c = 0;
+      // digits in descending order: thread t owns the kTopkBinsPerThread
+      // digits below nb - 1 - t * kTopkBinsPerThread
+      int cnt[kTopkBinsPerThread], tot = 0;
 #pragma unroll
-        for (int w = 0; w < kTopkThreads / 32; ++w) c += whist[w][d];
-        hist[d] = c;
+      for (int j = 0; j < kTopkBinsPerThread; ++j) {
+        const int d = nb - 1 - tid * kTopkBinsPerThread - j;
+        cnt[j] = d >= 0 ? hist[d] : 0;
+        tot += cnt[j];
       }
-      __syncthreads();
-      if (tid < 32) {
-        // buckets in descending order: lane l owns digits 255-8l ... 248-8l
-        int cnt[8], tot = 0;
+      int total;
+      const int before = block_exclusive_scan(tot, warp_sums, total);
+      if (before < need && before + tot >= need) {  // exactly one thread
+        int cum = before;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          cnt[j] = hist[255 - 8 * tid - j];
-          tot += cnt[j];
-        }
-        int incl = tot;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (tid >= o) incl += v;
-        }
-        const int need = s_need;
-        const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
-        const int owner = __ffs(hit) - 1;  // first lane whose running count reaches need
-        if (tid == owner) {
-          int cum = incl - tot, sel = 0, rem = need;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (cum + cnt[j] >= need) {
-              sel = 255 - 8 * tid - j;
-              rem = need - cum;
-              break;
-            }
-            cum += cnt[j];
+        for (int j = 0; j < kTopkBinsPerThread; ++j) {
+          if (cum + cnt[j] >= need) {
+            s_prefix = prefix | ((uint32_t)(nb - 1 - tid * kTopkBinsPerThread - j) << shift);
+            s_need = need - cum;
+            s_neq = cnt[j];
+            break;
           }
-          s_prefix = prefix | ((uint32_t)sel << shift);
-          s_need = rem;
+          cum += cnt[j];
         }
       }
-      mask |= 0xFFu << shift;
       __syncthreads();
+      prefix = s_prefix;
+      need = s_need;
+      n_eq = s_neq;
+      mask |= (uint32_t)(nb - 1) << shift;
+      free_bits = shift;
     }
-    const uint32_t T = s_prefix;  // key of the k-th largest score
-    const int need = s_need;      // how many keys equal to T are taken
-    // every key above T; count the keys equal to it
-    int eq = 0;
-    for (int p = tid; p < n; p += blockDim.x) {
-      const uint32_t key = keys[p];
-      if (key > T) take(p);
-      eq += key == T;
-    }
-    int n_eq;
-    block_exclusive_scan(eq, warp_sums, n_eq);
+    const uint32_t T = prefix;  // the k-th largest key; `need` of the n_eq keys equal to it are taken
+    // Selection words, one per warp step (bit i of word w: page 32 w + i): every
+    // key above T, and the keys equal to T -- all of them, or where more equal
+    // T than are taken, the lowest pages.
     if (n_eq == need) {
-      for (int p = tid; p < n; p += blockDim.x)
-        if (keys[p] == T) take(p);
+      for (int w = warp; w < words; w += nw) {
+        const int p = 32 * w + lane;
+        const unsigned bits = __ballot_sync(0xffffffffu, p < n && keys[p] >= T);
+        if (lane == 0) sbm[w] = bits;
+      }
     } else {
-      // more keys equal the k-th largest than are taken: the lowest indices,
-      // from a scan over per-thread index segments (thread order = index order)
-      const int seg = (n + blockDim.x - 1) / blockDim.x;
-      const int p0 = tid * seg, p1 = min(n, p0 + seg);
-      int cnt = 0;
-      for (int p = p0; p < p1; ++p) cnt += (keys[p] == T);
-      int tot;
-      int eq_before = block_exclusive_scan(cnt, warp_sums, tot);
-      for (int p = p0; p < p1; ++p) {
-        if (keys[p] == T) {
-          if (eq_before < need) take(p);
-          ++eq_before;
+      for (int w = warp; w < words; w += nw) {  // equal keys per word
+        const int p = 32 * w + lane;
+        const unsigned eq = __ballot_sync(0xffffffffu, p < n && keys[p] == T);
+        if (lane == 0) hist[w] = __popc(eq);
+      }
+      __syncthreads();
+      const int per = (words + blockDim.x - 1) / blockDim.x;  // words per thread, in order
+      const int w0 = tid * per, w1 = min(words, w0 + per);
+      int c = 0;
+      for (int w = w0; w < w1; ++w) c += hist[w];
+      int total;
+      int before = block_exclusive_scan(c, warp_sums, total);
+      for (int w = w0; w < w1; ++w) {  // equal keys in the words before w
+        const int cw = hist[w];
+        hist[w] = before;
+        before += cw;
+      }
+      __syncthreads();
+      for (int w = warp; w < words; w += nw) {
+        const int p = 32 * w + lane;
+        const uint32_t key = p < n ? keys[p] : 0u;
+        const unsigned gt = __ballot_sync(0xffffffffu, p < n && key > T);
+        unsigned eq = __ballot_sync(0xffffffffu, p < n && key == T);
+        if (lane == 0) {
+          unsigned take = 0u;
+          for (int left = need - hist[w]; left > 0 && eq; --left) {
+            const unsigned low = eq & (0u - eq);  // lowest equal page of the word
+            take |= low;
+            eq ^= low;
+          }
+          sbm[w] = gt | take;
         }
       }
     }
@@ -784,7 +950,8 @@ __global__ void __launch_bounds__(kTopkThreads)
 // with sparse attention): the sparse selector scores pages per kv head by the
 // same QUEST-style bound, taking the maximum over every block row and every q
 // head of the kv head: head score of page p = max_{i,g} tree_sum_c
-// max(q_c kmin_c, q_c kmax_c). The per-(row, head) bound is formed exactly as in
+// max(q_c kmin_c, q_c kmax_c). For float32 summaries (bf16: the head-score mode
+// of page_score_cols_kernel) the per-(row, head) bound is formed exactly as in
 // page_score_kernel (single-rounded products, stride-halving tree); the maximum
 // is order-free, taken on order-preserving keys with shared-memory atomics.
 // scores: [batch, Hkv, max_pages]. Block (0, hk, b) clears the (b, hk) bitmap.
@@ -794,9 +961,6 @@ __global__ void __launch_bounds__(kTopkThreads)
 // ---------------------------------------------------------------------------
 constexpr int kHsRows = 64;
 
-__device__ __forceinline__ float order_key_inv(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
-}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(256, 2)
@@ -807,15 +971,14 @@ __global__ void __launch_bounds__(256, 2)
                            int cpc) {
   grid_dependency_wait();  // launched as a programmatic dependent
   allow_dependent_launch();
+  static_assert(sizeof(T) == 4, "float32 summaries (bf16: page_score_cols_kernel)");
   constexpr int PS = ps_stride<T, D>();
-  constexpr bool kSel = sizeof(T) == 2;  // bf16: masked-select bound, warp per row
   extern __shared__ __align__(16) float sm[];
   __shared__ uint32_t best[kPsPages];
   const int RQ_all = B * G;
   const int RQmax = RQ_all < kHsRows ? RQ_all : kHsRows;
-  float* qs = sm;                                              // [RQmax][D], row r = i * G + g
-  uint32_t* qm = reinterpret_cast<uint32_t*>(qs + RQmax * D);  // [RQmax][D/2] (bf16)
-  T* sbuf = reinterpret_cast<T*>(qm + (kSel ? RQmax * (D / 2) : 0));  // stages of [64][PS]
+  float* qs = sm;                                  // [RQmax][D], row r = i * G + g
+  T* sbuf = reinterpret_cast<T*>(qs + RQmax * D);  // stages of [64][PS]
   const int hk = blockIdx.y, b = blockIdx.z;
   if (blockIdx.x == 0) {
     for (int w = threadIdx.x; w < words; w += blockDim.x)
@@ -827,33 +990,24 @@ __global__ void __launch_bounds__(256, 2)
   const int c1 = min(c0 + cpc, (n_pages + kPsPages - 1) / kPsPages);
   if (c0 >= c1) return;
   const PageRing<T, D> ring{sbuf, pmin, pmax, kv, b, hk, c0, c1, n_pages};
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, n_warps = blockDim.x >> 5;
   for (int row0 = 0; row0 < RQ_all; row0 += kHsRows) {
   const int RQ = RQ_all - row0 < kHsRows ? RQ_all - row0 : kHsRows;
   ring.prologue();
-  stage_q_rows<T, D>(q, nullptr, b, B, Hq, G, hk, B, RQ, qs, qm, row0);
+  stage_q_rows<T, D>(q, nullptr, b, B, Hq, G, hk, B, RQ, qs, row0);
   for (int ch = c0; ch < c1; ++ch) {
     for (int pg = threadIdx.x; pg < kPsPages; pg += blockDim.x) best[pg] = 0u;  // below every key
     ring.advance(ch);
     const T* smn = ring.mn(ch);
     const T* smx = ring.mx(ch);
     __syncthreads();  // chunk ch, the q rows and the cleared maxima visible to every thread
-    if constexpr (kSel) {
-      const int pg = (warp & 1) * 32 + lane;
-      uint32_t mx = 0u;  // below every key
-      for (int rq = warp >> 1; rq < RQ; rq += n_warps >> 1)
-        mx = max(mx, order_key(page_bound_sel<D>(qs + rq * D, qm + rq * (D / 2), smn + pg * PS,
-                                                  smx + pg * PS)));
-      if (ch * kPsPages + pg < n_pages) atomicMax(&best[pg], mx);
-    } else {
-      for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
-        const int pg = task % kPsPages, rq = task / kPsPages;
-        const int p = ch * kPsPages + pg;
-        if (p >= n_pages) continue;
-        const float yb = page_bound<T, D>(qs + rq * D, smn + pg * PS, smx + pg * PS);
-        atomicMax(&best[pg], order_key(yb));
-      }
+    for (int task = threadIdx.x; task < kPsPages * RQ; task += blockDim.x) {
+      const int pg = task % kPsPages, rq = task / kPsPages;
+      const int p = ch * kPsPages + pg;
+      if (p >= n_pages) continue;
+      const float yb = page_bound<T, D>(qs + rq * D, smn + pg * PS, smx + pg * PS);
+      atomicMax(&best[pg], order_key(yb));
     }
+
     __syncthreads();
     for (int pg = threadIdx.x; pg < kPsPages; pg += blockDim.x) {
       const int p = ch * kPsPages + pg;

@@ -103,6 +103,22 @@ size_t fb_workspace_size(const fb_kv* kv, int32_t block, int32_t n_heads_q, int3
                          int32_t topk_pages, int32_t num_sms);
 
 /*
+ * Byte offset, inside a workspace sized by fb_workspace_size with the same
+ * arguments, of the page scores that losa_select (and fb_step in LOSA mode)
+ * leave there ([LoSA] section 2, step 3: the page bound of each active row):
+ * float32 [batch, min(n_active, block), n_heads_q, pages], pages = the
+ * logical page count per sequence (max_pages_per_seq for a paged cache,
+ * ceil(max_seq_len / page_size) otherwise); entry (b, a, h, p) is the bound of
+ * the a-th active row (rank order) under q head h over page p, written for the
+ * sequence's own pages only. For inspection and tests: the next selection
+ * that uses the workspace overwrites them.
+ * Returns 0 on invalid arguments or when n_active or topk_pages is 0 (no
+ * scores); a valid offset is never 0.
+ */
+size_t fb_workspace_page_scores(const fb_kv* kv, int32_t block, int32_t n_heads_q,
+                                int32_t n_active, int32_t topk_pages, int32_t num_sms);
+
+/*
  * Block-external partial ([FB] section 2: A_out and L_out = log Z_out over J_out).
  * For every block row i and q head h:
  *   L_out = log sum_{t < seq_len[b]} exp(scale * <q_i,h , k_t>)

@@ -233,7 +233,7 @@ def test_losa_select_is_bit_exact(ov, n_active, topk):
     wl = _losa_small(**ov)
     steps = list(wl.steps(2))
     q_prev, q_cur = steps[0].q, steps[1].q
-    kv, act, rs, bm, ul, uc, _ = run_select(wl, q_cur, q_prev, n_active, topk)
+    kv, act, rs, bm, ul, uc, ws = run_select(wl, q_cur, q_prev, n_active, topk)
     score = olosa.locality_score(q_cur, q_prev, "bf16")
     np.testing.assert_array_equal(cpu(rs), score)  # bit-exact float32 tree
     act_ref = olosa.active_rows(score, n_active)
@@ -241,7 +241,44 @@ def test_losa_select_is_bit_exact(ov, n_active, topk):
     smin, smax = olosa.page_summary(wl.prefix, "bf16")
     _, union = olosa.select_pages(wl.prefix, q_cur, "bf16", act_ref, topk, smin, smax)
     npg = kv.n_pages
+    # every page bound, bit-exact (not only the ones near each top-k boundary)
+    sp = wl.spec
+    na, Hq, G = act_ref.shape[1], sp.n_heads_q, sp.n_heads_q // sp.n_heads_kv
+    off = fb.fb_workspace_page_scores(kv, sp.block, Hq, n_active, topk)
+    sc = cpu(ws[off:off + kv.batch * na * Hq * npg * 4].view(torch.float32)).reshape(
+        kv.batch, na, Hq, npg)
+    qf = olosa.to_f32(q_cur, "bf16")
+    for b in range(kv.batch):
+        n = -(-int(wl.prefix.seq_len[b]) // 16)
+        for h in range(Hq):
+            ref = olosa.page_scores(qf[b, act_ref[b], h], smin[b, :n, h // G], smax[b, :n, h // G])
+            np.testing.assert_array_equal(sc[b, :, h, :n], ref, err_msg=f"b={b} h={h}")
     bm_ref = olosa.union_bitmap(union, kv.batch, kv.c.n_heads_kv, npg)
+    np.testing.assert_array_equal(cpu(bm).view(np.uint32), bm_ref)
+    for (b, hk), pages in union.items():
+        assert int(cpu(uc)[b, hk]) == len(pages)
+        np.testing.assert_array_equal(cpu(ul)[b, hk, :len(pages)], pages)
+
+
+@pytest.mark.parametrize("period,topk", [(1, 20), (3, 7), (3, 100)])
+def test_losa_select_breaks_page_ties_by_lower_page(period, topk):
+    """Pages repeat with the given period (every page a copy of one of `period`
+    distinct pages), so many page bounds are equal and the k-th largest is
+    shared by more pages than are taken: the union must hold the lowest such
+    pages, as the oracle's selection does."""
+    wl = _losa_small()
+    pre = wl.prefix
+    n = int(pre.seq_len[0])
+    t = np.arange(pre.k.shape[0]) % n  # position within its sequence
+    src = (t // 16 % period) * 16 + t % 16 + (np.arange(pre.k.shape[0]) // n) * n
+    pre.k[:] = pre.k[src]
+    steps = list(wl.steps(2))
+    q_prev, q_cur = steps[0].q, steps[1].q
+    kv, act, rs, bm, ul, uc, ws = run_select(wl, q_cur, q_prev, 4, topk)
+    act_ref = olosa.active_rows(olosa.locality_score(q_cur, q_prev, "bf16"), 4)
+    smin, smax = olosa.page_summary(wl.prefix, "bf16")
+    _, union = olosa.select_pages(wl.prefix, q_cur, "bf16", act_ref, topk, smin, smax)
+    bm_ref = olosa.union_bitmap(union, kv.batch, kv.c.n_heads_kv, kv.n_pages)
     np.testing.assert_array_equal(cpu(bm).view(np.uint32), bm_ref)
     for (b, hk), pages in union.items():
         assert int(cpu(uc)[b, hk]) == len(pages)
