@@ -711,7 +711,8 @@ int block_attn_short_f32(const void* q, const void* k_in, const void* v_in, int 
 int block_attn_impl(const void* q, const void* k_in, const void* v_in, int batch, int B, int Hq,
                     int Hkv, int D, float scale, fb_dtype dt, float* a_in, float* l_in,
                     cudaStream_t stream, const float* mrg_a = nullptr,
-                    const float* mrg_l = nullptr, const int32_t* cu = nullptr, int total = 0) {
+                    const float* mrg_l = nullptr, const int32_t* cu = nullptr, int total = 0,
+                    void* ws = nullptr, size_t ws_bytes = 0, size_t ws_offset = 0) {
   fb_kv kv{};
   kv.k = k_in;
   kv.v = v_in;
@@ -752,6 +753,39 @@ int block_attn_impl(const void* q, const void* k_in, const void* v_in, int batch
   c.q_cu = cu;
   c.q_total = total;
   c.kv_cu = cu;
+  // One sequence, one q head per kv head, a last 256-row tile of at most 64
+  // rows (a video block of 1560 rows: 6 full tiles and 24 rows): that tile
+  // would cost a whole tcgen05 CTA and push the grid (7 tiles x heads) into a
+  // second wave. With workspace lent by the caller (fb_step), the full tiles
+  // run on the tcgen05 kernel (one wave) and the last rows on the streaming
+  // kernel, split over the block's keys (read from L2); each part merges its
+  // own rows. (Without workspace the last rows' single split per row tile
+  // streams every key tile in turn and gains nothing: measured 106 vs 101 us.)
+  const int tail = B % kT2Rows;
+  if (ws && !cu && batch == 1 && Hq == Hkv && use_tc(dt, D, B) && B > kT2Rows && tail > 0 &&
+      tail <= 64) {
+    PartialCall ct = c;
+    const size_t eb = elem_size(dt);
+    const long long r0 = (long long)(B - tail) * Hq;  // first (row, head) of the last rows
+    ct.q = static_cast<const char*>(q) + r0 * D * eb;
+    ct.B = tail;
+    ct.a_out = a_in + r0 * D;
+    ct.l_out = l_in + r0;
+    ct.mrg_a = mrg_a ? mrg_a + r0 * D : nullptr;
+    ct.mrg_l = mrg_l ? mrg_l + r0 : nullptr;
+    // the tail's split partials must fit the region the caller lent
+    const Plan pt = make_plan(dt, 1, Hkv, tail, ceil_div(B, kTK), c.num_sms, D);
+    const size_t need = partial_bytes(pt, 1, Hkv, tail, D);
+    ct.single_split = false;
+    ct.ws = ws;
+    ct.ws_bytes = ws_bytes;
+    ct.ws_offset = ws_offset;
+    if (aligned16(ct.q) && aligned16(ws) && ws_offset + need <= ws_bytes) {
+      c.B = B - tail;
+      if ((rc = launch_partial(c, stream))) return rc;
+      return launch_partial(ct, stream);
+    }
+  }
   return launch_partial(c, stream);
 }
 
@@ -1299,8 +1333,11 @@ static int step_impl(const fb_policy* policy, fb_cache* cache, const void* q, co
   // block-internal partial and the FlashBlock merge with the cached
   // block-external partial in one kernel: A_full directly
   float* lf = l_full ? l_full : reinterpret_cast<float*>(ws + w.l_in);
+  // (the in-block call may use the split-partial region of the workspace: the
+  // prefix partial's combine, earlier on the stream, is done with it)
   rc = block_attn_impl(q, k_in, v_in, batch, B, Hq, Hkv, D, policy->scale, prefix->dtype, a_full,
-                       lf, stream, cache->a_out, cache->l_out, cu, total);
+                       lf, stream, cache->a_out, cache->l_out, cu, total, workspace, w.scores,
+                       w.part);
   if (rc) return rc;
   cache->step = s + 1;
   return FB_OK;

@@ -122,6 +122,8 @@ def test_prefix_attn_empty_and_short_sequences():
     ("dllm", dict(block=33, head_dim=64, n_heads_q=4, n_heads_kv=2, prefix_min=64,
                   prefix_max=64)),
     ("video", dict(block=65, n_heads_q=2, n_heads_kv=2, prefix_min=64, prefix_max=64)),
+    # one sequence, 290 rows (a full 256-row tile and 34 rows) on the tcgen05 kernel
+    ("video", dict(block=290, n_heads_q=2, n_heads_kv=2, prefix_min=64, prefix_max=64)),
     # fp32 short-block kernel: one token, head_dim 128 with GQA stacking and keys past
     # 32, a full 64-token block with 256 stacked rows over 3 sequences; the last case
     # stacks too many rows for its shared memory and takes the general kernel

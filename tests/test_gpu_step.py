@@ -76,6 +76,28 @@ def test_threshold_steps_with_an_empty_prefix_side(name):
         assert_close_L(cpu(L), ref["L_full"], f"step {st.step}")
 
 
+@pytest.mark.parametrize("block,tau", [(300, 0), (300, 3), (520, 0)])
+def test_long_single_sequence_block_with_a_short_last_row_tile(block, tau):
+    """One sequence, one q head per kv head, more than 256 block rows with at
+    most 64 in the last 256-row tile: fb_step runs the full tiles on the
+    tcgen05 kernel and the last rows on the streaming kernel (split over the
+    block's keys); every row must match the oracle, merge included."""
+    wl = make_workload("video", prefix_min=1200, prefix_max=1200, block=block, n_heads_q=3,
+                       n_heads_kv=3, steps=3)
+    sp = wl.spec
+    kv = make_kv(wl.prefix, sp.dtype)
+    blk = BlockAttention(kv, sp.block, sp.n_heads_q, "threshold", tau=tau)
+    ctl = ThresholdController(wl.prefix, sp.dtype, tau)
+    A, L = _out(sp)
+    for st in wl.steps():
+        blk.step(dev(st.q, sp.dtype), dev(st.k_in, sp.dtype), dev(st.v_in, sp.dtype), A, L,
+                 m_updated=st.m_updated)
+        ref = ctl.step(st.step, st.q, st.k_in, st.v_in, st.m_updated)
+        sync()
+        assert_close_A(cpu(A), ref["A_full"], sp.dtype, f"step {st.step}")
+        assert_close_L(cpu(L), ref["L_full"], f"step {st.step}")
+
+
 def test_per_head_steps_match_oracle_with_bit_exact_cosine_replay():
     wl = make_workload("video", prefix_min=700, prefix_max=700, block=90, n_heads_q=6,
                        n_heads_kv=6, steps=8)
