@@ -400,6 +400,46 @@ int validate_scale(float scale) {
 
 int launch_partial(const PartialCall& c, cudaStream_t stream) {
   if (int rc_ = validate_scale(c.scale)) return rc_;
+  {
+    // One sequence whose stacked rows leave a last 256-row tile of at most 64
+    // rows (a video block of 1560 rows: 6 full tiles and 24 rows): on the
+    // tcgen05 kernel that tile costs as much as a full one and pushes the grid
+    // into another wave (video prefix: 7 x 24 tiles x 4 splits = 4.5 waves).
+    // With a workspace, the full tiles run on the tcgen05 kernel (video: 144
+    // CTAs, one wave, no split) and the last rows on the streaming kernel,
+    // which reads the key set once more at its HBM rate; each part writes (and
+    // merges) its own rows.
+    const fb_kv* kv = c.kv;
+    const int G = c.Hq / kv->n_heads_kv, R = c.B * G, tail = R % kT2Rows;
+    if (!c.single_split && c.ws && kv->batch == 1 && !c.q_cu && !c.row_list && !c.page_list &&
+        use_tc(kv->dtype, kv->head_dim, R) && R > kT2Rows && tail > 0 && tail <= 64 &&
+        tail % G == 0) {
+      const int Bt = tail / G, Bm = c.B - Bt;
+      const int max_tiles = ceil_div(kv->max_seq_len, kTK);
+      const Plan pm = make_plan(kv->dtype, 1, kv->n_heads_kv, Bm * G, max_tiles, c.num_sms,
+                                kv->head_dim);
+      const Plan pt = make_plan(kv->dtype, 1, kv->n_heads_kv, tail, max_tiles, c.num_sms,
+                                kv->head_dim);
+      const size_t nm = partial_bytes(pm, 1, kv->n_heads_kv, Bm * G, kv->head_dim);
+      const size_t nt = partial_bytes(pt, 1, kv->n_heads_kv, tail, kv->head_dim);
+      const long long r0 = (long long)Bm * c.Hq;  // first (row, head) of the last rows
+      const int D = kv->head_dim;
+      const void* qt = static_cast<const char*>(c.q) + r0 * D * elem_size(kv->dtype);
+      if (c.ws_offset + (nm > nt ? nm : nt) <= c.ws_bytes && aligned16(qt)) {
+        PartialCall cm = c, ct = c;
+        cm.B = Bm;
+        ct.q = qt;
+        ct.B = Bt;
+        ct.a_out = c.a_out + r0 * D;
+        ct.l_out = c.l_out + r0;
+        ct.a_prev = c.a_prev ? c.a_prev + r0 * D : nullptr;
+        ct.mrg_a = c.mrg_a ? c.mrg_a + r0 * D : nullptr;
+        ct.mrg_l = c.mrg_l ? c.mrg_l + r0 : nullptr;
+        if (int rc_ = launch_partial(cm, stream)) return rc_;
+        return launch_partial(ct, stream);
+      }
+    }
+  }
   const fb_kv* kv = c.kv;
   const int D = kv->head_dim, Hkv = kv->n_heads_kv, G = c.Hq / Hkv;
   AttnArgs a{};
@@ -744,8 +784,13 @@ int block_attn_impl(const void* q, const void* k_in, const void* v_in, int batch
   c.kv = &kv;
   c.a_out = a_in;
   c.l_out = l_in;
-  // the block is short: one split per (b, hk, row tile), no workspace needed
-  c.single_split = true;
+  // the block is short: one split per (b, hk, row tile) and no workspace,
+  // unless the caller lends one (launch_partial may then split off a short
+  // last row tile)
+  c.single_split = ws == nullptr;
+  c.ws = ws;
+  c.ws_bytes = ws_bytes;
+  c.ws_offset = ws_offset;
 
   c.num_sms = sm_count();
   c.mrg_a = mrg_a;
@@ -753,39 +798,6 @@ int block_attn_impl(const void* q, const void* k_in, const void* v_in, int batch
   c.q_cu = cu;
   c.q_total = total;
   c.kv_cu = cu;
-  // One sequence, one q head per kv head, a last 256-row tile of at most 64
-  // rows (a video block of 1560 rows: 6 full tiles and 24 rows): that tile
-  // would cost a whole tcgen05 CTA and push the grid (7 tiles x heads) into a
-  // second wave. With workspace lent by the caller (fb_step), the full tiles
-  // run on the tcgen05 kernel (one wave) and the last rows on the streaming
-  // kernel, split over the block's keys (read from L2); each part merges its
-  // own rows. (Without workspace the last rows' single split per row tile
-  // streams every key tile in turn and gains nothing: measured 106 vs 101 us.)
-  const int tail = B % kT2Rows;
-  if (ws && !cu && batch == 1 && Hq == Hkv && use_tc(dt, D, B) && B > kT2Rows && tail > 0 &&
-      tail <= 64) {
-    PartialCall ct = c;
-    const size_t eb = elem_size(dt);
-    const long long r0 = (long long)(B - tail) * Hq;  // first (row, head) of the last rows
-    ct.q = static_cast<const char*>(q) + r0 * D * eb;
-    ct.B = tail;
-    ct.a_out = a_in + r0 * D;
-    ct.l_out = l_in + r0;
-    ct.mrg_a = mrg_a ? mrg_a + r0 * D : nullptr;
-    ct.mrg_l = mrg_l ? mrg_l + r0 : nullptr;
-    // the tail's split partials must fit the region the caller lent
-    const Plan pt = make_plan(dt, 1, Hkv, tail, ceil_div(B, kTK), c.num_sms, D);
-    const size_t need = partial_bytes(pt, 1, Hkv, tail, D);
-    ct.single_split = false;
-    ct.ws = ws;
-    ct.ws_bytes = ws_bytes;
-    ct.ws_offset = ws_offset;
-    if (aligned16(ct.q) && aligned16(ws) && ws_offset + need <= ws_bytes) {
-      c.B = B - tail;
-      if ((rc = launch_partial(c, stream))) return rc;
-      return launch_partial(ct, stream);
-    }
-  }
   return launch_partial(c, stream);
 }
 

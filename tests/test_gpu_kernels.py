@@ -67,6 +67,13 @@ PREFIX_CASES = {
     # more groups than CTAs, each a few tiles
     "many_groups": ("gqa", dict(prefix_min=64, prefix_max=500, batch=40, block=8,
                                 n_heads_q=16, n_heads_kv=8)),
+    # one sequence with a short last 256-row tile: full tiles on the tcgen05
+    # kernel, the last rows (44; 24 stacked = 6 block rows x G 4) on the
+    # streaming kernel
+    "video_short_last_tile": ("video", dict(prefix_min=1300, prefix_max=1300, block=300,
+                                            n_heads_q=2, n_heads_kv=2)),
+    "gqa_one_seq_short_last_tile": ("gqa", dict(prefix_min=900, prefix_max=900, batch=1,
+                                                block=70, n_heads_q=8, n_heads_kv=2)),
 }
 
 
