@@ -223,6 +223,33 @@ def test_workspace_size_covers_the_split_partials_of_a_dllm_prefix(lib):
     assert ws_losa >= ws + 4 * 32 * (32768 // 16) * 4
 
 
+def test_page_score_offset_lies_inside_the_losa_workspace(lib):
+    # the page scores sit after the split partials, 256-byte aligned, with room
+    # for one float32 per (active row, q head, logical page) before the end
+    kv = make_kv(n_heads_kv=32, max_seq_len=32768, n_slots=32768)
+    args = (ctypes.byref(kv), 32, 32, 4, 256, 148)
+    off = lib.fb_workspace_page_scores(*args)
+    total = lib.fb_workspace_size(*args)
+    assert off > 0 and off % 256 == 0
+    assert off >= 9 * 32 * 32 * 128 * 4                   # after the nine-way split partials
+    assert off + 4 * 32 * (32768 // 16) * 4 <= total
+    # n_active caps at the block rows; a paged cache counts its page-table width
+    paged = make_kv(page_table=3 << 20,
+                    max_pages_per_seq=10, max_seq_len=160, n_slots=160)
+    pargs = (ctypes.byref(paged), 4, 4, 9, 3, 148)
+    off = lib.fb_workspace_page_scores(*pargs)
+    assert off > 0 and off + 4 * 4 * 10 * 4 <= lib.fb_workspace_size(*pargs)
+
+
+def test_page_score_offset_is_zero_without_a_selection_or_for_bad_shapes(lib):
+    kv = make_kv()
+    assert lib.fb_workspace_page_scores(ctypes.byref(kv), 4, 4, 0, 4, 148) == 0
+    assert lib.fb_workspace_page_scores(ctypes.byref(kv), 4, 4, 4, 0, 148) == 0
+    assert lib.fb_workspace_page_scores(ctypes.byref(kv), 4, 3, 4, 4, 148) == 0  # Hq % Hkv
+    bad = make_kv(head_dim=96)
+    assert lib.fb_workspace_page_scores(ctypes.byref(bad), 4, 4, 4, 4, 148) == 0
+
+
 def test_step_binding_rejects_too_few_update_counts():
     # the library reads m_updated[b] for every sequence b: a short host array is
     # refused before any pointer is taken
