@@ -114,6 +114,40 @@ def test_page_size_one_gives_exact_top_k_keys():
         assert set(top.tolist()) == set(np.argsort(-exact[r])[:10].tolist())
 
 
+def test_page_score_hand_worked():
+    # q = (1, -2). Page 0, kmin = (0, -1), kmax = (3, 1): channel 0 takes q * kmax
+    # = 3, channel 1 takes q * kmin = 2, so the bound is 5. Page 1 has kmin = kmax
+    # = (0.5, 0.25), so the bound is q.k itself: 0.5 - 0.5 = 0.
+    q = np.array([[1.0, -2.0]], dtype=np.float32)
+    smin = np.array([[0.0, -1.0], [0.5, 0.25]], dtype=np.float32)
+    smax = np.array([[3.0, 1.0], [0.5, 0.25]], dtype=np.float32)
+    np.testing.assert_array_equal(losa.page_scores(q, smin, smax), [[5.0, 0.0]])
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_select_pages_breaks_ties_by_the_lower_logical_page(paged):
+    """Logical pages score (0.5, 2, 0.5, 2) for q = (1, 0): top-1 is page 1 (not
+    3), top-3 adds page 0 (not 2). With the pool stored in reverse page order,
+    the tie still goes to the lower logical page, not the lower pool page."""
+    from workloads.gen import Prefix
+    low = [[0.0, 0.0], [0.5, 0.0]]
+    high = [[1.0, 0.0], [2.0, 0.0]]
+    logical = [low, high, low, high]
+    table = np.array([[3, 2, 1, 0]], dtype=np.int32) if paged else None
+    store = [None] * 4
+    for p in range(4):
+        store[table[0, p] if paged else p] = logical[p]
+    k = np.array(store, dtype=np.float32).reshape(8, 1, 2)
+    kv = Prefix(k, k.copy(), np.array([8], dtype=np.int32), table, 2, 8)
+    smin, smax = losa.page_summary(kv, "f32")
+    q = np.array([1.0, 0.0], dtype=np.float32).reshape(1, 1, 1, 2)
+    act = np.array([[0]])
+    for topk, want in ((1, [1]), (2, [1, 3]), (3, [1, 3, 0]), (4, [1, 3, 0, 2])):
+        chosen, union = losa.select_pages(kv, q, "f32", act, topk, smin, smax)
+        np.testing.assert_array_equal(chosen[(0, 0, 0)], want)
+        np.testing.assert_array_equal(union[(0, 0)], sorted(want))
+
+
 def test_union_size_bounds_and_bitmap():
     wl = _small(prefix_min=1000, prefix_max=1000, block=16)
     smin, smax = losa.page_summary(wl.prefix, "bf16")
